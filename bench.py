@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant KV-cache hot path on B200.
+
+One step is one decode step of a Llama-3.3-70B-shaped model over a packed
+cache: for each of 80 layers, append the new token's K/V (tq_quantize, 16
+sequences x 8 kv heads) and attend (tq_attend, 64 query heads, context
+32768 + 1, K at 3-bit + QJL, V at 4 bits). Value = packed-KV bytes read per
+step / step time (GB/s). The cache is 45 GB, far larger than L2, so no flush
+is needed between steps.
+
+Also reported on the same line: the attention kernels' roofline (measured
+copy-kernel and MEASURED_PEAKS.json HBM peaks), tq_quantize throughput on a
+bulk prefill, an end-to-end figure through host buffers, GPU clocks during
+the timed region, and the fp64 CPU oracle timed on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
+Multi-GPU runs (torchrun, one rank per GPU) are weak scaling: every rank runs
+its own copy of the workload; no collective touches the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tq_attend packed-KV GB/s and % of HBM peak; tq_quantize Mtokens/s"
+DEFAULT_WORKLOAD = "llama3.3-70b_decode_32k"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--layers", type=int, default=None, help="override layer count (development)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- plumbing
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(self.local_rank)
+        if self.world > 1:
+            from datetime import timedelta
+            dist.init_process_group(backend, timeout=timedelta(seconds=600),
+                                    device_id=torch.device("cuda", self.local_rank))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j.get("hbm_gbs"), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def cpu_oracle_sample(w, seconds: float, streams: int = 4, N: int | None = None):
+    """Time the fp64 oracle's decode attention on `streams` (batch, kv-head)
+    streams of the workload (all their query heads, full context), repeated
+    until about `seconds` of work. Returns (GB/s, description, threads)."""
+    import numpy as np
+    import torch
+    from kv_cache_vector_04_b200 import inputs
+    from oracle import oracle as O
+
+    N = w.N if N is None else N
+    tab = O.Tables(w.d, w.bits, 1)
+    g = w.Hq // w.Hkv
+    k, v = inputs.kv_pair(w, N, layer=0, device="cpu", B=1, Hkv=streams)
+    codes = [[O.quantize(tab, k[0, h].numpy(), v[0, h].numpy()) for h in range(streams)]]
+    cap = N
+    st = {}
+    for key in ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm"):
+        st[key] = np.stack([c[key] for c in codes[0]])[None]
+    q = inputs.queries(w, B=1, Hq=streams * g)
+    qb = q.contiguous().view(torch.int16).numpy().view(np.uint16)
+    seq = np.array([N], np.int32)
+    reps, t_total = 0, 0.0
+    while t_total < seconds or reps == 0:
+        t0 = time.perf_counter()
+        O.attend_batch(tab, qb, w.q_dtype == torch.bfloat16, st, seq, streams)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    bytes_per_rep = streams * N * (w.bits * w.d // 4 + 6)
+    gbs = bytes_per_rep * reps / t_total / 1e9
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = ("fp64 C oracle decode attention over %d (batch, kv-head) streams x %d query heads x "
+            "%d tokens of layer 0, %d repetitions in %.1f s (append of one token excluded: "
+            "<0.01%% of the step)" % (streams, g, N, reps, t_total))
+    return gbs, desc, threads, t_total / reps
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_tq(args, dist: Dist):
+    import torch
+    import kv_cache_vector_04_b200 as tq
+    from kv_cache_vector_04_b200 import inputs
+
+    w = inputs.WORKLOADS[args.workload]
+    layers = args.layers or w.layers
+    dev = torch.device("cuda", dist.local_rank)
+    ctx = tq.tq_init(w.d, w.bits, 1)
+    lay = tq.tq_cache_layout(ctx)
+    per_tok = lay["tile_bytes"] // 16                     # K + V bytes per head-token
+    N = w.N
+    cap = N + 16
+    zeros = torch.zeros(w.B, dtype=torch.int32, device=dev)
+
+    # ---- prefill: quantize every layer's cache (inputs drawn on the device)
+    caches = []
+    q_tput = None
+    for L in range(layers):
+        k, v = inputs.kv_pair(w, N, layer=L, device=dev)
+        cache = tq.new_cache(ctx, w.B, w.Hkv, cap, device=dev)
+        if L == 0:
+            # bulk tq_quantize throughput, timed on this layer's prefill
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for _ in range(2):
+                tq.tq_quantize(ctx, k, v, zeros, cache)
+            torch.cuda.synchronize()
+            reps = 5
+            s.record()
+            for _ in range(reps):
+                tq.tq_quantize(ctx, k, v, zeros, cache)
+            e.record()
+            torch.cuda.synchronize()
+            t = s.elapsed_time(e) / 1e3 / reps
+            toks = w.B * w.Hkv * N
+            q_bytes = toks * (2 * w.d * 2 + per_tok)
+            q_tput = {"metric": "tq_quantize Mtokens/s (bulk prefill; token = one K+V head-vector pair)",
+                      "value": round(toks / t / 1e6, 2), "unit": "Mtokens/s",
+                      "workload": "one layer: %d seq x %d kv heads x %d tokens" % (w.B, w.Hkv, N),
+                      "ms_per_launch": round(t * 1e3, 4),
+                      "Mkeys_per_s": round(toks / t / 1e6, 2),
+                      "hbm_gbs": round(q_bytes / t / 1e9, 1)}
+        else:
+            tq.tq_quantize(ctx, k, v, zeros, cache)
+        caches.append(cache)
+        del k, v
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()      # release the prefill's generator temporaries
+    assert tq.tq_status(ctx) == 0
+
+    # ---- decode-step inputs (one new token per sequence and layer)
+    qs = [inputs.queries(w, layer=L, device=dev) for L in range(layers)]
+    news = [inputs.kv_pair(w, 1, layer=10_000 + L, device=dev) for L in range(layers)]
+    start = torch.full((w.B,), N, dtype=torch.int32, device=dev)
+    seq = torch.full((w.B,), N + 1, dtype=torch.int32, device=dev)
+    ws = tq.new_workspace(ctx, w.B, w.Hq, w.Hkv, N + 1)
+    outs = [torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev) for _ in range(layers)]
+    launches_per_step = layers * (1 + 3)
+
+    def step(events=None):
+        for L in range(layers):
+            nk, nv = news[L]
+            tq.tq_quantize(ctx, nk, nv, start, caches[L])
+            if events is not None:
+                events[L][0].record()
+            tq.tq_attend(ctx, qs[L], caches[L], seq, N + 1, out=outs[L], workspace=ws)
+            if events is not None:
+                events[L][1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- copy-kernel HBM peak in the same process (1 GiB -> 1 GiB)
+    src = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    for _ in range(3):
+        tq.tq_copy(src, dst)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(10):
+        tq.tq_copy(src, dst)
+    e.record()
+    torch.cuda.synchronize()
+    copy_gbs = 2 * (1 << 30) * 10 / (s.elapsed_time(e) / 1e3) / 1e9
+    del src, dst
+
+    # ---- timed region
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(vis.split(",")[dist.local_rank] if vis else dist.local_rank)
+    clocks.start()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(layers)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for k_ in range(args.steps):
+        step(ev[k_])
+    t_end.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    attend_ms = statistics.mean(a.elapsed_time(b) for row in ev for (a, b) in row)
+    ms = dist.max(ms)
+    assert tq.tq_status(ctx) == 0
+
+    bytes_step = layers * w.B * w.Hkv * (N + 1) * per_tok
+    bytes_attend = w.B * w.Hkv * (N + 1) * per_tok
+    total_bytes = dist.sum(bytes_step)
+    value = total_bytes / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_attend / (attend_ms / 1e3) / 1e9
+
+    # ---- end to end through host buffers: q, new K/V from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        q_host = [q.cpu().pin_memory() for q in qs]
+        k_host = [(a.cpu().pin_memory(), b.cpu().pin_memory()) for a, b in news]
+        out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        q_dev = [torch.empty_like(q) for q in qs[:1]]
+        kv_dev = [(torch.empty_like(a), torch.empty_like(b)) for a, b in news[:1]]
+
+        def host_step():
+            for L in range(layers):
+                kv_dev[0][0].copy_(k_host[L][0], non_blocking=True)
+                kv_dev[0][1].copy_(k_host[L][1], non_blocking=True)
+                tq.tq_quantize(ctx, kv_dev[0][0], kv_dev[0][1], start, caches[L])
+                tq.attend_host(ctx, q_host[L], caches[L], seq, N + 1, out_host[L], ws,
+                               q_dev[0], outs[L])
+
+        for _ in range(max(args.warmup, 3)):
+            host_step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        s.record()
+        for _ in range(args.steps):
+            host_step()
+        e.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        e2e_ms = dist.max(s.elapsed_time(e) / args.steps)
+        h2d = layers * (qs[0].numel() * qs[0].element_size() +
+                        2 * news[0][0].numel() * news[0][0].element_size())
+        d2h = layers * outs[0].numel() * outs[0].element_size()
+        e2e = {"value": round(total_bytes / (e2e_ms / 1e3) / 1e9, 1), "unit": "GB/s",
+               "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 tensor-core operands, f32 accumulate (codes u2-u4)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "layers": layers, "batch": w.B, "q_heads": w.Hq,
+                   "kv_heads": w.Hkv, "head_dim": w.d, "bits": w.bits, "context": N + 1,
+                   "packed_cache_gb": round(layers * w.B * w.Hkv * cap * per_tok / 1e9, 2),
+                   "step": "per layer: tq_quantize (append 1 token) + tq_attend",
+                   "l2": "inputs larger than L2 (%.0f MB per layer)" % (bytes_attend / 1e6),
+                   "parallelism": "replicas x%d (weak)" % dist.world},
+        "pct_of_hbm_peak": round(100.0 * value / dist.world / peak, 1),
+        "roofline": {"bound": "hbm", "kernel": "tq_attend (prologue + split + reduce launches)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
+                     "traffic": None,
+                     "algorithmic_bytes_per_launch": bytes_attend,
+                     "frac_of_same_run_copy_kernel": round(achieved / copy_gbs, 3)},
+        "copy_kernel_gbs": round(copy_gbs, 1),
+        "quantize": q_tput,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        gbs, desc, threads, _ = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
+                                "kind": "oracle", "sample": desc}
+    for L in range(layers):
+        caches[L] = None
+    return line
+
+
+def run_reference(args, dist: Dist):
+    """The fp64 CPU oracle as the reference arm: each step is a bounded sample
+    (2 streams of the workload) of oracle decode attention."""
+    import torch
+    from kv_cache_vector_04_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    if dist.rank != 0:
+        return None
+    times = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        gbs, desc, threads, t = cpu_oracle_sample(w, 0.0, streams=2)
+        if i >= args.warmup:
+            times.append(gbs)
+    value = statistics.mean(times)
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv,
+                       "head_dim": w.d, "bits": w.bits, "context": w.N},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        # the oracle runs on the host; only rank 0 works, the others exit cleanly
+        line = run_reference(args, dist)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    dist.init()
+    try:
+        line = run_tq(args, dist)
+        if dist.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,524 @@
+// tq_attend / tq_scores: split-K flash decoding straight from the packed cache.
+//
+// The logit of query head h against cached token n is the QJL-corrected
+// estimate ("[Benchmark] TurboQuant 實測：KV Cache 3-bit 壓縮，真的零損失？",
+// ai-muninn.com, §"TurboQuant 是什麼：30 秒懶人包": the QJL step makes the
+// attention score unbiased):
+//   l_n = |k_n| (<q~, cK[idx_n]> + rho_n sqrt(pi/2)/m <S q~, 2 s_n - 1>) / sqrt(d),
+// with q~ = Pi q; values stay in the rotated domain and are rotated back once
+// per output: o = Pi^T sum_n softmax(l)_n |v_n| cV[vidx_n].
+//
+// Three kernels:
+//  prologue  q~ = H (D o q) / sqrt(d) and p = S q~ per query head, written as
+//            fp16 m16n8k16 B fragments (log2(e) and the norms' scales folded in);
+//  split     one CTA per (batch, kv head, group of 8 query heads, context
+//            split); each warp streams 16-token tiles with 128-bit loads of its
+//            own lane string, decodes codes to fp16 tensor-core A fragments
+//            through a lane-replicated shared-memory table (2 ALU ops + 1 LDS
+//            per fp16x2) and sign pairs with 2 ALU ops, and runs
+//              logits: [16 tok x d] x [d x 8 heads]  (codebook term)
+//                      [16 tok x m] x [m x 8 heads]  (QJL sign term)
+//              PV:     [d x 16 tok] x [16 tok x 8 heads]
+//            on mma.sync with fp32 accumulation, with an online softmax per
+//            head in registers; the 4 warps of a CTA merge in shared memory;
+//  reduce    merges the splits per query head and applies Pi^T (fp32 WHT).
+// Operands come from registers because every A fragment is decoded on the
+// fly; the contraction is skinny (N = 8 heads), so the legacy register-fed
+// MMA fits better here than shared-memory/TMEM-fed tcgen05 tiles.
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace tq {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D, int BITS>
+struct AttTraits {
+    static constexpr int BK = BITS - 1, BV = BITS;
+    static constexpr int KF = 2 * BK, VF = 2 * BV;          // field widths
+    static constexpr int LW = BITS * D / 32;                 // words per lane string
+    static constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;
+    static constexpr int CW = CB / 4;
+    static constexpr int SBW = BK * D / 64;                  // first sign word
+    static constexpr int VB = (BK + 1) * D / 2;              // first value bit
+    static constexpr int KK = D / 16;                        // k-steps / coordinate blocks
+    static constexpr int NLK = 1 << KF, NLV = 1 << VF;       // LUT entries
+    static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
+    static constexpr size_t MERGE_BYTES = (size_t)4 * 8 * (D + 2) * 4;
+    static constexpr size_t DYN_SMEM = QF_BYTES > MERGE_BYTES ? QF_BYTES : MERGE_BYTES;
+};
+
+// Row offset (field value * 128) of an F-bit field starting at bit `pos` of the
+// lane string, OR-ed with `lane_bits` (lane * 4 plus the table base, which is
+// aligned to the table size): a lane-replicated table address in one funnel
+// (or plain) shift and one LOP3.
+__device__ __forceinline__ uint32_t lut_addr(const uint32_t* s, int pos, int F, uint32_t lane_bits)
+{
+    const int wi = pos >> 5, o = pos & 31;
+    const uint32_t mask = ((1u << F) - 1u) << 7;
+    uint32_t v;
+    if (o + F <= 32)
+        v = (o >= 7) ? (s[wi] >> (o - 7)) : (s[wi] << (7 - o));
+    else
+        v = __funnelshift_r(s[wi], s[wi + 1], o - 7);
+    return (v & mask) | lane_bits;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t shared_addr)
+{
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(shared_addr));
+    return v;
+}
+
+// fp16x2 (+1/-1, +1/-1) from sign pair p: element 0 at bit p%16, element 1 at
+// bit 16 + p%16 of sign word p/16 (bit 1 = +1).
+__device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q)
+{
+    const uint32_t x = word << (15 - q);
+    return (x & 0x80008000u) ^ 0xBC00BC00u;
+}
+
+// ---------------------------------------------------------------- prologue
+// Per query head: q~ = H (D o q) / sqrt(d), p = S q~, and the fp16 B fragments
+// of [log2(e) 2^7 q~ / (d alpha)] and [log2(e) 2^7 kappa p / sqrt(d)], each as
+// a hi part and a lo part (x - hi), so that the two tensor-core products
+// carry ~22 significant bits. alpha is the scale that makes the key codebook
+// almost exact in fp16 (chosen on the host).
+template <int D>
+__global__ void __launch_bounds__(D) attend_prologue(DevTables tb, AttendArgs a)
+{
+    __shared__ float qs[D];
+    __shared__ float bc[D], bs[D];
+    const int b = blockIdx.y;
+    const int unit = blockIdx.x >> 3, col = blockIdx.x & 7;
+    const int groups = a.plan.groups;
+    const int ratio = a.Hq / a.Hkv;
+    const int hkv = unit / groups, grp = unit % groups;
+    const int j = grp * 8 + col;
+    const int i = threadIdx.x;
+    const bool live = j < ratio;   // block-uniform
+    float vc = 0.f, vs = 0.f;
+    if (live) {
+        const int hq = hkv * ratio + j;
+        const size_t off = ((size_t)b * a.Hq + hq) * D + i;
+        float x;
+        if (a.q_bf16)
+            x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[off]);
+        else
+            x = __half2float(reinterpret_cast<const __half*>(a.q)[off]);
+        qs[i] = x * tb.signs[i];
+        __syncthreads();
+#pragma unroll
+        for (int s = 1; s < D; s <<= 1) {
+            const float mine = qs[i], other = qs[i ^ s];
+            __syncthreads();
+            qs[i] = (i & s) ? (other - mine) : (mine + other);
+            __syncthreads();
+        }
+        const float qt = qs[i] * rsqrtf((float)D);
+        __syncthreads();
+        qs[i] = qt;
+        __syncthreads();
+        float p = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) p = fmaf(tb.s_t[(size_t)k * D + i], qs[k], p);
+        vc = qt * (kLog2e * 128.0f / ((float)D * tb.alpha_k));
+        vs = p * (kLog2e * 128.0f * 1.2533141373155003f / ((float)D * sqrtf((float)D)));
+    }
+    bc[i] = vc;
+    bs[i] = vs;
+    __syncthreads();
+    if (i < D / 4) {
+        const int kk = i >> 2, t = i & 3;
+        const int c0 = 16 * kk + 2 * t;
+        const int idx[4] = {c0, c0 + 1, c0 + 8, c0 + 9};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const float* src = q ? bs : bc;
+            float h[4], l[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                h[e] = __half2float(__float2half_rn(src[idx[e]]));
+                l[e] = src[idx[e]] - h[e];
+            }
+            hi[2 * q] = pack_half2(h[0], h[1]);
+            hi[2 * q + 1] = pack_half2(h[2], h[3]);
+            lo[2 * q] = pack_half2(l[0], l[1]);
+            lo[2 * q + 1] = pack_half2(l[2], l[3]);
+        }
+        const size_t units = (size_t)a.Hkv * groups;
+        uint4* dst = reinterpret_cast<uint4*>(a.qfrag) +
+                     ((((size_t)b * units + unit) * (D / 16) + kk) * 32 + col * 4 + t) * 2;
+        dst[0] = make_uint4(hi[0], hi[1], lo[0], lo[1]);   // codebook term: b0,b1 hi; b0,b1 lo
+        dst[1] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
+    }
+}
+
+// ---------------------------------------------------------------- split kernel
+template <int D, int BITS, int CW>
+__device__ __forceinline__ void load_tile(const uint8_t* tp, int lane, int g, uint32_t (&s)[BITS * D / 32],
+                                          uint2& kn, uint32_t& vn)
+{
+    constexpr int CB = CW * 4, NCH = BITS * D / 8 / CB;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        const uint8_t* src = tp + ((size_t)c * 32 + lane) * CB;
+        if constexpr (CW == 4) {
+            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src));
+            s[4 * c] = v.x; s[4 * c + 1] = v.y; s[4 * c + 2] = v.z; s[4 * c + 3] = v.w;
+        } else {
+            const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src));
+            s[2 * c] = v.x; s[2 * c + 1] = v.y;
+        }
+    }
+    kn = __ldcs(reinterpret_cast<const uint2*>(tp + 4 * BITS * D + 8 * g));
+    vn = __ldcs(reinterpret_cast<const uint32_t*>(tp + 4 * BITS * D + 64 + 4 * g));
+}
+
+template <int D, int BITS, bool SCORES>
+__global__ void __launch_bounds__(128) attend_split(DevTables tb, AttendArgs a)
+{
+    using Tr = AttTraits<D, BITS>;
+    constexpr int KK = Tr::KK, LW = Tr::LW;
+    // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l. Each
+    // table is aligned to its size so that a table address is (field*128) | (4l + base).
+    __shared__ __align__(Tr::NLV * 128) uint32_t lutv[Tr::NLV * 32];
+    __shared__ __align__(Tr::NLK * 128) uint32_t lutk[Tr::NLK * 32];
+    extern __shared__ uint4 dyn_smem[];
+    uint4* qf = dyn_smem;                                  // [KK][32][2] during the tile loop
+    float* mrg = reinterpret_cast<float*>(dyn_smem);       // [4][8][D+2] after it
+
+    const int split = blockIdx.x, unit = blockIdx.y, b = blockIdx.z;
+    const int groups = a.plan.groups;
+    const int hkv = unit / groups, grp = unit % groups;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const size_t units = (size_t)a.Hkv * groups;
+
+    for (int e = tid; e < Tr::NLK * 32; e += 128) lutk[e] = __ldg(tb.lut_k + (e >> 5));
+    for (int e = tid; e < Tr::NLV * 32; e += 128) lutv[e] = __ldg(tb.lut_v + (e >> 5));
+    const uint4* qsrc = reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64;
+    for (int e = tid; e < KK * 64; e += 128) qf[e] = qsrc[e];
+
+    int seq = a.seq_len[b];
+    const int lim = min(a.max_len, a.capacity);
+    if (seq < 0 || seq > lim) {
+        if (tid == 0 && split == 0 && unit == 0) atomicOr(tb.status, TQ_STATUS_SEQ_LEN);
+        seq = min(max(seq, 0), lim);
+    }
+    __syncthreads();
+
+    const int ntiles = SCORES ? a.plan.tiles : (seq + 15) >> 4;
+    const int t_begin = split * a.plan.tps;
+    const int t_end = min(t_begin + a.plan.tps, ntiles);
+    const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
+                                         (size_t)a.tile_bytes;
+    const uint32_t lk_bits = (uint32_t)__cvta_generic_to_shared(lutk) + 4u * lane;
+    const uint32_t lv_bits = (uint32_t)__cvta_generic_to_shared(lutv) + 4u * lane;
+    const int ratio = a.Hq / a.Hkv;
+
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+    float acc[KK][4];
+#pragma unroll
+    for (int kk = 0; kk < KK; ++kk) acc[kk][0] = acc[kk][1] = acc[kk][2] = acc[kk][3] = 0.f;
+
+    // software pipeline: the next tile's lane string is in flight while this one is decoded
+    uint32_t nxt[LW];
+    uint2 kn_n = make_uint2(0u, 0u);
+    uint32_t vn_n = 0u;
+    int tl = t_begin + w;
+    const bool skip_decode_past = SCORES;   // scores: tiles past seq need no decode
+    if (tl < t_end && !(skip_decode_past && tl * 16 >= seq))
+        load_tile<D, BITS, Tr::CW>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, nxt, kn_n, vn_n);
+
+#pragma unroll 1
+    for (; tl < t_end; tl += 4) {
+        const int pos0 = tl * 16 + g, pos1 = pos0 + 8;
+        if (SCORES && tl * 16 >= seq) {
+            const int j0 = grp * 8 + 2 * t;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                if (j0 + hh >= ratio) continue;
+                float* row = a.out + ((size_t)b * a.Hq + hkv * ratio + j0 + hh) * a.max_len;
+                if (pos0 < a.max_len) row[pos0] = -CUDART_INF_F;
+                if (pos1 < a.max_len) row[pos1] = -CUDART_INF_F;
+            }
+            continue;
+        }
+        uint32_t s[LW];
+#pragma unroll
+        for (int i = 0; i < LW; ++i) s[i] = nxt[i];
+        const uint2 kn = kn_n;
+        const uint32_t vn = vn_n;
+        const int tn = tl + 4;
+        if (tn < t_end && !(skip_decode_past && tn * 16 >= seq))
+            load_tile<D, BITS, Tr::CW>(sbase + (size_t)tn * (size_t)a.tile_bytes, lane, g, nxt, kn_n, vn_n);
+
+        float cc[4] = {0.f, 0.f, 0.f, 0.f}, cs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+            const uint4 bc = qf[(kk * 32 + lane) * 2];
+            const uint4 bs = qf[(kk * 32 + lane) * 2 + 1];
+            uint32_t ak[4], as[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int p = 4 * kk + r;
+                ak[r] = lds32(lut_addr(s, Tr::KF * p, Tr::KF, lk_bits));
+                as[r] = sign_pair(s[Tr::SBW + (p >> 4)], p & 15);
+            }
+            mma_16816(cc, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
+            mma_16816(cc, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+            mma_16816(cs, as[0], as[1], as[2], as[3], bs.x, bs.y);
+            mma_16816(cs, as[0], as[1], as[2], as[3], bs.z, bs.w);
+        }
+        const float kn_g = half_bits_to_float((uint16_t)(kn.x & 0xffff));
+        const float rho_g = half_bits_to_float((uint16_t)(kn.x >> 16));
+        const float kn_h = half_bits_to_float((uint16_t)(kn.y & 0xffff));
+        const float rho_h = half_bits_to_float((uint16_t)(kn.y >> 16));
+        // the B operands carry a factor 2^7
+        float L0 = (kn_g * (1.0f / 128.0f)) * fmaf(rho_g, cs[0], cc[0]);
+        float L1 = (kn_g * (1.0f / 128.0f)) * fmaf(rho_g, cs[1], cc[1]);
+        float L2 = (kn_h * (1.0f / 128.0f)) * fmaf(rho_h, cs[2], cc[2]);
+        float L3 = (kn_h * (1.0f / 128.0f)) * fmaf(rho_h, cs[3], cc[3]);
+        if (pos0 >= seq) L0 = L1 = -CUDART_INF_F;
+        if (pos1 >= seq) L2 = L3 = -CUDART_INF_F;
+
+        if constexpr (SCORES) {
+            const int j0 = grp * 8 + 2 * t;
+            const float L[4] = {L0, L1, L2, L3};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                if (j0 + hh >= ratio) continue;
+                float* row = a.out + ((size_t)b * a.Hq + hkv * ratio + j0 + hh) * a.max_len;
+                if (pos0 < a.max_len) row[pos0] = L[hh] * kLn2;
+                if (pos1 < a.max_len) row[pos1] = L[2 + hh] * kLn2;
+            }
+            continue;
+        } else {
+            float mx0 = fmaxf(L0, L2), mx1 = fmaxf(L1, L3);
+#pragma unroll
+            for (int sh = 4; sh <= 16; sh <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
+            }
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            if (__any_sync(kFull, mn0 != m0 || mn1 != m1)) {   // rescale only when a max moved
+                const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+                l0 *= al0;
+                l1 *= al1;
+#pragma unroll
+                for (int kk = 0; kk < KK; ++kk) {
+                    acc[kk][0] *= al0;
+                    acc[kk][1] *= al1;
+                    acc[kk][2] *= al0;
+                    acc[kk][3] *= al1;
+                }
+                m0 = mn0;
+                m1 = mn1;
+            }
+            const float p0 = exp2f(L0 - m0), p1 = exp2f(L1 - m1);
+            const float p2 = exp2f(L2 - m0), p3 = exp2f(L3 - m1);
+            l0 += p0 + p2;
+            l1 += p1 + p3;
+            // slots past seq_len may hold anything (even NaN norms): select, never multiply
+            const float vn_g = pos0 < seq ? half_bits_to_float((uint16_t)(vn & 0xffff)) : 0.f;
+            const float vn_h = pos1 < seq ? half_bits_to_float((uint16_t)(vn >> 16)) : 0.f;
+            const uint32_t b0 = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
+            const uint32_t b1 = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
+#pragma unroll
+            for (int kk = 0; kk < KK; ++kk) {
+                uint32_t av[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    av[r] = lds32(lut_addr(s, Tr::VB + Tr::VF * (4 * kk + r), Tr::VF, lv_bits));
+                mma_16816(acc[kk], av[0], av[1], av[2], av[3], b0, b1);
+            }
+        }
+    }
+    if constexpr (!SCORES) {
+#pragma unroll
+        for (int sh = 4; sh <= 16; sh <<= 1) {
+            l0 += __shfl_xor_sync(kFull, l0, sh);
+            l1 += __shfl_xor_sync(kFull, l1, sh);
+        }
+        __syncthreads();   // every warp is done with qf: reuse it for the merge
+        constexpr int RS = D + 2;
+        float* mw = mrg + (size_t)w * 8 * RS;
+        if (g == 0) {
+            mw[(2 * t) * RS] = m0;
+            mw[(2 * t) * RS + 1] = l0;
+            mw[(2 * t + 1) * RS] = m1;
+            mw[(2 * t + 1) * RS + 1] = l1;
+        }
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+            mw[(2 * t) * RS + 2 + 16 * kk + g] = acc[kk][0];
+            mw[(2 * t + 1) * RS + 2 + 16 * kk + g] = acc[kk][1];
+            mw[(2 * t) * RS + 2 + 16 * kk + g + 8] = acc[kk][2];
+            mw[(2 * t + 1) * RS + 2 + 16 * kk + g + 8] = acc[kk][3];
+        }
+        __syncthreads();
+        float* dst = a.partial + (((size_t)b * units + unit) * a.plan.nsplit + split) * 8 * RS;
+        for (int e = tid; e < 8 * RS; e += 128) {
+            const int head = e / RS, c = e % RS;
+            float M = -CUDART_INF_F;
+#pragma unroll
+            for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, mrg[(ww * 8 + head) * RS]);
+            float sum = 0.f;
+            if (c == 0) {
+                sum = M;
+            } else {
+#pragma unroll
+                for (int ww = 0; ww < 4; ++ww) {
+                    const float mwv = mrg[(ww * 8 + head) * RS];
+                    if (mwv != -CUDART_INF_F) sum += mrg[(ww * 8 + head) * RS + c] * exp2f(mwv - M);
+                }
+            }
+            dst[e] = sum;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- reduction
+template <int D>
+__global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
+{
+    __shared__ float os[D];
+    const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+    const int ratio = a.Hq / a.Hkv, groups = a.plan.groups;
+    const int hkv = hq / ratio, j = hq % ratio, grp = j >> 3, col = j & 7;
+    const size_t units = (size_t)a.Hkv * groups;
+    const size_t unit = (size_t)hkv * groups + grp;
+    constexpr int RS = D + 2;
+    const float* P = a.partial + ((size_t)b * units + unit) * a.plan.nsplit * 8 * RS + col * RS;
+    const int ns = a.plan.nsplit;
+    float M = -CUDART_INF_F;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, P[(size_t)s * 8 * RS]);
+    float L = 0.f, acc = 0.f;
+    if (M != -CUDART_INF_F) {
+        for (int s = 0; s < ns; ++s) {
+            const float* ps = P + (size_t)s * 8 * RS;
+            const float ms = ps[0];
+            if (ms == -CUDART_INF_F) continue;
+            const float f = exp2f(ms - M);
+            L = fmaf(ps[1], f, L);
+            acc = fmaf(ps[2 + i], f, acc);
+        }
+    }
+    os[i] = (L > 0.f) ? acc / L : 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int s = 1; s < D; s <<= 1) {
+        const float mine = os[i], other = os[i ^ s];
+        __syncthreads();
+        os[i] = (i & s) ? (other - mine) : (mine + other);
+        __syncthreads();
+    }
+    // Pi^T = D H / sqrt(d), and the value table carries a factor sqrt(d)
+    a.out[((size_t)b * a.Hq + hq) * D + i] = os[i] * tb.signs[i] * (1.0f / (float)D);
+}
+
+// cudaFuncSetAttribute once per (kernel, device).
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long& done_mask)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (__atomic_load_n(&done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) __atomic_fetch_or(&done_mask, bit, __ATOMIC_ACQ_REL);
+    return e;
+}
+
+template <int D, int BITS>
+cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool scores, cudaStream_t st)
+{
+    using Tr = AttTraits<D, BITS>;
+    static unsigned long long done_scores = 0, done_attend = 0;
+    const int units = a.Hkv * a.plan.groups;
+    attend_prologue<D><<<dim3(units * 8, a.B), D, 0, st>>>(tb, a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const dim3 grid(a.plan.nsplit, units, a.B);
+    if (scores) {
+        auto kern = attend_split<D, BITS, true>;
+        if ((e = allow_smem(kern, Tr::DYN_SMEM, done_scores)) != cudaSuccess) return e;
+        if (a.plan.tiles > 0) kern<<<grid, 128, Tr::DYN_SMEM, st>>>(tb, a);
+        return cudaGetLastError();
+    }
+    auto kern = attend_split<D, BITS, false>;
+    if ((e = allow_smem(kern, Tr::DYN_SMEM, done_attend)) != cudaSuccess) return e;
+    kern<<<grid, 128, Tr::DYN_SMEM, st>>>(tb, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attend_reduce<D><<<dim3(a.Hq, a.B), D, 0, st>>>(tb, a);
+    return cudaGetLastError();
+}
+
+__global__ void copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n)
+{
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
+}
+
+}  // namespace
+
+AttendPlan plan_attend(int d, int B, int Hq, int Hkv, int max_len, int num_sms)
+{
+    AttendPlan p{};
+    const int ratio = Hq / Hkv;
+    p.groups = (ratio + 7) / 8;
+    const long long units = (long long)B * Hkv * p.groups;
+    p.tiles = (max_len + 15) / 16;
+    const long long target = 8LL * num_sms;           // CTAs of 4 warps: ~2 waves at 4 CTAs/SM
+    long long ns = (target + units - 1) / units;
+    const long long max_ns = (p.tiles + 7) / 8;        // at least 8 tiles (2 per warp) per split
+    if (ns > max_ns) ns = max_ns;
+    if (ns < 1) ns = 1;
+    p.tps = p.tiles > 0 ? (int)((p.tiles + ns - 1) / ns) : 0;
+    p.nsplit = p.tps > 0 ? (p.tiles + p.tps - 1) / p.tps : 1;
+    p.qfrag_bytes = (size_t)units * (d / 16) * 32 * 32;
+    p.partial_bytes = (size_t)units * p.nsplit * 8 * (d + 2) * sizeof(float);
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    p.total_bytes = up(p.qfrag_bytes) + up(p.partial_bytes);
+    return p;
+}
+
+cudaError_t launch_attend(int d, int bits, const DevTables& tb, const AttendArgs& a, bool scores,
+                          cudaStream_t st)
+{
+#define TQ_A(DD, BB) \
+    if (d == DD && bits == BB) return launch_attend_t<DD, BB>(tb, a, scores, st);
+    TQ_A(64, 2) TQ_A(64, 3) TQ_A(64, 4)
+    TQ_A(128, 2) TQ_A(128, 3) TQ_A(128, 4)
+    TQ_A(256, 2) TQ_A(256, 3) TQ_A(256, 4)
+#undef TQ_A
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st)
+{
+    const size_t n = bytes / 16;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    size_t blocks = (n + 255) / 256;
+    const size_t cap = (size_t)sms * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks == 0) return cudaSuccess;
+    copy_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint4*>(src),
+                                                  reinterpret_cast<uint4*>(dst), n);
+    return cudaGetLastError();
+}
+
+}  // namespace tq

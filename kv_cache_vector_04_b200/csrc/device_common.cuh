@@ -1,0 +1,116 @@
+// Device-side helpers shared by the TurboQuant kernels (sm_100a).
+#pragma once
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// Device copies of one context's tables (all pointers into one allocation).
+struct DevTables {
+    const float* centroids_k;   // [2^BK] fp32
+    const double* bounds_k;     // [2^BK - 1] fp64 copies of the fp32 bounds
+    const double* centroids_kd; // [2^BK] fp64 copies of the fp32 centroids
+    const double* bounds_v;     // [2^BV - 1]
+    const float* signs;         // D as fp32 +-1, [d]
+    const uint2* s_frag;        // S^T as m16n8k16 B fragments: [d/16][m/8][32 lanes] (fp16 pairs)
+    const float* s_t;           // S^T fp32 [d][m]
+    const uint32_t* lut_k;      // [4^BK] fp16x2: alpha_k sqrt(d) (cK[f & (2^BK-1)], cK[f >> BK])
+    const uint32_t* lut_v;      // [4^BV] fp16x2, the same for the value codebook
+    unsigned* status;           // sticky TQ_STATUS_* bits
+    float alpha_k;              // lut_k holds alpha_k * sqrt(d) * cK (see choose_decode_scale)
+};
+
+// D = A(16x16, row) * B(16x8, col) + D with fp16 inputs and fp32 accumulation.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit values held in the m8n8 fragment layout
+// (lane 4g+t holds row g, columns 2t and 2t+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)
+{
+    uint32_t y;
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t b)
+{
+    return __half2float(__ushort_as_half(b));
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v)
+{
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(kFull, v, s);
+    return v;
+}
+
+// In-lane Walsh–Hadamard butterflies over the V consecutive coordinates a lane
+// holds (coordinate = lane * V + k), then the cross-lane stages by shuffles.
+// Sylvester (natural) order, unnormalised.
+template <int V>
+__device__ __forceinline__ void wht_warp(double (&x)[V], int lane)
+{
+#pragma unroll
+    for (int s = 1; s < V; s <<= 1) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            if (!(i & s)) {
+                const double a = x[i], b = x[i + s];
+                x[i] = a + b;
+                x[i + s] = a - b;
+            }
+        }
+    }
+#pragma unroll
+    for (int s = 1; s < 32; s <<= 1) {
+        const bool upper = (lane & s) != 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const double o = __shfl_xor_sync(kFull, x[i], s);
+            x[i] = upper ? (o - x[i]) : (x[i] + o);
+        }
+    }
+}
+
+// Cell index = number of boundaries strictly below y (binary search over the
+// 2^B - 1 sorted boundaries).
+template <int B>
+__device__ __forceinline__ int encode_cell(double y, const double* bounds)
+{
+    int idx = 0;
+#pragma unroll
+    for (int s = (1 << B) / 2; s >= 1; s >>= 1)
+        if (y > bounds[idx + s - 1]) idx += s;
+    return idx;
+}
+
+// fp16 storage of a norm: round to nearest even, saturating at 65504.
+__device__ __forceinline__ uint16_t norm_to_half_bits(double v, unsigned& sat)
+{
+    if (v > 65504.0) {
+        sat = 1u;
+        return 0x7bffu;
+    }
+    return __half_as_ushort(__double2half(v));
+}
+
+}  // namespace tq

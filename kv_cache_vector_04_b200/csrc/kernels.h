@@ -1,0 +1,50 @@
+// Launch interfaces between the host API (api.cu) and the kernels.
+#pragma once
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace tq {
+
+struct DevTables;
+
+struct QuantizeArgs {
+    const __half* k;          // [B][Hkv][T][d]
+    const __half* v;          // [B][Hkv][T][d]
+    const int32_t* start_pos; // [B]
+    uint8_t* cache;           // [B][Hkv][capacity/16][tile_bytes]
+    int B, Hkv, T, capacity;
+    long long tile_bytes;
+};
+
+// Split-K geometry of one attention call.
+struct AttendPlan {
+    int groups;     // head groups of 8 per kv head: ceil((Hq/Hkv) / 8)
+    int nsplit;     // splits of the context per (b, kv head, group)
+    int tiles;      // ceil(max_len / 16)
+    int tps;        // tiles per split
+    size_t qfrag_bytes, partial_bytes, total_bytes;
+};
+
+struct AttendArgs {
+    const void* q;            // [B][Hq][d] fp16 / bf16
+    int q_bf16;
+    const int32_t* seq_len;   // [B]
+    const uint8_t* cache;
+    int B, Hq, Hkv, capacity, max_len;
+    long long tile_bytes;
+    uint32_t* qfrag;          // workspace: [B][Hkv*groups][d/16][32][4] fp16x2 B fragments
+    float* partial;           // workspace: [B][Hkv*groups][nsplit][8][d + 2]
+    float* out;               // [B][Hq][d] (attend) or scores [B][Hq][max_len]
+    AttendPlan plan;
+};
+
+cudaError_t launch_quantize(int d, int bits, const DevTables& tb, const QuantizeArgs& a,
+                            cudaStream_t st);
+cudaError_t launch_attend(int d, int bits, const DevTables& tb, const AttendArgs& a,
+                          bool scores, cudaStream_t st);
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
+
+AttendPlan plan_attend(int d, int B, int Hq, int Hkv, int max_len, int num_sms);
+
+}  // namespace tq

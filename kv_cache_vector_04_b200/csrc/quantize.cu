@@ -1,0 +1,386 @@
+// tq_quantize: TurboQuant compression of K/V vectors into the packed cache.
+//
+// Per token and head ("[Benchmark] TurboQuant 實測：KV Cache 3-bit 壓縮，真的零損失？",
+// ai-muninn.com, §"TurboQuant 是什麼：30 秒懶人包"; "turboquant-kvquant-vllm-
+// benchmark", ai-coding.wiselychen.com, §"TurboQuant 是什麼", steps 1-3):
+//   u = x / |x|;  y = H (D o u) / sqrt(d)       random sign flip + Walsh–Hadamard
+//   idx_i = #{j : y_i > t_j}                     Lloyd–Max cell per coordinate
+//   keys:   r = y - c[idx], rho = |r|, s = [S r >= 0]   1-bit QJL residual sketch
+// then bit-packing into the tile layout of tq.h.
+//
+// One CTA of 4 warps owns one 16-token tile of one (batch, kv head):
+//  1. each warp quantizes 4 keys and 4 values; one vector is spread over the
+//     32 lanes (d/32 consecutive coordinates per lane) and rotated with an
+//     fp64 register/shuffle butterfly, so cell decisions agree with an fp64
+//     reference except within ~1e-16 of a boundary;
+//  2. z = S r for the 16 keys on the tensor cores: r is scaled by 2^12 and
+//     split into fp16 hi + lo parts (22 significant bits), S is fp16-exact by
+//     construction, products are exact and accumulate in fp32 (mma.sync
+//     m16n8k16), so only sign(z) within ~1e-7 |z| of 0 can differ from fp64;
+//  3. the 128 threads assemble the 32 lane strings of the tile from shared
+//     memory and write them with 128-bit (or 64-bit) coalesced stores, merging
+//     with the tile's previous bits when only part of it is new.
+#include <cuda_runtime.h>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace tq {
+namespace {
+
+template <int D, int BITS>
+struct QuantTraits {
+    static constexpr int BK = BITS - 1, BV = BITS, M = D;
+    static constexpr int VPL = D / 32;                 // coordinates per lane per vector
+    static constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;  // chunk bytes
+    static constexpr int NCH = BITS * D / 8 / CB;      // chunks per lane string
+    static constexpr int CW = CB / 4;                  // words per chunk
+    static constexpr int KF = 2 * BK, VF = 2 * BV;     // field widths (two codes each)
+    static constexpr int SBW = BK * D / 64;            // first sign word of a lane string
+    static constexpr int VBW = (BK + 1) * D / 64;      // first value word
+    static constexpr int NT = M / 8;                   // n-tiles of z = S r
+    static constexpr int NTW = NT / 4;                 // n-tiles per warp
+};
+
+// Place a field of up to 8 bits whose first bit sits at (signed) offset `off`
+// inside a 32-bit word.
+__device__ __forceinline__ uint32_t place(uint32_t v, int off)
+{
+    return off >= 0 ? (off < 32 ? (v << off) : 0u) : (off > -32 ? (v >> (-off)) : 0u);
+}
+
+// Shared memory of one tile (dynamic: about 59 KB at d = 256).
+template <int D>
+struct QuantSmem {
+    double rd[16][D];                 // fp64 residual r of each key, for exact near-zero signs
+    uint32_t rh[16][D / 2 + 4];       // fp16x2 hi part of 2^12 r (rows padded: no bank conflicts)
+    uint32_t rl[16][D / 2 + 4];       // fp16x2 lo part
+    uint32_t sg[16][D / 32];          // QJL sign bits, row j at bit j%32 of word j/32
+    uint8_t kc[16][D];                // key cell indices
+    uint8_t vc[16][D];                // value cell indices
+    double ck[16], tk[16], tv[16];    // key centroids, key / value boundaries (fp64 copies)
+    float rho[16];                    // |r| of each key
+    uint16_t nk[16], nr[16], nv[16];  // fp16 norms
+};
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArgs a)
+{
+    using Tr = QuantTraits<D, BITS>;
+    constexpr int BK = Tr::BK, BV = Tr::BV, M = Tr::M, VPL = Tr::VPL;
+
+    extern __shared__ __align__(16) unsigned char quant_smem_raw[];
+    QuantSmem<D>& sm = *reinterpret_cast<QuantSmem<D>*>(quant_smem_raw);
+    auto& kc = sm.kc;
+    auto& vc = sm.vc;
+    auto& rh = sm.rh;
+    auto& rl = sm.rl;
+    auto& sg = sm.sg;
+    auto& nk = sm.nk;
+    auto& nr = sm.nr;
+    auto& nv = sm.nv;
+    auto& ck_s = sm.ck;
+    auto& tk_s = sm.tk;
+    auto& tv_s = sm.tv;
+
+    const int b = blockIdx.z, h = blockIdx.y;
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int start = a.start_pos[b];
+    if (start < 0 || (long long)start + a.T > (long long)a.capacity) {
+        if (tid == 0 && blockIdx.x == 0 && h == 0) atomicOr(tb.status, TQ_STATUS_CAPACITY);
+        return;
+    }
+    const int tile = start / 16 + blockIdx.x;
+    const int first = tile * 16;
+    if (first >= start + a.T) return;
+    const int lo_slot = max(start - first, 0);
+    const int hi_slot = min(start + a.T - first, 16);
+    const bool full = (lo_slot == 0 && hi_slot == 16);
+
+    if (tid < (1 << BK)) ck_s[tid] = tb.centroids_kd[tid];
+    if (tid < (1 << BK) - 1) tk_s[tid] = tb.bounds_k[tid];
+    if (tid < (1 << BV) - 1) tv_s[tid] = tb.bounds_v[tid];
+    for (int i = tid; i < 16 * M / 32; i += 128) (&sg[0][0])[i] = 0u;
+    __syncthreads();
+
+    double dsign[VPL];
+#pragma unroll
+    for (int k = 0; k < VPL; ++k) dsign[k] = (double)tb.signs[lane * VPL + k];
+
+    // ---------------- 1. normalise, rotate, encode (fp64) ----------------
+    unsigned sat = 0u;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+#pragma unroll 1
+    for (int it = 0; it < 8; ++it) {
+        const int n = w + 4 * (it & 3);
+        const bool is_key = it < 4;
+        if (n < lo_slot || n >= hi_slot) {
+            if (is_key) {
+#pragma unroll
+                for (int k = 0; k < VPL / 2; ++k) {
+                    rh[n][lane * (VPL / 2) + k] = 0u;
+                    rl[n][lane * (VPL / 2) + k] = 0u;
+                }
+                if (lane == 0) sm.rho[n] = 0.f;
+            }
+            continue;
+        }
+        const size_t row = (((size_t)b * a.Hkv + h) * (size_t)a.T + (size_t)(first + n - start)) * D;
+        const __half* src = (is_key ? a.k : a.v) + row + lane * VPL;
+        double x[VPL];
+        if constexpr (VPL == 2) {
+            const __half2 p = *reinterpret_cast<const __half2*>(src);
+            x[0] = (double)__low2float(p);
+            x[1] = (double)__high2float(p);
+        } else {
+#pragma unroll
+            for (int k = 0; k < VPL; k += 4) {
+                const uint2 u = *reinterpret_cast<const uint2*>(src + k);
+                const __half2 p0 = *reinterpret_cast<const __half2*>(&u.x);
+                const __half2 p1 = *reinterpret_cast<const __half2*>(&u.y);
+                x[k] = (double)__low2float(p0);
+                x[k + 1] = (double)__high2float(p0);
+                x[k + 2] = (double)__low2float(p1);
+                x[k + 3] = (double)__high2float(p1);
+            }
+        }
+        double ss = 0.0;
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) {
+            ss += x[k] * x[k];
+            x[k] *= dsign[k];
+        }
+        ss = warp_sum(ss);
+        wht_warp<VPL>(x, lane);
+        const double nrm = sqrt(ss);
+        const double scale = nrm > 0.0 ? inv_sqrt_d / nrm : 0.0;
+        if (is_key) {
+            double r[VPL], rr = 0.0;
+#pragma unroll
+            for (int k = 0; k < VPL; ++k) {
+                const double y = x[k] * scale;
+                const int idx = encode_cell<BK>(y, tk_s);
+                kc[n][lane * VPL + k] = (uint8_t)idx;
+                r[k] = y - ck_s[idx];
+                sm.rd[n][lane * VPL + k] = r[k];
+                rr += r[k] * r[k];
+            }
+            rr = warp_sum(rr);
+            if (lane == 0) sm.rho[n] = (float)sqrt(rr);
+#pragma unroll
+            for (int k = 0; k < VPL; k += 2) {
+                const double s0 = r[k] * 4096.0, s1 = r[k + 1] * 4096.0;
+                const __half h0 = __double2half(s0), h1 = __double2half(s1);
+                const __half l0 = __double2half(s0 - (double)__half2float(h0));
+                const __half l1 = __double2half(s1 - (double)__half2float(h1));
+                rh[n][(lane * VPL + k) / 2] = (uint32_t)__half_as_ushort(h0) |
+                                              ((uint32_t)__half_as_ushort(h1) << 16);
+                rl[n][(lane * VPL + k) / 2] = (uint32_t)__half_as_ushort(l0) |
+                                              ((uint32_t)__half_as_ushort(l1) << 16);
+            }
+            if (lane == 0) {
+                nk[n] = norm_to_half_bits(nrm, sat);
+                nr[n] = norm_to_half_bits(sqrt(rr), sat);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < VPL; ++k)
+                vc[n][lane * VPL + k] = (uint8_t)encode_cell<BV>(x[k] * scale, tv_s);
+            if (lane == 0) nv[n] = norm_to_half_bits(nrm, sat);
+        }
+    }
+    __syncthreads();
+
+    // ---------------- 2. z = S r on the tensor cores ----------------
+    {
+        const int g = lane >> 2, t = lane & 3;
+        float acc[Tr::NTW][4];
+#pragma unroll
+        for (int j = 0; j < Tr::NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll 2
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t h0 = rh[g][8 * kk + t], h1 = rh[g + 8][8 * kk + t];
+            const uint32_t h2 = rh[g][8 * kk + 4 + t], h3 = rh[g + 8][8 * kk + 4 + t];
+            const uint32_t l0 = rl[g][8 * kk + t], l1 = rl[g + 8][8 * kk + t];
+            const uint32_t l2 = rl[g][8 * kk + 4 + t], l3 = rl[g + 8][8 * kk + 4 + t];
+#pragma unroll
+            for (int j = 0; j < Tr::NTW; ++j) {
+                const int nt = w * Tr::NTW + j;
+                const uint2 bf = __ldg(tb.s_frag + ((size_t)kk * Tr::NT + nt) * 32 + lane);
+                mma_16816(acc[j], h0, h1, h2, h3, bf.x, bf.y);
+                mma_16816(acc[j], l0, l1, l2, l3, bf.x, bf.y);
+            }
+        }
+        // A z this close to 0 could have the wrong sign after the fp16 split and
+        // the fp32 accumulation (|error| <= ~2^-19 sum_i |S_ji r_i| <=
+        // 2^-19 |S_j| |r|, |S_j| ~ sqrt(d)); the warp recomputes each one as an
+        // fp64 dot product from the fp64 residual. Threshold: ~10x that bound,
+        // in the 2^12-scaled units of acc.
+        const float tau_scale = 4096.0f * 1.5f * sqrtf((float)D) * (1.0f / 65536.0f);
+#pragma unroll
+        for (int j = 0; j < Tr::NTW; ++j) {
+            const int nt = w * Tr::NTW + j;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int tok = g + 8 * (e >> 1);
+                unsigned todo = __ballot_sync(kFull, fabsf(acc[j][e]) < sm.rho[tok] * tau_scale);
+                while (todo) {
+                    const int src = __ffs(todo) - 1;
+                    todo &= todo - 1;
+                    const int stok = (src >> 2) + 8 * (e >> 1);
+                    const int srow = 8 * nt + 2 * (src & 3) + (e & 1);
+                    double part = 0.0;
+                    for (int i = lane; i < D; i += 32)
+                        part += (double)__ldg(tb.s_t + (size_t)i * M + srow) * sm.rd[stok][i];
+                    part = warp_sum(part);
+                    if (lane == src) acc[j][e] = part >= 0.0 ? 1.f : -1.f;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < Tr::NTW; ++j) {
+            const int row0 = 8 * (w * Tr::NTW + j) + 2 * t;
+            const uint32_t lo = (acc[j][0] >= 0.f ? 1u : 0u) | (acc[j][1] >= 0.f ? 2u : 0u);
+            const uint32_t hi = (acc[j][2] >= 0.f ? 1u : 0u) | (acc[j][3] >= 0.f ? 2u : 0u);
+            if (lo) atomicOr(&sg[g][row0 >> 5], lo << (row0 & 31));
+            if (hi) atomicOr(&sg[g + 8][row0 >> 5], hi << (row0 & 31));
+        }
+    }
+    __syncthreads();
+
+    // ---------------- 3. pack the 32 lane strings ----------------
+    uint8_t* tile_ptr = a.cache + (((size_t)b * a.Hkv + h) * (size_t)(a.capacity / 16) + tile) *
+                                      (size_t)a.tile_bytes;
+    {
+        const int L = lane, gL = L >> 2, tL = L & 3;
+        auto is_new = [&](int tok) { return tok >= lo_slot && tok < hi_slot; };
+#pragma unroll 1
+        for (int c = w; c < Tr::NCH; c += 4) {
+            uint32_t word[Tr::CW], mask[Tr::CW];
+#pragma unroll
+            for (int q = 0; q < Tr::CW; ++q) {
+                const int wi = c * Tr::CW + q;
+                uint32_t val = 0u, msk = 0u;
+                if (wi < Tr::SBW) {                      // key cell fields
+                    const int bit0 = 32 * wi;
+                    for (int p = bit0 / Tr::KF; p <= (bit0 + 31) / Tr::KF; ++p) {
+                        const int kk = p >> 2, r = p & 3;
+                        const int tok = gL + 8 * (r & 1);
+                        const int i0 = 16 * kk + 8 * (r >> 1) + 2 * tL;
+                        // slots that are not new hold stale shared memory: clip every
+                        // code to its width so nothing spills into a neighbour
+                        constexpr uint32_t cm = (1u << BK) - 1u;
+                        const uint32_t f = ((uint32_t)kc[tok][i0] & cm) |
+                                           (((uint32_t)kc[tok][i0 + 1] & cm) << BK);
+                        const uint32_t fm = is_new(tok) ? ((1u << Tr::KF) - 1u) : 0u;
+                        const int off = Tr::KF * p - bit0;
+                        val |= place(f, off);
+                        msk |= place(fm, off);
+                    }
+                } else if (wi < Tr::VBW) {               // QJL sign pairs
+                    const int s = wi - Tr::SBW;
+#pragma unroll 4
+                    for (int q2 = 0; q2 < 16; ++q2) {
+                        const int p = 16 * s + q2;
+                        const int kk = p >> 2, r = p & 3;
+                        const int tok = gL + 8 * (r & 1);
+                        const int row = 16 * kk + 8 * (r >> 1) + 2 * tL;
+                        const uint32_t bits = (sg[tok][row >> 5] >> (row & 31)) & 3u;
+                        val |= ((bits & 1u) << q2) | ((bits >> 1) << (16 + q2));
+                        if (is_new(tok)) msk |= (1u << q2) | (1u << (16 + q2));
+                    }
+                } else {                                  // value cell fields
+                    const int bit0 = 32 * (wi - Tr::VBW);
+                    for (int p = bit0 / Tr::VF; p <= (bit0 + 31) / Tr::VF; ++p) {
+                        const int kk = p >> 2, r = p & 3;
+                        const int tok0 = 2 * tL + 8 * (r >> 1);
+                        const int coord = 16 * kk + gL + 8 * (r & 1);
+                        constexpr uint32_t cm = (1u << BV) - 1u;
+                        const uint32_t f = ((uint32_t)vc[tok0][coord] & cm) |
+                                           (((uint32_t)vc[tok0 + 1][coord] & cm) << BV);
+                        const uint32_t fm = (is_new(tok0) ? ((1u << BV) - 1u) : 0u) |
+                                            (is_new(tok0 + 1) ? (((1u << BV) - 1u) << BV) : 0u);
+                        const int off = Tr::VF * p - bit0;
+                        val |= place(f, off);
+                        msk |= place(fm, off);
+                    }
+                }
+                word[q] = val;
+                mask[q] = msk;
+            }
+            uint8_t* dst = tile_ptr + ((size_t)c * 32 + L) * Tr::CB;
+            if constexpr (Tr::CW == 4) {
+                uint4 v = make_uint4(word[0], word[1], word[2], word[3]);
+                if (!full) {
+                    const uint4 o = *reinterpret_cast<const uint4*>(dst);
+                    v.x = (o.x & ~mask[0]) | (v.x & mask[0]);
+                    v.y = (o.y & ~mask[1]) | (v.y & mask[1]);
+                    v.z = (o.z & ~mask[2]) | (v.z & mask[2]);
+                    v.w = (o.w & ~mask[3]) | (v.w & mask[3]);
+                }
+                *reinterpret_cast<uint4*>(dst) = v;
+            } else {
+                uint2 v = make_uint2(word[0], word[1]);
+                if (!full) {
+                    const uint2 o = *reinterpret_cast<const uint2*>(dst);
+                    v.x = (o.x & ~mask[0]) | (v.x & mask[0]);
+                    v.y = (o.y & ~mask[1]) | (v.y & mask[1]);
+                }
+                *reinterpret_cast<uint2*>(dst) = v;
+            }
+        }
+        // norms: 32 halves of |k|, rho then 16 halves of |v|
+        if (tid < 48) {
+            const size_t base = (size_t)4 * BITS * D;
+            int tok, off;
+            uint16_t v16;
+            if (tid < 32) {
+                const int g2 = tid >> 2, s = tid & 3;
+                tok = g2 + 8 * (s >> 1);
+                v16 = (s & 1) ? nr[tok] : nk[tok];
+                off = 8 * g2 + 2 * s;
+            } else {
+                const int u = tid - 32, g2 = u >> 1, s = u & 1;
+                tok = g2 + 8 * s;
+                v16 = nv[tok];
+                off = 64 + 4 * g2 + 2 * s;
+            }
+            if (is_new(tok)) *reinterpret_cast<uint16_t*>(tile_ptr + base + off) = v16;
+        }
+    }
+    if (sat) atomicOr(tb.status, TQ_STATUS_NORM_SAT);
+}
+
+template <int D, int BITS>
+cudaError_t launch_quantize_t(const DevTables& tb, const QuantizeArgs& a, cudaStream_t st)
+{
+    const int tiles = (a.T + 15) / 16 + 1;
+    dim3 grid(tiles, a.Hkv, a.B);
+    const size_t smem = sizeof(QuantSmem<D>);
+    static bool attr_set = false;   // one attribute call per instantiation
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(quantize_kernel<D, BITS>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    quantize_kernel<D, BITS><<<grid, 128, smem, st>>>(tb, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(int d, int bits, const DevTables& tb, const QuantizeArgs& a,
+                            cudaStream_t st)
+{
+#define TQ_Q(DD, BB) \
+    if (d == DD && bits == BB) return launch_quantize_t<DD, BB>(tb, a, st);
+    TQ_Q(64, 2) TQ_Q(64, 3) TQ_Q(64, 4)
+    TQ_Q(128, 2) TQ_Q(128, 3) TQ_Q(128, 4)
+    TQ_Q(256, 2) TQ_Q(256, 3) TQ_Q(256, 4)
+#undef TQ_Q
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tq

@@ -180,14 +180,18 @@ static double Phi(double x) { return 0.5 * erfc(-x / M_SQRT2); }
 /* Optimal L = 2^B level scalar quantizer for N(0,1) by Lloyd's iteration:
  * boundaries are midpoints of neighbouring centroids, each centroid is the
  * conditional mean of its cell, (phi(lo) - phi(hi)) / (Phi(hi) - Phi(lo)).
- * Starts from evenly spaced centroids on [-2, 2]; stops when no centroid moves
- * by 1e-13; the result is made exactly symmetric. Returns 0 on convergence. */
+ * Starts from evenly spaced centroids on [-2, 2] and iterates to fp64
+ * convergence: once no centroid moves by 1e-12, it continues until the largest
+ * step stops shrinking (the fp64 noise floor), so the fixed point is known far
+ * below fp32 resolution; the result is made exactly symmetric. Returns 0 on
+ * convergence. */
 int oracle_lloyd_max_unit(int B, double* c, int* iters_out)
 {
     int L = 1 << B;
     double nc[16];
     for (int j = 0; j < L; ++j) c[j] = -2.0 + 4.0 * (j + 0.5) / L;
     int it, ok = -1;
+    double prev = INFINITY;
     for (it = 0; it < 2000000; ++it) {
         double delta = 0.0;
         for (int j = 0; j < L; ++j) {
@@ -200,7 +204,10 @@ int oracle_lloyd_max_unit(int B, double* c, int* iters_out)
             if (dd > delta) delta = dd;
         }
         memcpy(c, nc, sizeof(double) * L);
-        if (delta < 1e-13) { ok = 0; break; }
+        /* below 1e-12 the iteration is in its linear regime: run it down to
+         * the fp64 noise floor, i.e. until the step stops shrinking */
+        if (delta == 0.0 || (delta < 1e-12 && delta >= prev)) { ok = 0; break; }
+        prev = delta;
     }
     for (int j = 0; j < L / 2; ++j) {
         double s = 0.5 * (c[L - 1 - j] - c[j]);
@@ -385,7 +392,7 @@ void oracle_quantize_values(int d, int N, const uint16_t* x, const int8_t* D,
 /*   K code of token g + 8(r&1), coordinate 16kk + 8(r>>1) + 2t + e,          */
 /*        B_K bits at bit 2*B_K*p + e*B_K;                                    */
 /*   sign of the same token for QJL row 16kk + 8(r>>1) + 2t + e,              */
-/*        at bit B_K*d/2 + 2p + e;                                            */
+/*        at bit B_K*d/2 + 32*(p/16) + 16e + (p%16);                          */
 /*   V code of token 2t + 8(r>>1) + e, coordinate 16kk + g + 8(r&1),          */
 /*        B_V bits at bit (B_K+1)*d/2 + 2*B_V*p + e*B_V.                      */
 /* ------------------------------------------------------------------------- */
@@ -421,6 +428,10 @@ static unsigned get_bits(const uint8_t* tile, int d, int b, int lane, int64_t bi
     return v;
 }
 
+/* Sign pair p of a lane: element 0 at bit p%16, element 1 at bit 16 + p%16 of
+ * the lane's sign word p/16. */
+static int64_t sign_bit(int p, int e) { return 32LL * (p / 16) + 16 * e + (p % 16); }
+
 static void put_half(uint8_t* p, uint16_t h) { p[0] = (uint8_t)(h & 0xff); p[1] = (uint8_t)(h >> 8); }
 static uint16_t get_half(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 
@@ -451,7 +462,7 @@ void oracle_pack_stream(int d, int b, int N, const uint8_t* kidx, const uint8_t*
                         if (BK > 0)
                             put_bits(tile, d, b, lane, 2LL * BK * p + e * BK, BK,
                                      kidx[(size_t)nk * d + ik]);
-                        put_bits(tile, d, b, lane, sbase + 2 * p + e, 1,
+                        put_bits(tile, d, b, lane, sbase + sign_bit(p, e), 1,
                                  ksign[(size_t)nk * m + ik]);
                     }
                     if (nv < N)
@@ -496,7 +507,7 @@ void oracle_unpack_stream(int d, int b, int N, const uint8_t* in, uint8_t* kidx,
                         kidx[(size_t)nk * d + ik] = (uint8_t)(BK > 0 ?
                             get_bits(tile, d, b, lane, 2LL * BK * p + e * BK, BK) : 0);
                         ksign[(size_t)nk * m + ik] =
-                            (uint8_t)get_bits(tile, d, b, lane, sbase + 2 * p + e, 1);
+                            (uint8_t)get_bits(tile, d, b, lane, sbase + sign_bit(p, e), 1);
                     }
                     if (nv < N)
                         vidx[(size_t)nv * d + iv] =
