@@ -41,9 +41,7 @@ template <int D, int BITS>
 struct AttTraits {
     static constexpr int BK = BITS - 1, BV = BITS;
     static constexpr int KF = 2 * BK, VF = 2 * BV;          // field widths
-    static constexpr int LW = BITS * D / 32;                 // words per lane string
     static constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;
-    static constexpr int CW = CB / 4;
     static constexpr int SBW = BK * D / 64;                  // first sign word
     static constexpr int VB = (BK + 1) * D / 2;              // first value bit
     static constexpr int KK = D / 16;                        // k-steps / coordinate blocks
@@ -53,11 +51,14 @@ struct AttTraits {
     static constexpr size_t DYN_SMEM = QF_BYTES > MERGE_BYTES ? QF_BYTES : MERGE_BYTES;
 };
 
-// Row offset (field value * 128) of an F-bit field starting at bit `pos` of the
-// lane string, OR-ed with `lane_bits` (lane * 4 plus the table base, which is
-// aligned to the table size): a lane-replicated table address in one funnel
-// (or plain) shift and one LOP3.
-__device__ __forceinline__ uint32_t lut_addr(const uint32_t* s, int pos, int F, uint32_t lane_bits)
+// Offset, inside a lane-replicated table, of the entry selected by the F-bit
+// field at bit `pos` of the lane string: field * 128 + 4 * lane, built with one
+// funnel (or plain) shift and one LOP3 (lane4 = 4 * lane occupies bits 2..6,
+// the field bits 7 and up). The table's own shared address is added by the
+// load as an immediate, so no alignment of the table is assumed: shared
+// memory does not start at address 0 of the window, and declared alignments
+// above 1 KB are not honoured there.
+__device__ __forceinline__ uint32_t lut_off(const uint32_t* s, int pos, int F, uint32_t lane4)
 {
     const int wi = pos >> 5, o = pos & 31;
     const uint32_t mask = ((1u << F) - 1u) << 7;
@@ -66,14 +67,12 @@ __device__ __forceinline__ uint32_t lut_addr(const uint32_t* s, int pos, int F, 
         v = (o >= 7) ? (s[wi] >> (o - 7)) : (s[wi] << (7 - o));
     else
         v = __funnelshift_r(s[wi], s[wi + 1], o - 7);
-    return (v & mask) | lane_bits;
+    return (v & mask) | lane4;
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t shared_addr)
+__device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t byte_off)
 {
-    uint32_t v;
-    asm("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(shared_addr));
-    return v;
+    return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(table) + byte_off);
 }
 
 // fp16x2 (+1/-1, +1/-1) from sign pair p: element 0 at bit p%16, element 1 at
@@ -155,45 +154,174 @@ __global__ void __launch_bounds__(D) attend_prologue(DevTables tb, AttendArgs a)
         }
         const size_t units = (size_t)a.Hkv * groups;
         uint4* dst = reinterpret_cast<uint4*>(a.qfrag) +
-                     ((((size_t)b * units + unit) * (D / 16) + kk) * 32 + col * 4 + t) * 2;
-        dst[0] = make_uint4(hi[0], hi[1], lo[0], lo[1]);   // codebook term: b0,b1 hi; b0,b1 lo
-        dst[1] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
+                     (((size_t)b * units + unit) * (D / 16) + kk) * 64 + col * 4 + t;
+        dst[0] = make_uint4(hi[0], hi[1], lo[0], lo[1]);    // codebook term: b0,b1 hi; b0,b1 lo
+        dst[32] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
     }
 }
 
 // ---------------------------------------------------------------- split kernel
-template <int D, int BITS, int CW>
-__device__ __forceinline__ void load_tile(const uint8_t* tp, int lane, int g, uint32_t (&s)[BITS * D / 32],
-                                          uint2& kn, uint32_t& vn)
+template <int D, int BITS>
+struct TileData {
+    uint32_t s[BITS * D / 32];   // this lane's string of the tile
+    uint2 kn;                    // fp16 {|k_g|, rho_g, |k_g+8|, rho_g+8}
+    uint32_t vn;                 // fp16 {|v_g|, |v_g+8|}
+};
+
+template <int D, int BITS>
+__device__ __forceinline__ void load_tile(const uint8_t* tp, int lane, int g, TileData<D, BITS>& td)
 {
-    constexpr int CB = CW * 4, NCH = BITS * D / 8 / CB;
+    using Tr = AttTraits<D, BITS>;
+    constexpr int CB = Tr::CB, NCH = BITS * D / 8 / CB;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
         const uint8_t* src = tp + ((size_t)c * 32 + lane) * CB;
-        if constexpr (CW == 4) {
+        if constexpr (CB == 16) {
             const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src));
-            s[4 * c] = v.x; s[4 * c + 1] = v.y; s[4 * c + 2] = v.z; s[4 * c + 3] = v.w;
+            td.s[4 * c] = v.x; td.s[4 * c + 1] = v.y; td.s[4 * c + 2] = v.z; td.s[4 * c + 3] = v.w;
         } else {
             const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src));
-            s[2 * c] = v.x; s[2 * c + 1] = v.y;
+            td.s[2 * c] = v.x; td.s[2 * c + 1] = v.y;
         }
     }
-    kn = __ldcs(reinterpret_cast<const uint2*>(tp + 4 * BITS * D + 8 * g));
-    vn = __ldcs(reinterpret_cast<const uint32_t*>(tp + 4 * BITS * D + 64 + 4 * g));
+    td.kn = __ldcs(reinterpret_cast<const uint2*>(tp + 4 * BITS * D + 8 * g));
+    td.vn = __ldcs(reinterpret_cast<const uint32_t*>(tp + 4 * BITS * D + 64 + 4 * g));
+}
+
+// Query B fragments of one k-step: x,y = hi (b0, b1), z,w = lo, for the
+// codebook term (c) and the QJL term (s). Kept in registers for d <= 128
+// (they do not change from tile to tile), in shared memory for d = 256.
+template <int KK, bool IN_REGS>
+struct QueryFrags;
+
+template <int KK>
+struct QueryFrags<KK, true> {
+    uint4 c[KK], s[KK];
+    __device__ __forceinline__ void load(const uint4* src, uint4*, int lane, int)
+    {
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+            c[kk] = src[kk * 64 + lane];
+            s[kk] = src[kk * 64 + 32 + lane];
+        }
+    }
+    __device__ __forceinline__ uint4 fc(int kk, int) const { return c[kk]; }
+    __device__ __forceinline__ uint4 fs(int kk, int) const { return s[kk]; }
+};
+
+template <int KK>
+struct QueryFrags<KK, false> {
+    const uint4* sm;
+    __device__ __forceinline__ void load(const uint4* src, uint4* smem, int, int tid)
+    {
+        for (int e = tid; e < KK * 64; e += 128) smem[e] = src[e];
+        sm = smem;
+    }
+    __device__ __forceinline__ uint4 fc(int kk, int lane) const { return sm[kk * 64 + lane]; }
+    __device__ __forceinline__ uint4 fs(int kk, int lane) const { return sm[kk * 64 + 32 + lane]; }
+};
+
+template <int D>
+struct SplitState {
+    float m0, m1, l0, l1;
+    float acc[D / 16][4];
+};
+
+// Logits of one tile (log2 units) for tokens g, g+8 and heads 2t, 2t+1.
+template <int D, int BITS, typename QF>
+__device__ __forceinline__ void tile_logits(const TileData<D, BITS>& td, const QF& qf, int lane,
+                                            const uint32_t* lutk, uint32_t lane4, float (&L)[4])
+{
+    using Tr = AttTraits<D, BITS>;
+    // four independent accumulation chains: codebook hi/lo, QJL hi/lo
+    float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
+    float sh[4] = {0.f, 0.f, 0.f, 0.f}, sl[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < Tr::KK; ++kk) {
+        const uint4 bc = qf.fc(kk, lane);
+        const uint4 bs = qf.fs(kk, lane);
+        uint32_t ak[4], as[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int p = 4 * kk + r;
+            ak[r] = lut_load(lutk, lut_off(td.s, Tr::KF * p, Tr::KF, lane4));
+            as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15);
+        }
+        mma_16816(ch, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
+        mma_16816(cl, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+        mma_16816(sh, as[0], as[1], as[2], as[3], bs.x, bs.y);
+        mma_16816(sl, as[0], as[1], as[2], as[3], bs.z, bs.w);
+    }
+    const float kn_g = half_bits_to_float((uint16_t)(td.kn.x & 0xffff)) * (1.0f / 128.0f);
+    const float rho_g = half_bits_to_float((uint16_t)(td.kn.x >> 16));
+    const float kn_h = half_bits_to_float((uint16_t)(td.kn.y & 0xffff)) * (1.0f / 128.0f);
+    const float rho_h = half_bits_to_float((uint16_t)(td.kn.y >> 16));
+    // the B operands carry a factor 2^7
+    L[0] = kn_g * fmaf(rho_g, sh[0] + sl[0], ch[0] + cl[0]);
+    L[1] = kn_g * fmaf(rho_g, sh[1] + sl[1], ch[1] + cl[1]);
+    L[2] = kn_h * fmaf(rho_h, sh[2] + sl[2], ch[2] + cl[2]);
+    L[3] = kn_h * fmaf(rho_h, sh[3] + sl[3], ch[3] + cl[3]);
+}
+
+// Online-softmax update and P V for one tile.
+template <int D, int BITS>
+__device__ __forceinline__ void tile_accumulate(const TileData<D, BITS>& td, float (&L)[4], bool v0,
+                                                bool v1, const uint32_t* lutv, uint32_t lane4,
+                                                SplitState<D>& st)
+{
+    using Tr = AttTraits<D, BITS>;
+    float mx0 = fmaxf(L[0], L[2]), mx1 = fmaxf(L[1], L[3]);
+#pragma unroll
+    for (int sh = 4; sh <= 16; sh <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
+    }
+    const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+    if (__any_sync(kFull, mn0 != st.m0 || mn1 != st.m1)) {   // rescale only when a max moved
+        const float al0 = exp2f(st.m0 - mn0), al1 = exp2f(st.m1 - mn1);
+        st.l0 *= al0;
+        st.l1 *= al1;
+#pragma unroll
+        for (int kk = 0; kk < Tr::KK; ++kk) {
+            st.acc[kk][0] *= al0;
+            st.acc[kk][1] *= al1;
+            st.acc[kk][2] *= al0;
+            st.acc[kk][3] *= al1;
+        }
+        st.m0 = mn0;
+        st.m1 = mn1;
+    }
+    const float p0 = exp2f(L[0] - st.m0), p1 = exp2f(L[1] - st.m1);
+    const float p2 = exp2f(L[2] - st.m0), p3 = exp2f(L[3] - st.m1);
+    st.l0 += p0 + p2;
+    st.l1 += p1 + p3;
+    // slots past seq_len may hold anything (even NaN norms): select, never multiply
+    const float vn_g = v0 ? half_bits_to_float((uint16_t)(td.vn & 0xffff)) : 0.f;
+    const float vn_h = v1 ? half_bits_to_float((uint16_t)(td.vn >> 16)) : 0.f;
+    const uint32_t b0 = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
+    const uint32_t b1 = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
+#pragma unroll
+    for (int kk = 0; kk < Tr::KK; ++kk) {
+        uint32_t av[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            av[r] = lut_load(lutv, lut_off(td.s, Tr::VB + Tr::VF * (4 * kk + r), Tr::VF, lane4));
+        mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0, b1);
+    }
 }
 
 template <int D, int BITS, bool SCORES>
-__global__ void __launch_bounds__(128) attend_split(DevTables tb, AttendArgs a)
+__global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables tb, AttendArgs a)
 {
     using Tr = AttTraits<D, BITS>;
-    constexpr int KK = Tr::KK, LW = Tr::LW;
-    // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l. Each
-    // table is aligned to its size so that a table address is (field*128) | (4l + base).
-    __shared__ __align__(Tr::NLV * 128) uint32_t lutv[Tr::NLV * 32];
-    __shared__ __align__(Tr::NLK * 128) uint32_t lutk[Tr::NLK * 32];
+    constexpr int KK = Tr::KK;
+    constexpr bool kRegQ = D <= 128;
+    // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l, so
+    // the 32 lanes of a warp always hit 32 different banks.
+    __shared__ __align__(16) uint32_t lutv[Tr::NLV * 32];
+    __shared__ __align__(16) uint32_t lutk[Tr::NLK * 32];
     extern __shared__ uint4 dyn_smem[];
-    uint4* qf = dyn_smem;                                  // [KK][32][2] during the tile loop
-    float* mrg = reinterpret_cast<float*>(dyn_smem);       // [4][8][D+2] after it
+    float* mrg = reinterpret_cast<float*>(dyn_smem);       // [4][8][D+2] after the tile loop
 
     const int split = blockIdx.x, unit = blockIdx.y, b = blockIdx.z;
     const int groups = a.plan.groups;
@@ -204,8 +332,9 @@ __global__ void __launch_bounds__(128) attend_split(DevTables tb, AttendArgs a)
 
     for (int e = tid; e < Tr::NLK * 32; e += 128) lutk[e] = __ldg(tb.lut_k + (e >> 5));
     for (int e = tid; e < Tr::NLV * 32; e += 128) lutv[e] = __ldg(tb.lut_v + (e >> 5));
-    const uint4* qsrc = reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64;
-    for (int e = tid; e < KK * 64; e += 128) qf[e] = qsrc[e];
+    QueryFrags<KK, kRegQ> qf;
+    qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64, dyn_smem,
+            lane, tid);
 
     int seq = a.seq_len[b];
     const int lim = min(a.max_len, a.capacity);
@@ -220,79 +349,22 @@ __global__ void __launch_bounds__(128) attend_split(DevTables tb, AttendArgs a)
     const int t_end = min(t_begin + a.plan.tps, ntiles);
     const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
                                          (size_t)a.tile_bytes;
-    const uint32_t lk_bits = (uint32_t)__cvta_generic_to_shared(lutk) + 4u * lane;
-    const uint32_t lv_bits = (uint32_t)__cvta_generic_to_shared(lutv) + 4u * lane;
+    const uint32_t lane4 = 4u * lane;
     const int ratio = a.Hq / a.Hkv;
 
-    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
-    float acc[KK][4];
-#pragma unroll
-    for (int kk = 0; kk < KK; ++kk) acc[kk][0] = acc[kk][1] = acc[kk][2] = acc[kk][3] = 0.f;
-
-    // software pipeline: the next tile's lane string is in flight while this one is decoded
-    uint32_t nxt[LW];
-    uint2 kn_n = make_uint2(0u, 0u);
-    uint32_t vn_n = 0u;
-    int tl = t_begin + w;
-    const bool skip_decode_past = SCORES;   // scores: tiles past seq need no decode
-    if (tl < t_end && !(skip_decode_past && tl * 16 >= seq))
-        load_tile<D, BITS, Tr::CW>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, nxt, kn_n, vn_n);
-
+    if constexpr (SCORES) {
+        const int j0 = grp * 8 + 2 * t;
+        TileData<D, BITS> td;
 #pragma unroll 1
-    for (; tl < t_end; tl += 4) {
-        const int pos0 = tl * 16 + g, pos1 = pos0 + 8;
-        if (SCORES && tl * 16 >= seq) {
-            const int j0 = grp * 8 + 2 * t;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (j0 + hh >= ratio) continue;
-                float* row = a.out + ((size_t)b * a.Hq + hkv * ratio + j0 + hh) * a.max_len;
-                if (pos0 < a.max_len) row[pos0] = -CUDART_INF_F;
-                if (pos1 < a.max_len) row[pos1] = -CUDART_INF_F;
+        for (int tl = t_begin + w; tl < t_end; tl += 4) {
+            const int pos0 = tl * 16 + g, pos1 = pos0 + 8;
+            float L[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+            if (tl * 16 < seq) {   // warp-uniform
+                load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, td);
+                tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
+                if (pos0 >= seq) L[0] = L[1] = -CUDART_INF_F;
+                if (pos1 >= seq) L[2] = L[3] = -CUDART_INF_F;
             }
-            continue;
-        }
-        uint32_t s[LW];
-#pragma unroll
-        for (int i = 0; i < LW; ++i) s[i] = nxt[i];
-        const uint2 kn = kn_n;
-        const uint32_t vn = vn_n;
-        const int tn = tl + 4;
-        if (tn < t_end && !(skip_decode_past && tn * 16 >= seq))
-            load_tile<D, BITS, Tr::CW>(sbase + (size_t)tn * (size_t)a.tile_bytes, lane, g, nxt, kn_n, vn_n);
-
-        float cc[4] = {0.f, 0.f, 0.f, 0.f}, cs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-            const uint4 bc = qf[(kk * 32 + lane) * 2];
-            const uint4 bs = qf[(kk * 32 + lane) * 2 + 1];
-            uint32_t ak[4], as[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int p = 4 * kk + r;
-                ak[r] = lds32(lut_addr(s, Tr::KF * p, Tr::KF, lk_bits));
-                as[r] = sign_pair(s[Tr::SBW + (p >> 4)], p & 15);
-            }
-            mma_16816(cc, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
-            mma_16816(cc, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
-            mma_16816(cs, as[0], as[1], as[2], as[3], bs.x, bs.y);
-            mma_16816(cs, as[0], as[1], as[2], as[3], bs.z, bs.w);
-        }
-        const float kn_g = half_bits_to_float((uint16_t)(kn.x & 0xffff));
-        const float rho_g = half_bits_to_float((uint16_t)(kn.x >> 16));
-        const float kn_h = half_bits_to_float((uint16_t)(kn.y & 0xffff));
-        const float rho_h = half_bits_to_float((uint16_t)(kn.y >> 16));
-        // the B operands carry a factor 2^7
-        float L0 = (kn_g * (1.0f / 128.0f)) * fmaf(rho_g, cs[0], cc[0]);
-        float L1 = (kn_g * (1.0f / 128.0f)) * fmaf(rho_g, cs[1], cc[1]);
-        float L2 = (kn_h * (1.0f / 128.0f)) * fmaf(rho_h, cs[2], cc[2]);
-        float L3 = (kn_h * (1.0f / 128.0f)) * fmaf(rho_h, cs[3], cc[3]);
-        if (pos0 >= seq) L0 = L1 = -CUDART_INF_F;
-        if (pos1 >= seq) L2 = L3 = -CUDART_INF_F;
-
-        if constexpr (SCORES) {
-            const int j0 = grp * 8 + 2 * t;
-            const float L[4] = {L0, L1, L2, L3};
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 if (j0 + hh >= ratio) continue;
@@ -300,69 +372,79 @@ __global__ void __launch_bounds__(128) attend_split(DevTables tb, AttendArgs a)
                 if (pos0 < a.max_len) row[pos0] = L[hh] * kLn2;
                 if (pos1 < a.max_len) row[pos1] = L[2 + hh] * kLn2;
             }
-            continue;
-        } else {
-            float mx0 = fmaxf(L0, L2), mx1 = fmaxf(L1, L3);
+        }
+        return;
+    } else {
+        SplitState<D> st;
+        st.m0 = st.m1 = -CUDART_INF_F;
+        st.l0 = st.l1 = 0.f;
 #pragma unroll
-            for (int sh = 4; sh <= 16; sh <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
-            }
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            if (__any_sync(kFull, mn0 != m0 || mn1 != m1)) {   // rescale only when a max moved
-                const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-                l0 *= al0;
-                l1 *= al1;
-#pragma unroll
-                for (int kk = 0; kk < KK; ++kk) {
-                    acc[kk][0] *= al0;
-                    acc[kk][1] *= al1;
-                    acc[kk][2] *= al0;
-                    acc[kk][3] *= al1;
-                }
-                m0 = mn0;
-                m1 = mn1;
-            }
-            const float p0 = exp2f(L0 - m0), p1 = exp2f(L1 - m1);
-            const float p2 = exp2f(L2 - m0), p3 = exp2f(L3 - m1);
-            l0 += p0 + p2;
-            l1 += p1 + p3;
-            // slots past seq_len may hold anything (even NaN norms): select, never multiply
-            const float vn_g = pos0 < seq ? half_bits_to_float((uint16_t)(vn & 0xffff)) : 0.f;
-            const float vn_h = pos1 < seq ? half_bits_to_float((uint16_t)(vn >> 16)) : 0.f;
-            const uint32_t b0 = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
-            const uint32_t b1 = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
-#pragma unroll
-            for (int kk = 0; kk < KK; ++kk) {
-                uint32_t av[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    av[r] = lds32(lut_addr(s, Tr::VB + Tr::VF * (4 * kk + r), Tr::VF, lv_bits));
-                mma_16816(acc[kk], av[0], av[1], av[2], av[3], b0, b1);
+        for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
+
+        // two tile buffers: the next tile's lane string is in flight while this one is
+        // decoded (d = 256 strings are too large to double-buffer in registers)
+        TileData<D, BITS> ta, tb2;
+        if constexpr (D > 128) {
+#pragma unroll 1
+            for (int tl = t_begin + w; tl < t_end; tl += 4) {
+                load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, ta);
+                float L[4];
+                tile_logits<D, BITS>(ta, qf, lane, lutk, lane4, L);
+                const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
+                if (!v0) L[0] = L[1] = -CUDART_INF_F;
+                if (!v1) L[2] = L[3] = -CUDART_INF_F;
+                tile_accumulate<D, BITS>(ta, L, v0, v1, lutv, lane4, st);
             }
         }
-    }
-    if constexpr (!SCORES) {
+        int tl = D > 128 ? t_end : t_begin + w;
+        if (tl < t_end) load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, ta);
+#pragma unroll 1
+        for (; tl < t_end; tl += 8) {
+            if (tl + 4 < t_end)
+                load_tile<D, BITS>(sbase + (size_t)(tl + 4) * (size_t)a.tile_bytes, lane, g, tb2);
+            {
+                float L[4];
+                tile_logits<D, BITS>(ta, qf, lane, lutk, lane4, L);
+                const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
+                if (!v0) L[0] = L[1] = -CUDART_INF_F;
+                if (!v1) L[2] = L[3] = -CUDART_INF_F;
+                tile_accumulate<D, BITS>(ta, L, v0, v1, lutv, lane4, st);
+            }
+            if (tl + 4 >= t_end) break;
+            if (tl + 8 < t_end)
+                load_tile<D, BITS>(sbase + (size_t)(tl + 8) * (size_t)a.tile_bytes, lane, g, ta);
+            {
+                const int t2 = tl + 4;
+                float L[4];
+                tile_logits<D, BITS>(tb2, qf, lane, lutk, lane4, L);
+                const bool v0 = t2 * 16 + g < seq, v1 = t2 * 16 + g + 8 < seq;
+                if (!v0) L[0] = L[1] = -CUDART_INF_F;
+                if (!v1) L[2] = L[3] = -CUDART_INF_F;
+                tile_accumulate<D, BITS>(tb2, L, v0, v1, lutv, lane4, st);
+            }
+        }
+
+        float l0 = st.l0, l1 = st.l1;
 #pragma unroll
         for (int sh = 4; sh <= 16; sh <<= 1) {
             l0 += __shfl_xor_sync(kFull, l0, sh);
             l1 += __shfl_xor_sync(kFull, l1, sh);
         }
-        __syncthreads();   // every warp is done with qf: reuse it for the merge
+        __syncthreads();   // every warp is done with the dynamic area: reuse it for the merge
         constexpr int RS = D + 2;
         float* mw = mrg + (size_t)w * 8 * RS;
         if (g == 0) {
-            mw[(2 * t) * RS] = m0;
+            mw[(2 * t) * RS] = st.m0;
             mw[(2 * t) * RS + 1] = l0;
-            mw[(2 * t + 1) * RS] = m1;
+            mw[(2 * t + 1) * RS] = st.m1;
             mw[(2 * t + 1) * RS + 1] = l1;
         }
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk) {
-            mw[(2 * t) * RS + 2 + 16 * kk + g] = acc[kk][0];
-            mw[(2 * t + 1) * RS + 2 + 16 * kk + g] = acc[kk][1];
-            mw[(2 * t) * RS + 2 + 16 * kk + g + 8] = acc[kk][2];
-            mw[(2 * t + 1) * RS + 2 + 16 * kk + g + 8] = acc[kk][3];
+            mw[(2 * t) * RS + 2 + 16 * kk + g] = st.acc[kk][0];
+            mw[(2 * t + 1) * RS + 2 + 16 * kk + g] = st.acc[kk][1];
+            mw[(2 * t) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][2];
+            mw[(2 * t + 1) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][3];
         }
         __syncthreads();
         float* dst = a.partial + (((size_t)b * units + unit) * a.plan.nsplit + split) * 8 * RS;
