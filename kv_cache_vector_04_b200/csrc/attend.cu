@@ -48,7 +48,15 @@ struct AttTraits {
     static constexpr int NLK = 1 << KF, NLV = 1 << VF;       // LUT entries
     static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
     static constexpr size_t MERGE_BYTES = (size_t)4 * 8 * (D + 2) * 4;
-    static constexpr size_t DYN_SMEM = QF_BYTES > MERGE_BYTES ? QF_BYTES : MERGE_BYTES;
+    // cp.async staging ring: per warp STAGES copies of {32 lane strings, 32 K-norm
+    // and 32 V-norm copies}; each lane stages and reads back only its own bytes
+    static constexpr int STAGES = 3;
+    static constexpr int NCH = BITS * D / 8 / CB;
+    static constexpr int STAGE_BYTES = NCH * 32 * CB + 32 * 8 + 32 * 4;
+    static constexpr size_t RING_BYTES = (size_t)4 * STAGES * STAGE_BYTES;
+    static constexpr size_t QF_SMEM = D <= 128 ? 0 : QF_BYTES;      // d = 256 keeps B in smem
+    static constexpr size_t LOOP_BYTES = RING_BYTES + QF_SMEM;
+    static constexpr size_t DYN_SMEM = LOOP_BYTES > MERGE_BYTES ? LOOP_BYTES : MERGE_BYTES;
 };
 
 // Offset, inside a lane-replicated table, of the entry selected by the F-bit
@@ -161,6 +169,22 @@ __global__ void __launch_bounds__(D) attend_prologue(DevTables tb, AttendArgs a)
 }
 
 // ---------------------------------------------------------------- split kernel
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 template <int D, int BITS>
 struct TileData {
     uint32_t s[BITS * D / 32];   // this lane's string of the tile
@@ -186,6 +210,45 @@ __device__ __forceinline__ void load_tile(const uint8_t* tp, int lane, int g, Ti
     }
     td.kn = __ldcs(reinterpret_cast<const uint2*>(tp + 4 * BITS * D + 8 * g));
     td.vn = __ldcs(reinterpret_cast<const uint32_t*>(tp + 4 * BITS * D + 64 + 4 * g));
+}
+
+// Stage this lane's bytes of tile `tp` into ring slot `slot` (shared address).
+template <int D, int BITS>
+__device__ __forceinline__ void stage_tile(uint32_t slot, const uint8_t* tp, int lane, int g)
+{
+    using Tr = AttTraits<D, BITS>;
+#pragma unroll
+    for (int c = 0; c < Tr::NCH; ++c) {
+        const uint32_t off = (uint32_t)(c * 32 + lane) * Tr::CB;
+        if constexpr (Tr::CB == 16)
+            cp_async16(slot + off, tp + off);
+        else
+            cp_async8(slot + off, tp + off);
+    }
+    constexpr uint32_t nb = Tr::NCH * 32 * Tr::CB;
+    cp_async8(slot + nb + 8u * lane, tp + 4 * BITS * D + 8 * g);
+    cp_async4(slot + nb + 256u + 4u * lane, tp + 4 * BITS * D + 64 + 4 * g);
+}
+
+// Read back this lane's bytes of a staged tile.
+template <int D, int BITS>
+__device__ __forceinline__ void read_stage(const uint8_t* slot, int lane, TileData<D, BITS>& td)
+{
+    using Tr = AttTraits<D, BITS>;
+#pragma unroll
+    for (int c = 0; c < Tr::NCH; ++c) {
+        const uint8_t* src = slot + (c * 32 + lane) * Tr::CB;
+        if constexpr (Tr::CB == 16) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src);
+            td.s[4 * c] = v.x; td.s[4 * c + 1] = v.y; td.s[4 * c + 2] = v.z; td.s[4 * c + 3] = v.w;
+        } else {
+            const uint2 v = *reinterpret_cast<const uint2*>(src);
+            td.s[2 * c] = v.x; td.s[2 * c + 1] = v.y;
+        }
+    }
+    constexpr int nb = Tr::NCH * 32 * Tr::CB;
+    td.kn = *reinterpret_cast<const uint2*>(slot + nb + 8 * lane);
+    td.vn = *reinterpret_cast<const uint32_t*>(slot + nb + 256 + 4 * lane);
 }
 
 // Query B fragments of one k-step: x,y = hi (b0, b1), z,w = lo, for the
@@ -270,14 +333,18 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, BITS>& td, flo
                                                 SplitState<D>& st)
 {
     using Tr = AttTraits<D, BITS>;
-    float mx0 = fmaxf(L[0], L[2]), mx1 = fmaxf(L[1], L[3]);
+    // The running max only moves when some logit exceeds it (rarely, after the
+    // first tiles): only then reduce across the 8 token lanes and rescale.
+    // Otherwise every p = exp2(L - m) <= 1, which also keeps p*|v| in fp16 range.
+    const bool above = (L[0] > st.m0) || (L[2] > st.m0) || (L[1] > st.m1) || (L[3] > st.m1);
+    if (__any_sync(kFull, above)) {
+        float mx0 = fmaxf(L[0], L[2]), mx1 = fmaxf(L[1], L[3]);
 #pragma unroll
-    for (int sh = 4; sh <= 16; sh <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
-    }
-    const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
-    if (__any_sync(kFull, mn0 != st.m0 || mn1 != st.m1)) {   // rescale only when a max moved
+        for (int sh = 4; sh <= 16; sh <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
+        }
+        const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
         const float al0 = exp2f(st.m0 - mn0), al1 = exp2f(st.m1 - mn1);
         st.l0 *= al0;
         st.l1 *= al1;
@@ -333,8 +400,8 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
     for (int e = tid; e < Tr::NLK * 32; e += 128) lutk[e] = __ldg(tb.lut_k + (e >> 5));
     for (int e = tid; e < Tr::NLV * 32; e += 128) lutv[e] = __ldg(tb.lut_v + (e >> 5));
     QueryFrags<KK, kRegQ> qf;
-    qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64, dyn_smem,
-            lane, tid);
+    qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64,
+            reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dyn_smem) + Tr::RING_BYTES), lane, tid);
 
     int seq = a.seq_len[b];
     const int lim = min(a.max_len, a.capacity);
@@ -381,48 +448,42 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
 
-        // two tile buffers: the next tile's lane string is in flight while this one is
-        // decoded (d = 256 strings are too large to double-buffer in registers)
-        TileData<D, BITS> ta, tb2;
-        if constexpr (D > 128) {
-#pragma unroll 1
-            for (int tl = t_begin + w; tl < t_end; tl += 4) {
-                load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, ta);
-                float L[4];
-                tile_logits<D, BITS>(ta, qf, lane, lutk, lane4, L);
-                const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
-                if (!v0) L[0] = L[1] = -CUDART_INF_F;
-                if (!v1) L[2] = L[3] = -CUDART_INF_F;
-                tile_accumulate<D, BITS>(ta, L, v0, v1, lutv, lane4, st);
-            }
+        // cp.async pipeline: STAGES - 1 tiles of this warp are in flight while
+        // one is decoded; every lane stages and reads back only its own bytes,
+        // so the only synchronisation is the per-thread wait_group.
+        constexpr int S = Tr::STAGES;
+        uint8_t* ring = reinterpret_cast<uint8_t*>(dyn_smem) + (size_t)w * S * Tr::STAGE_BYTES;
+        const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+        const int my_first = t_begin + w;
+#pragma unroll
+        for (int i = 0; i < S - 1; ++i) {
+            const int tl = my_first + 4 * i;
+            if (tl < t_end)
+                stage_tile<D, BITS>(ring_s + i * Tr::STAGE_BYTES, sbase + (size_t)tl * (size_t)a.tile_bytes,
+                                    lane, g);
+            cp_async_commit();
         }
-        int tl = D > 128 ? t_end : t_begin + w;
-        if (tl < t_end) load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, ta);
+        TileData<D, BITS> td;
+        int slot = 0;
 #pragma unroll 1
-        for (; tl < t_end; tl += 8) {
-            if (tl + 4 < t_end)
-                load_tile<D, BITS>(sbase + (size_t)(tl + 4) * (size_t)a.tile_bytes, lane, g, tb2);
-            {
-                float L[4];
-                tile_logits<D, BITS>(ta, qf, lane, lutk, lane4, L);
-                const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
-                if (!v0) L[0] = L[1] = -CUDART_INF_F;
-                if (!v1) L[2] = L[3] = -CUDART_INF_F;
-                tile_accumulate<D, BITS>(ta, L, v0, v1, lutv, lane4, st);
-            }
-            if (tl + 4 >= t_end) break;
-            if (tl + 8 < t_end)
-                load_tile<D, BITS>(sbase + (size_t)(tl + 8) * (size_t)a.tile_bytes, lane, g, ta);
-            {
-                const int t2 = tl + 4;
-                float L[4];
-                tile_logits<D, BITS>(tb2, qf, lane, lutk, lane4, L);
-                const bool v0 = t2 * 16 + g < seq, v1 = t2 * 16 + g + 8 < seq;
-                if (!v0) L[0] = L[1] = -CUDART_INF_F;
-                if (!v1) L[2] = L[3] = -CUDART_INF_F;
-                tile_accumulate<D, BITS>(tb2, L, v0, v1, lutv, lane4, st);
-            }
+        for (int tl = my_first; tl < t_end; tl += 4) {
+            const int tn = tl + 4 * (S - 1);
+            const int nslot = slot == 0 ? S - 1 : slot - 1;   // the slot consumed last iteration
+            if (tn < t_end)
+                stage_tile<D, BITS>(ring_s + nslot * Tr::STAGE_BYTES, sbase + (size_t)tn * (size_t)a.tile_bytes,
+                                    lane, g);
+            cp_async_commit();
+            cp_async_wait<S - 1>();
+            read_stage<D, BITS>(ring + slot * Tr::STAGE_BYTES, lane, td);
+            slot = slot == S - 1 ? 0 : slot + 1;
+            float L[4];
+            tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
+            const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
+            if (!v0) L[0] = L[1] = -CUDART_INF_F;
+            if (!v1) L[2] = L[3] = -CUDART_INF_F;
+            tile_accumulate<D, BITS>(td, L, v0, v1, lutv, lane4, st);
         }
+        cp_async_wait<0>();
 
         float l0 = st.l0, l1 = st.l1;
 #pragma unroll
@@ -430,7 +491,7 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
             l0 += __shfl_xor_sync(kFull, l0, sh);
             l1 += __shfl_xor_sync(kFull, l1, sh);
         }
-        __syncthreads();   // every warp is done with the dynamic area: reuse it for the merge
+        __syncthreads();   // every warp is done with the ring: reuse it for the merge
         constexpr int RS = D + 2;
         float* mw = mrg + (size_t)w * 8 * RS;
         if (g == 0) {
