@@ -58,7 +58,7 @@ class _Cache(ctypes.Structure):
 def _load(path: str = LIB_PATH):
     if not os.path.exists(path):
         raise ImportError("libtq.so not found at %s: build it with "
-                          "`python -m kv_cache_vector_04_b200.build`" % path)
+                          "`python kv_cache_vector_04_b200/build.py`" % path)
     lib = ctypes.CDLL(path)
     P, I, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
     sig = {

@@ -1,6 +1,7 @@
 """Build the in-tree CUDA library ``libtq.so`` for sm_100a with nvcc.
 
-Usage: ``python -m kv_cache_vector_04_b200.build [--force] [--verbose]``.
+Usage: ``python kv_cache_vector_04_b200/build.py [--force] [--verbose]`` (run it by path:
+importing the package itself needs the library).
 The shared library is written next to this file so that it travels with the
 source tree; nothing is installed into site-packages.
 """

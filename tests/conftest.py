@@ -8,6 +8,19 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_library_if_stale():
+    # load the builder by path: importing the package requires the library
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_tq_build", os.path.join(ROOT, "kv_cache_vector_04_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_build_library_if_stale()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU statistics")
