@@ -33,7 +33,8 @@ TQ_DTYPE_BF16 = 1
 # every symbol include/tq.h declares
 EXPORTS = ("tq_init", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
            "tq_build_tables", "tq_quantize", "tq_attend_workspace", "tq_attend", "tq_scores",
-           "tq_status", "tq_copy", "tq_strerror")
+           "tq_attend_noalloc", "tq_status", "tq_copy", "tq_strerror")
+TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class TQError(RuntimeError):
@@ -72,6 +73,7 @@ def _load(path: str = LIB_PATH):
         "tq_attend_workspace": (I, [P, I, I, I, I, ctypes.POINTER(SZ)]),
         "tq_attend": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, P]),
         "tq_scores": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, P]),
+        "tq_attend_noalloc": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P]),
         "tq_status": (I, [P, ctypes.POINTER(ctypes.c_uint32)]),
         "tq_copy": (I, [P, P, SZ, P]),
         "tq_strerror": (ctypes.c_char_p, [I]),
@@ -272,6 +274,24 @@ def tq_scores(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor
         out = torch.empty((q.shape[0], q.shape[1], max_len), dtype=torch.float32, device=q.device)
     return _attend_like(_lib.tq_scores, "tq_scores", ctx, q, cache, seq_len, max_len, out,
                         workspace, stream)
+
+
+def tq_attend_noalloc(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor,
+                      max_len: int, out: torch.Tensor | None = None, stream=None):
+    """tq_attend with the library's static device scratch instead of a
+    workspace: for callers that cannot allocate device memory (see tq.h).
+    Overlapping calls on one GPU race on that scratch."""
+    if q.dim() != 3 or q.shape[2] != ctx.d:
+        raise ValueError("q must be [B, Hq, d] with d = %d" % ctx.d)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    B, Hq, _ = q.shape
+    c = cache.struct()
+    _check(_lib.tq_attend_noalloc(ctx.handle, _dev(q, "q"), _q_dtype(q), B, Hq, ctypes.byref(c),
+                                  _dev(seq_len, "seq_len", torch.int32), int(max_len),
+                                  _dev(out, "out", torch.float32),
+                                  ctypes.c_void_p(_stream_ptr(stream))), "tq_attend_noalloc")
+    return out
 
 
 def tq_status(ctx: Context) -> int:

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["api.cu", "quantize.cu", "attend.cu", "tables.cpp"]
+SOURCES = ["api.cu", "quantize.cu", "attend.cu", "noalloc.cu", "tables.cpp"]
 HEADERS = ["device_common.cuh", "kernels.h", "tables.h"]
 
 
