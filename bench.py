@@ -147,6 +147,27 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per attend_split launch from the committed ncu summary, if it
+    was taken on this workload and on the kernel source as it is now (else None)."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "attend_split_llama70b_32k.md")
+    src = os.path.join(ROOT, "kv_cache_vector_04_b200", "csrc", "attend.cu")
+    if workload != DEFAULT_WORKLOAD or not os.path.exists(prof):
+        return None
+    fields = {}
+    for line in open(prof, encoding="utf-8"):
+        if ":" in line and line.split(":", 1)[0].strip() in ("kernel_source_sha1",
+                                                             "dram_bytes_per_launch"):
+            key, val = line.split(":", 1)
+            fields[key.strip()] = val.split()[0]
+    with open(src, "rb") as f:
+        sha = hashlib.sha1(f.read()).hexdigest()
+    if fields.get("kernel_source_sha1") != sha or "dram_bytes_per_launch" not in fields:
+        return None
+    return int(fields["dram_bytes_per_launch"])
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -362,7 +383,10 @@ def run_tq(args, dist: Dist):
         "roofline": {"bound": "hbm", "kernel": "tq_attend (prologue + split + reduce launches)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
-                     "traffic": None,
+                     "traffic": profiled_traffic(w.name),
+                     "traffic_note": "dram read+write bytes of one attend_split launch (ncu, "
+                                     "profiles/attend_split_llama70b_32k.md); null when the "
+                                     "kernel source changed since",
                      "algorithmic_bytes_per_launch": bytes_attend,
                      "frac_of_same_run_copy_kernel": round(achieved / copy_gbs, 3)},
         "copy_kernel_gbs": round(copy_gbs, 1),

@@ -304,23 +304,25 @@ static double nearest_boundary_dist(double y, const float* bounds, int L)
     return best;
 }
 
-/* Normalise a fp16 vector: returns ||x|| and writes u = x / ||x|| (u = 0 for
- * the zero vector). */
-static double normalise(int d, const uint16_t* x, double* u)
+/* Rotated unit vector of a fp16 vector: y = Pi (x / ||x||), written as
+ * Pi x / ||x|| (the same value) so that a coordinate whose Walsh–Hadamard sum
+ * cancels exactly stays exactly 0 and meets the tie rule of the encoder.
+ * Returns ||x||; y = 0 for the zero vector. */
+static double rotate_unit(int d, const int8_t* D, const uint16_t* x, double* y)
 {
-    double ss = 0.0;
+    double xv[256], ss = 0.0;
     for (int i = 0; i < d; ++i) {
-        double v = oracle_half_to_double(x[i]);
-        u[i] = v;
-        ss += v * v;
+        xv[i] = oracle_half_to_double(x[i]);
+        ss += xv[i] * xv[i];
     }
     double n = sqrt(ss);
-    for (int i = 0; i < d; ++i) u[i] = (n > 0.0) ? u[i] / n : 0.0;
+    oracle_rotate(d, D, xv, y);
+    for (int i = 0; i < d; ++i) y[i] = (n > 0.0) ? y[i] / n : 0.0;
     return n;
 }
 
 /* Keys [MUNINN §30 秒懶人包 step 1 and 2; WISELY steps 1-3]:
- * u = x/||x||, y = Pi u, idx_i = encode(y_i) with the (B_K)-bit codebook,
+ * y = Pi (x/||x||), idx_i = encode(y_i) with the (B_K)-bit codebook,
  * r = y - c[idx], rho = ||r||, z = S r, sign bit s_j = [z_j >= 0].
  * Stores ||x|| and rho as fp16. ydist/zabs report how close each decision was
  * to its threshold (for counting boundary cases in parity tests). */
@@ -332,10 +334,9 @@ void oracle_quantize_keys(int d, int N, const uint16_t* x, const int8_t* D, cons
     int L = 1 << BK, m = d;
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; ++n) {
-        double u[256], y[256], r[256];
+        double y[256], r[256];
         uint8_t s0 = 0;
-        double nrm = normalise(d, x + (size_t)n * d, u);
-        oracle_rotate(d, D, u, y);
+        double nrm = rotate_unit(d, D, x + (size_t)n * d, y);
         double rr = 0.0;
         for (int i = 0; i < d; ++i) {
             int id = oracle_encode(y[i], tK, L);
@@ -365,10 +366,9 @@ void oracle_quantize_values(int d, int N, const uint16_t* x, const int8_t* D,
     (void)cV;
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; ++n) {
-        double u[256], y[256];
+        double y[256];
         uint8_t s0 = 0;
-        double nrm = normalise(d, x + (size_t)n * d, u);
-        oracle_rotate(d, D, u, y);
+        double nrm = rotate_unit(d, D, x + (size_t)n * d, y);
         for (int i = 0; i < d; ++i) {
             vidx[(size_t)n * d + i] = (uint8_t)oracle_encode(y[i], tV, L);
             if (ydist) ydist[(size_t)n * d + i] = nearest_boundary_dist(y[i], tV, L);

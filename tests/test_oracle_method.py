@@ -57,6 +57,22 @@ def test_quantize_keys_brute_force_small():
         assert out["rnorm"][n] == np.float16(np.linalg.norm(r)).view(np.uint16)
 
 
+def test_exact_cancellation_meets_the_tie_rule():
+    # D o x = (1, 1, 0, ...) gives Walsh-Hadamard sums 1 + (-1)^(i&1): every
+    # odd coordinate of the rotated vector is exactly 0, which the strict '>'
+    # rule puts in the cell below the middle boundary (which is exactly 0).
+    d, bits = 64, 3
+    tab = O.Tables(d, bits, seed=3)
+    x = np.zeros((1, d), np.float16)
+    x[0, 0] = tab.D[0]
+    x[0, 1] = tab.D[1]
+    out = O.quantize(tab, x, x)
+    L_k, L_v = 1 << tab.BK, 1 << tab.BV
+    assert np.all(out["kidx"][0, 1::2] == L_k // 2 - 1)
+    assert np.all(out["vidx"][0, 1::2] == L_v // 2 - 1)
+    assert np.all(out["kydist"][0, 1::2] == 0.0)
+
+
 def test_norm_saturation_flag():
     tab = O.Tables(64, 3, seed=1)
     x = np.full((2, 64), 60000.0, dtype=np.float16)

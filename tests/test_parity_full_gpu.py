@@ -1,0 +1,94 @@
+"""Full-size parity on sampled slices.
+
+Each workload's layer is drawn at its real size on the GPU and quantized
+there; the oracle recomputes sampled (batch, kv-head) streams from the same
+fp16 inputs, copied to the host, and every token's codes, signs and norms are
+compared. Attention then runs in the launch configuration the bench uses
+(every sequence and head, the full context) after the sampled streams of the
+cache are replaced by the oracle's packing of its own codes, so the GPU and
+the oracle attend over the same codes; every query head reading a sampled
+stream is compared.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_vector_04_b200 as tq
+from kv_cache_vector_04_b200 import inputs
+from oracle import oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_layer(w, samples, seq_fn=None):
+    """Quantize + attend one layer of workload `w` on the GPU, then check the
+    sampled (b, kv head) streams against the oracle."""
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    ctx = tq.tq_init(w.d, w.bits, 1)
+    tab = O.Tables(w.d, w.bits, 1)
+    k, v = inputs.kv_pair(w, w.N, layer=0, device=dev)
+    cache = tq.new_cache(ctx, w.B, w.Hkv, w.N)
+    tq.tq_quantize(ctx, k, v, torch.zeros(w.B, dtype=torch.int32, device=dev), cache)
+    assert tq.tq_status(ctx) == 0
+    host = cache.data.cpu().numpy()
+    lay = tq.tq_cache_layout(ctx)
+    per_stream = (cache.capacity // 16) * lay["tile_bytes"]
+    g = w.Hq // w.Hkv
+    stats = P.QuantStats()
+    oracle_streams = {}
+    for (b, h) in samples:
+        ora = O.quantize(tab, k[b, h].cpu().numpy(), v[b, h].cpu().numpy())
+        sb = P.stream_bytes(host, lay["tile_bytes"], cache.capacity, w.Hkv, b, h, w.N)
+        gpu = O.unpack_stream(w.d, w.bits, w.N, sb)
+        P.compare_stream(tab, gpu, ora, w.N, stats)
+        oracle_streams[(b, h)] = ora
+        packed = torch.from_numpy(O.pack_stream(w.d, w.bits, ora)).to(dev)
+        s0 = (b * w.Hkv + h) * per_stream
+        cache.data[s0: s0 + packed.numel()].copy_(packed)
+    stats.check()
+    del k, v
+    q = inputs.queries(w, device=dev)
+    seq = torch.full((w.B,), w.N, dtype=torch.int32) if seq_fn is None else seq_fn(w)
+    out = tq.tq_attend(ctx, q, cache, seq.to(dev), w.N).cpu().numpy().astype(np.float64)
+    assert tq.tq_status(ctx) == 0
+    qbits_all = P.q_bits(q.cpu())
+    for (b, h) in samples:
+        ora = oracle_streams[(b, h)]
+        n = int(seq[b])
+        codes = {key: ora[key][None, None] for key in ("kidx", "ksign", "knorm", "rnorm", "vidx",
+                                                      "vnorm")}
+        qb = np.ascontiguousarray(qbits_all[b:b + 1, h * g:(h + 1) * g])
+        ref = O.attend_batch(tab, qb, w.q_dtype == torch.bfloat16, codes,
+                             np.array([n], np.int32), 1)
+        err = P.attn_error(out[b:b + 1, h * g:(h + 1) * g], ref)
+        assert err.max() <= P.ATTN_TOL, (b, h, err.max())
+    return stats
+
+
+def test_llama70b_shaped_layer_32k():
+    # 16 sequences x 8 kv heads x 32768 tokens, K 3-bit + QJL, V 4-bit; 64 query heads
+    w = inputs.WORKLOADS["llama3.3-70b_decode_32k"]
+    _run_layer(w, samples=[(0, 0), (15, 7), (9, 3)])
+
+
+def test_qwen32b_shaped_layer_128k():
+    # one sequence x 8 kv heads x 131072 tokens, 3 bits, 2% spiky tokens; 40 query heads
+    w = inputs.WORKLOADS["qwen2.5-32b_prefill_decode_128k"]
+    _run_layer(w, samples=[(0, 2)])
+
+
+def test_qwen3b_shaped_layer_8k():
+    # one sequence x 2 kv heads x 8192 tokens, 3 bits, outlier channels x15
+    w = inputs.WORKLOADS["qwen2.5-3b_decode_8k"]
+    _run_layer(w, samples=[(0, 0), (0, 1)])
+
+
+@pytest.mark.parametrize("name", ["sweep_d64_b2_n65536", "sweep_d256_b4_n65536",
+                                  "sweep_d128_b3_n16384", "sweep_d256_b2_n4096"])
+def test_sweep_points(name):
+    w = {x.name: x for x in inputs.sweep_workloads()}[name]
+    # unequal lengths across the batch
+    _run_layer(w, samples=[(7, 5)],
+               seq_fn=lambda w: torch.tensor([w.N - 37 * i for i in range(w.B)], dtype=torch.int32))
