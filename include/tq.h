@@ -172,8 +172,9 @@ int tq_attend_workspace(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_len, 
  *            dequantized values (zero when seq_len[b] = 0).
  *  workspace: device scratch of at least tq_attend_workspace(...) bytes,
  *            256-byte aligned; its contents need no initialisation.
- * Three launches on `stream`: query prologue (Pi q, S Pi q), split kernel,
- * cross-split reduction with the inverse rotation. */
+ * Three launches on `stream`: the query prologue (Pi q, S Pi q for each group
+ * of 8 query heads), the split kernel, and the cross-split reduction with the
+ * inverse rotation. */
 int tq_attend(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,
               const int32_t* seq_len, int max_len, float* out, void* workspace,
               size_t workspace_bytes, void* stream);

@@ -9,8 +9,9 @@
 // per output: o = Pi^T sum_n softmax(l)_n |v_n| cV[vidx_n].
 //
 // Three kernels:
-//  prologue  q~ = H (D o q) / sqrt(d) and p = S q~ per query head, written as
-//            fp16 m16n8k16 B fragments (log2(e) and the norms' scales folded in);
+//  prologue  q~ = H (D o q) / sqrt(d) and p = S q~ per group of 8 query heads,
+//            written as fp16 m16n8k16 B fragments (hi/lo; log2(e) and the
+//            norms' scales folded in);
 //  split     one CTA per (batch, kv head, group of 8 query heads, context
 //            split); each warp streams 16-token tiles with 128-bit loads of its
 //            own lane string, decodes codes to fp16 tensor-core A fragments
@@ -92,80 +93,134 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q)
 }
 
 // ---------------------------------------------------------------- prologue
-// Per query head: q~ = H (D o q) / sqrt(d), p = S q~, and the fp16 B fragments
-// of [log2(e) 2^7 q~ / (d alpha)] and [log2(e) 2^7 kappa p / sqrt(d)], each as
-// a hi part and a lo part (x - hi), so that the two tensor-core products
-// carry ~22 significant bits. alpha is the scale that makes the key codebook
-// almost exact in fp16 (chosen on the host).
+// One CTA per (batch, kv head, group of 8 query heads): q~ = H (D o q) / sqrt(d)
+// and p = S q~ for the 8 heads (S is read once per CTA), written as the fp16 B
+// fragments of [log2(e) 2^7 q~ / (d alpha)] and [log2(e) 2^7 kappa p / sqrt(d)],
+// each as a hi part and a lo part (x - hi), so that the two tensor-core
+// products carry ~22 significant bits. alpha is the scale that makes the key
+// codebook almost exact in fp16 (chosen on the host).
 template <int D>
-__global__ void __launch_bounds__(D) attend_prologue(DevTables tb, AttendArgs a)
+__global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArgs a)
 {
-    __shared__ float qs[D];
-    __shared__ float bc[D], bs[D];
-    const int b = blockIdx.y;
-    const int unit = blockIdx.x >> 3, col = blockIdx.x & 7;
-    const int groups = a.plan.groups;
-    const int ratio = a.Hq / a.Hkv;
+    constexpr int NT = 2 * D;
+    __shared__ float qt[D][8];          // rotated queries, [coordinate][head]
+    __shared__ float pp[2][D][8];       // p = S q~, two partial halves over k
+    const int unit = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int groups = a.plan.groups, ratio = a.Hq / a.Hkv;
     const int hkv = unit / groups, grp = unit % groups;
-    const int j = grp * 8 + col;
-    const int i = threadIdx.x;
-    const bool live = j < ratio;   // block-uniform
-    float vc = 0.f, vs = 0.f;
-    if (live) {
-        const int hq = hkv * ratio + j;
-        const size_t off = ((size_t)b * a.Hq + hq) * D + i;
-        float x;
-        if (a.q_bf16)
-            x = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[off]);
-        else
-            x = __half2float(reinterpret_cast<const __half*>(a.q)[off]);
-        qs[i] = x * tb.signs[i];
-        __syncthreads();
-#pragma unroll
-        for (int s = 1; s < D; s <<= 1) {
-            const float mine = qs[i], other = qs[i ^ s];
-            __syncthreads();
-            qs[i] = (i & s) ? (other - mine) : (mine + other);
-            __syncthreads();
+    const size_t units = (size_t)a.Hkv * groups;
+
+    for (int e = tid; e < 8 * D; e += NT) {
+        const int h = e / D, i = e % D, j = grp * 8 + h;
+        float x = 0.f;
+        if (j < ratio) {
+            const size_t off = ((size_t)b * a.Hq + hkv * ratio + j) * D + i;
+            x = a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[off])
+                         : __half2float(reinterpret_cast<const __half*>(a.q)[off]);
+            x *= tb.signs[i];
         }
-        const float qt = qs[i] * rsqrtf((float)D);
-        __syncthreads();
-        qs[i] = qt;
-        __syncthreads();
-        float p = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < D; ++k) p = fmaf(tb.s_t[(size_t)k * D + i], qs[k], p);
-        vc = qt * (kLog2e * 128.0f / ((float)D * tb.alpha_k));
-        vs = p * (kLog2e * 128.0f * 1.2533141373155003f / ((float)D * sqrtf((float)D)));
+        qt[i][h] = x;
     }
-    bc[i] = vc;
-    bs[i] = vs;
     __syncthreads();
-    if (i < D / 4) {
-        const int kk = i >> 2, t = i & 3;
+#pragma unroll 1
+    for (int st = 1; st < D; st <<= 1) {            // Walsh-Hadamard butterflies, 8 heads
+        for (int e = tid; e < 4 * D; e += NT) {
+            const int h = e & 7, bf = e >> 3;
+            const int i = (bf / st) * 2 * st + (bf % st);
+            const float x0 = qt[i][h], x1 = qt[i + st][h];
+            qt[i][h] = x0 + x1;
+            qt[i + st][h] = x0 - x1;
+        }
+        __syncthreads();
+    }
+    const float rs = rsqrtf((float)D);
+    for (int e = tid; e < 8 * D; e += NT) (&qt[0][0])[e] *= rs;
+    __syncthreads();
+    {
+        const int j = tid % D, half = tid / D;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const int k0 = half * (D / 2);
+#pragma unroll 4
+        for (int k = k0; k < k0 + D / 2; ++k) {
+            const float sv = __ldg(tb.s_t + (size_t)k * D + j);
+            const float4 q0 = *reinterpret_cast<const float4*>(&qt[k][0]);
+            const float4 q1 = *reinterpret_cast<const float4*>(&qt[k][4]);
+            acc[0] = fmaf(sv, q0.x, acc[0]); acc[1] = fmaf(sv, q0.y, acc[1]);
+            acc[2] = fmaf(sv, q0.z, acc[2]); acc[3] = fmaf(sv, q0.w, acc[3]);
+            acc[4] = fmaf(sv, q1.x, acc[4]); acc[5] = fmaf(sv, q1.y, acc[5]);
+            acc[6] = fmaf(sv, q1.z, acc[6]); acc[7] = fmaf(sv, q1.w, acc[7]);
+        }
+#pragma unroll
+        for (int h = 0; h < 8; ++h) pp[half][j][h] = acc[h];
+    }
+    __syncthreads();
+    {
+        // one fragment entry (k-step, thread-in-group, head column) per thread
+        const int e = tid, col = e & 7, t = (e >> 3) & 3, kk = e >> 5;
         const int c0 = 16 * kk + 2 * t;
         const int idx[4] = {c0, c0 + 1, c0 + 8, c0 + 9};
+        const float scale_c = kLog2e * 128.0f / ((float)D * tb.alpha_k);
+        const float scale_s = kLog2e * 128.0f * 1.2533141373155003f / ((float)D * sqrtf((float)D));
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const float* src = q ? bs : bc;
-            float h[4], l[4];
+            float hv[4], lv[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                h[e] = __half2float(__float2half_rn(src[idx[e]]));
-                l[e] = src[idx[e]] - h[e];
+            for (int u = 0; u < 4; ++u) {
+                const float x = q ? (pp[0][idx[u]][col] + pp[1][idx[u]][col]) * scale_s
+                                  : qt[idx[u]][col] * scale_c;
+                hv[u] = __half2float(__float2half_rn(x));
+                lv[u] = x - hv[u];
             }
-            hi[2 * q] = pack_half2(h[0], h[1]);
-            hi[2 * q + 1] = pack_half2(h[2], h[3]);
-            lo[2 * q] = pack_half2(l[0], l[1]);
-            lo[2 * q + 1] = pack_half2(l[2], l[3]);
+            hi[2 * q] = pack_half2(hv[0], hv[1]);
+            hi[2 * q + 1] = pack_half2(hv[2], hv[3]);
+            lo[2 * q] = pack_half2(lv[0], lv[1]);
+            lo[2 * q + 1] = pack_half2(lv[2], lv[3]);
         }
-        const size_t units = (size_t)a.Hkv * groups;
         uint4* dst = reinterpret_cast<uint4*>(a.qfrag) +
                      (((size_t)b * units + unit) * (D / 16) + kk) * 64 + col * 4 + t;
         dst[0] = make_uint4(hi[0], hi[1], lo[0], lo[1]);    // codebook term: b0,b1 hi; b0,b1 lo
         dst[32] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
     }
+}
+
+// ---------------------------------------------------------------- reduction
+template <int D>
+__global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
+{
+    __shared__ float os[D];
+    const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+    const int ratio = a.Hq / a.Hkv, groups = a.plan.groups;
+    const int hkv = hq / ratio, j = hq % ratio, grp = j >> 3, col = j & 7;
+    const size_t units = (size_t)a.Hkv * groups;
+    const size_t unit = (size_t)hkv * groups + grp;
+    constexpr int RS = D + 2;
+    const float* P = a.partial + ((size_t)b * units + unit) * a.plan.nsplit * 8 * RS + col * RS;
+    const int ns = a.plan.nsplit;
+    float M = -CUDART_INF_F;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, P[(size_t)s * 8 * RS]);
+    float L = 0.f, acc = 0.f;
+    if (M != -CUDART_INF_F) {
+        for (int s = 0; s < ns; ++s) {
+            const float* ps = P + (size_t)s * 8 * RS;
+            const float ms = ps[0];
+            if (ms == -CUDART_INF_F) continue;
+            const float f = exp2f(ms - M);
+            L = fmaf(ps[1], f, L);
+            acc = fmaf(ps[2 + i], f, acc);
+        }
+    }
+    os[i] = (L > 0.f) ? acc / L : 0.f;
+    __syncthreads();
+#pragma unroll
+    for (int s = 1; s < D; s <<= 1) {
+        const float mine = os[i], other = os[i ^ s];
+        __syncthreads();
+        os[i] = (i & s) ? (other - mine) : (mine + other);
+        __syncthreads();
+    }
+    // Pi^T = D H / sqrt(d), and the value table carries a factor sqrt(d)
+    a.out[((size_t)b * a.Hq + hq) * D + i] = os[i] * tb.signs[i] * (1.0f / (float)D);
 }
 
 // ---------------------------------------------------------------- split kernel
@@ -529,45 +584,6 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
     }
 }
 
-// ---------------------------------------------------------------- reduction
-template <int D>
-__global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
-{
-    __shared__ float os[D];
-    const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
-    const int ratio = a.Hq / a.Hkv, groups = a.plan.groups;
-    const int hkv = hq / ratio, j = hq % ratio, grp = j >> 3, col = j & 7;
-    const size_t units = (size_t)a.Hkv * groups;
-    const size_t unit = (size_t)hkv * groups + grp;
-    constexpr int RS = D + 2;
-    const float* P = a.partial + ((size_t)b * units + unit) * a.plan.nsplit * 8 * RS + col * RS;
-    const int ns = a.plan.nsplit;
-    float M = -CUDART_INF_F;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, P[(size_t)s * 8 * RS]);
-    float L = 0.f, acc = 0.f;
-    if (M != -CUDART_INF_F) {
-        for (int s = 0; s < ns; ++s) {
-            const float* ps = P + (size_t)s * 8 * RS;
-            const float ms = ps[0];
-            if (ms == -CUDART_INF_F) continue;
-            const float f = exp2f(ms - M);
-            L = fmaf(ps[1], f, L);
-            acc = fmaf(ps[2 + i], f, acc);
-        }
-    }
-    os[i] = (L > 0.f) ? acc / L : 0.f;
-    __syncthreads();
-#pragma unroll
-    for (int s = 1; s < D; s <<= 1) {
-        const float mine = os[i], other = os[i ^ s];
-        __syncthreads();
-        os[i] = (i & s) ? (other - mine) : (mine + other);
-        __syncthreads();
-    }
-    // Pi^T = D H / sqrt(d), and the value table carries a factor sqrt(d)
-    a.out[((size_t)b * a.Hq + hq) * D + i] = os[i] * tb.signs[i] * (1.0f / (float)D);
-}
-
 // cudaFuncSetAttribute once per (kernel, device).
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long& done_mask)
@@ -588,7 +604,7 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
     using Tr = AttTraits<D, BITS>;
     static unsigned long long done_scores = 0, done_attend = 0;
     const int units = a.Hkv * a.plan.groups;
-    attend_prologue<D><<<dim3(units * 8, a.B), D, 0, st>>>(tb, a);
+    attend_prologue<D><<<dim3(units, a.B), 2 * D, 0, st>>>(tb, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const dim3 grid(a.plan.nsplit, units, a.B);
