@@ -56,6 +56,8 @@ extern "C" {
 #define TQ_STATUS_CAPACITY 0x1u  /* tq_quantize: start_pos < 0 or start_pos+T > capacity; batch item skipped */
 #define TQ_STATUS_SEQ_LEN 0x2u   /* tq_attend/tq_scores: seq_len < 0 or > min(max_len, capacity); clamped */
 #define TQ_STATUS_NORM_SAT 0x4u  /* tq_quantize: a norm exceeded 65504 and was stored as 65504 */
+#define TQ_STATUS_WAIT_TIMEOUT 0x8u /* tq_attend: a copy into shared memory did not complete within the
+                                     * kernel's bounded wait; that call's output is unspecified */
 
 #define TQ_TILE 16 /* tokens per packed tile */
 

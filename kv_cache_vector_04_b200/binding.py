@@ -26,6 +26,7 @@ TQ_ERR_DEVICE = -5
 TQ_STATUS_CAPACITY = 0x1
 TQ_STATUS_SEQ_LEN = 0x2
 TQ_STATUS_NORM_SAT = 0x4
+TQ_STATUS_WAIT_TIMEOUT = 0x8
 TQ_TILE = 16
 TQ_DTYPE_F16 = 0
 TQ_DTYPE_BF16 = 1

@@ -189,7 +189,9 @@ int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const 
     a.max_len = max_len;
     a.tile_bytes = make_layout(ctx->d, ctx->bits).tile_bytes;
     a.qfrag = static_cast<uint32_t*>(ws);
-    a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(plan.qfrag_bytes));
+    a.prefix = reinterpret_cast<long long*>(static_cast<uint8_t*>(ws) + align256(plan.qfrag_bytes));
+    a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(plan.qfrag_bytes) +
+                                         align256(plan.prefix_bytes));
     a.out = out;
     a.plan = plan;
     const cudaError_t e = tq::launch_attend(ctx->d, ctx->bits, ctx->tables, a, scores,

@@ -21,7 +21,7 @@
 //                      [16 tok x m] x [m x 8 heads]  (QJL sign term)
 //              PV:     [d x 16 tok] x [16 tok x 8 heads]
 //            on mma.sync with fp32 accumulation, with an online softmax per
-//            head in registers; the 4 warps of a CTA merge in shared memory;
+//            head in registers; the 8 warps of a CTA merge in shared memory;
 //  reduce    merges the splits per query head and applies Pi^T (fp32 WHT).
 // Operands come from registers because every A fragment is decoded on the
 // fly; the contraction is skinny (N = 8 heads), so the legacy register-fed
@@ -48,14 +48,19 @@ struct AttTraits {
     static constexpr int KK = D / 16;                        // k-steps / coordinate blocks
     static constexpr int NLK = 1 << KF, NLV = 1 << VF;       // LUT entries
     static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
-    static constexpr size_t MERGE_BYTES = (size_t)4 * 8 * (D + 2) * 4;
-    // cp.async staging ring: per warp STAGES copies of {32 lane strings, 32 K-norm
-    // and 32 V-norm copies}; each lane stages and reads back only its own bytes
+    // d <= 128: CTAs of 4 warps, 3 per SM, query fragments in registers;
+    // d = 256: CTAs of 8 warps, 1 per SM, query fragments in shared memory
+    static constexpr bool QREG = D <= 128;
+    static constexpr int WARPS = QREG ? 4 : 8, NT = 32 * WARPS, CTAS_PER_SM = QREG ? 3 : 1;
+    static constexpr size_t MERGE_BYTES = (size_t)WARPS * 8 * (D + 2) * 4;
+    // staging ring: per warp STAGES images of whole tiles, each brought in by
+    // one bulk copy
     static constexpr int STAGES = 3;
     static constexpr int NCH = BITS * D / 8 / CB;
-    static constexpr int STAGE_BYTES = NCH * 32 * CB + 32 * 8 + 32 * 4;
-    static constexpr size_t RING_BYTES = (size_t)4 * STAGES * STAGE_BYTES;
-    static constexpr size_t QF_SMEM = D <= 128 ? 0 : QF_BYTES;      // d = 256 keeps B in smem
+    static constexpr int TILE_BYTES = 16 * (BITS * D / 4 + 6);
+    static constexpr int STAGE_BYTES = TILE_BYTES;
+    static constexpr size_t RING_BYTES = (size_t)WARPS * STAGES * STAGE_BYTES;
+    static constexpr size_t QF_SMEM = QREG ? 0 : QF_BYTES;
     static constexpr size_t LOOP_BYTES = RING_BYTES + QF_SMEM;
     static constexpr size_t DYN_SMEM = LOOP_BYTES > MERGE_BYTES ? LOOP_BYTES : MERGE_BYTES;
 };
@@ -84,15 +89,51 @@ __device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t byt
     return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(table) + byte_off);
 }
 
-// fp16x2 (+1/-1, +1/-1) from sign pair p: element 0 at bit p%16, element 1 at
-// bit 16 + p%16 of sign word p/16 (bit 1 = +1).
-__device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q)
+// fp16x2 (+-rho, +-rho) from sign pair p: element 0 at bit p%16, element 1 at
+// bit 16 + p%16 of sign word p/16 (bit 1 = +); nrho2 holds -rho in both halves.
+// The residual norm rho rides on the sign operand, so the QJL products land in
+// the same accumulators as the codebook products.
+__device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q, uint32_t nrho2)
 {
     const uint32_t x = word << (15 - q);
-    return (x & 0x80008000u) ^ 0xBC00BC00u;
+    return (x & 0x80008000u) ^ nrho2;
 }
 
 // ---------------------------------------------------------------- prologue
+// Warp 0 of CTA (0, 0) also lays the units' tiles end to end for the split
+// kernel: prefix[b] = sum over sequences b' < b of ceil(seq'/16) x units per
+// sequence (seq clamped to [0, min(max_len, capacity)], flagging a clamp),
+// prefix[B] = the total.
+__device__ __forceinline__ void tile_prefix(const DevTables& tb, const AttendArgs& a, int lane)
+{
+    const int lim = min(a.max_len, a.capacity);
+    const long long upb = (long long)a.Hkv * a.plan.groups;
+    long long run = 0;
+    bool bad = false;
+    for (int b0 = 0; b0 < a.B; b0 += 32) {
+        const int b = b0 + lane;
+        long long v = 0;
+        if (b < a.B) {
+            int s = a.seq_len[b];
+            if (s < 0 || s > lim) {
+                bad = true;
+                s = min(max(s, 0), lim);
+            }
+            v = (long long)((s + 15) >> 4) * upb;
+        }
+        long long incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (b < a.B) a.prefix[b] = run + incl - v;
+        run += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) a.prefix[a.B] = run;
+    if (__any_sync(kFull, bad) && lane == 0) atomicOr(tb.status, TQ_STATUS_SEQ_LEN);
+}
+
 // One CTA per (batch, kv head, group of 8 query heads): q~ = H (D o q) / sqrt(d)
 // and p = S q~ for the 8 heads (S is read once per CTA), written as the fp16 B
 // fragments of [log2(e) 2^7 q~ / (d alpha)] and [log2(e) 2^7 kappa p / sqrt(d)],
@@ -109,6 +150,7 @@ __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArg
     const int groups = a.plan.groups, ratio = a.Hq / a.Hkv;
     const int hkv = unit / groups, grp = unit % groups;
     const size_t units = (size_t)a.Hkv * groups;
+    if (unit == 0 && b == 0 && tid < 32) tile_prefix(tb, a, tid);
 
     for (int e = tid; e < 8 * D; e += NT) {
         const int h = e / D, i = e % D, j = grp * 8 + h;
@@ -185,29 +227,41 @@ __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArg
 }
 
 // ---------------------------------------------------------------- reduction
+// One CTA per (query head, batch): merges the partials of the CTAs whose
+// ranges cover the head's unit (the range of CTA c is [c W / G, (c+1) W / G)
+// of the W tiles, so tile x lies in CTA ((x + 1) G - 1) / W), then applies
+// Pi^T with an fp32 Walsh-Hadamard transform.
 template <int D>
 __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
 {
     __shared__ float os[D];
     const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
     const int ratio = a.Hq / a.Hkv, groups = a.plan.groups;
-    const int hkv = hq / ratio, j = hq % ratio, grp = j >> 3, col = j & 7;
-    const size_t units = (size_t)a.Hkv * groups;
-    const size_t unit = (size_t)hkv * groups + grp;
+    const int hkv = hq / ratio, jh = hq % ratio, grp = jh >> 3, col = jh & 7;
+    const int upb = a.Hkv * groups, ju = hkv * groups + grp;
+    const size_t u = (size_t)b * upb + ju;
     constexpr int RS = D + 2;
-    const float* P = a.partial + ((size_t)b * units + unit) * a.plan.nsplit * 8 * RS + col * RS;
-    const int ns = a.plan.nsplit;
-    float M = -CUDART_INF_F;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, P[(size_t)s * 8 * RS]);
-    float L = 0.f, acc = 0.f;
-    if (M != -CUDART_INF_F) {
-        for (int s = 0; s < ns; ++s) {
-            const float* ps = P + (size_t)s * 8 * RS;
-            const float ms = ps[0];
-            if (ms == -CUDART_INF_F) continue;
-            const float f = exp2f(ms - M);
-            L = fmaf(ps[1], f, L);
-            acc = fmaf(ps[2 + i], f, acc);
+    const long long W = a.prefix[a.B], pb = a.prefix[b];
+    const long long T = (a.prefix[b + 1] - pb) / upb;
+    const long long G = a.plan.ctas;
+    float M = -CUDART_INF_F, L = 0.f, acc = 0.f;
+    if (T > 0) {
+        const long long U0 = pb + ju * T, U1 = U0 + T;
+        const int cf = (int)(((U0 + 1) * G - 1) / W), cl = (int)((U1 * G - 1) / W);
+        for (int c = cf; c <= cl; ++c) {
+            if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;   // empty range
+            M = fmaxf(M, a.partial[((size_t)c + u) * 8 * RS + col * RS]);
+        }
+        if (M != -CUDART_INF_F) {
+            for (int c = cf; c <= cl; ++c) {
+                if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;
+                const float* ps = a.partial + ((size_t)c + u) * 8 * RS + col * RS;
+                const float ms = ps[0];
+                if (ms == -CUDART_INF_F) continue;
+                const float f = exp2f(ms - M);
+                L = fmaf(ps[1], f, L);
+                acc = fmaf(ps[2 + i], f, acc);
+            }
         }
     }
     os[i] = (L > 0.f) ? acc / L : 0.f;
@@ -224,21 +278,49 @@ __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
 }
 
 // ---------------------------------------------------------------- split kernel
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
+// mbarrier + bulk-copy helpers (shared addresses are 32-bit).
+constexpr int kWaitLimit = 1 << 22;   // bounded waits: give up and flag TQ_STATUS_WAIT_TIMEOUT
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src)
+__device__ __forceinline__ void fence_mbar_init()
 {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(src) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src)
+// Orders this thread's earlier generic-proxy accesses of shared memory before
+// later async-proxy (bulk copy) writes to it.
+__device__ __forceinline__ void fence_proxy_async()
 {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+// One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from global memory into this CTA's shared memory, completing on `bar`,
+// whose expected transaction count is raised by the same amount.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// Wait for phase `parity` of `bar` to complete; false after kWaitLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    for (int i = 0; i < kWaitLimit; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
 
 template <int D, int BITS>
 struct TileData {
@@ -267,25 +349,8 @@ __device__ __forceinline__ void load_tile(const uint8_t* tp, int lane, int g, Ti
     td.vn = __ldcs(reinterpret_cast<const uint32_t*>(tp + 4 * BITS * D + 64 + 4 * g));
 }
 
-// Stage this lane's bytes of tile `tp` into ring slot `slot` (shared address).
-template <int D, int BITS>
-__device__ __forceinline__ void stage_tile(uint32_t slot, const uint8_t* tp, int lane, int g)
-{
-    using Tr = AttTraits<D, BITS>;
-#pragma unroll
-    for (int c = 0; c < Tr::NCH; ++c) {
-        const uint32_t off = (uint32_t)(c * 32 + lane) * Tr::CB;
-        if constexpr (Tr::CB == 16)
-            cp_async16(slot + off, tp + off);
-        else
-            cp_async8(slot + off, tp + off);
-    }
-    constexpr uint32_t nb = Tr::NCH * 32 * Tr::CB;
-    cp_async8(slot + nb + 8u * lane, tp + 4 * BITS * D + 8 * g);
-    cp_async4(slot + nb + 256u + 4u * lane, tp + 4 * BITS * D + 64 + 4 * g);
-}
-
-// Read back this lane's bytes of a staged tile.
+// Read this lane's bytes of a tile image in shared memory (the image has the
+// cache's own layout: chunk-major lane strings, then K norms, then V norms).
 template <int D, int BITS>
 __device__ __forceinline__ void read_stage(const uint8_t* slot, int lane, TileData<D, BITS>& td)
 {
@@ -301,22 +366,24 @@ __device__ __forceinline__ void read_stage(const uint8_t* slot, int lane, TileDa
             td.s[2 * c] = v.x; td.s[2 * c + 1] = v.y;
         }
     }
-    constexpr int nb = Tr::NCH * 32 * Tr::CB;
-    td.kn = *reinterpret_cast<const uint2*>(slot + nb + 8 * lane);
-    td.vn = *reinterpret_cast<const uint32_t*>(slot + nb + 256 + 4 * lane);
+    constexpr int nb = 4 * BITS * D;
+    const int g = lane >> 2;
+    td.kn = *reinterpret_cast<const uint2*>(slot + nb + 8 * g);
+    td.vn = *reinterpret_cast<const uint32_t*>(slot + nb + 64 + 4 * g);
 }
 
 // Query B fragments of one k-step: x,y = hi (b0, b1), z,w = lo, for the
-// codebook term (c) and the QJL term (s). Kept in registers for d <= 128
-// (they do not change from tile to tile), in shared memory for d = 256.
-template <int KK, bool IN_REGS>
+// codebook term (c) and the QJL term (s). Held in registers (they do not
+// change from tile to tile) or, where registers are short, in shared memory.
+template <int KK, int NT, bool IN_REGS>
 struct QueryFrags;
 
-template <int KK>
-struct QueryFrags<KK, true> {
+template <int KK, int NT>
+struct QueryFrags<KK, NT, true> {
     uint4 c[KK], s[KK];
-    __device__ __forceinline__ void load(const uint4* src, uint4*, int lane, int)
+    __device__ __forceinline__ void load(const uint4* src, uint4*, int tid)
     {
+        const int lane = tid & 31;
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk) {
             c[kk] = src[kk * 64 + lane];
@@ -327,12 +394,12 @@ struct QueryFrags<KK, true> {
     __device__ __forceinline__ uint4 fs(int kk, int) const { return s[kk]; }
 };
 
-template <int KK>
-struct QueryFrags<KK, false> {
+template <int KK, int NT>
+struct QueryFrags<KK, NT, false> {
     const uint4* sm;
-    __device__ __forceinline__ void load(const uint4* src, uint4* smem, int, int tid)
+    __device__ __forceinline__ void load(const uint4* src, uint4* smem, int tid)
     {
-        for (int e = tid; e < KK * 64; e += 128) smem[e] = src[e];
+        for (int e = tid; e < KK * 64; e += NT) smem[e] = src[e];
         sm = smem;
     }
     __device__ __forceinline__ uint4 fc(int kk, int lane) const { return sm[kk * 64 + lane]; }
@@ -351,9 +418,12 @@ __device__ __forceinline__ void tile_logits(const TileData<D, BITS>& td, const Q
                                             const uint32_t* lutk, uint32_t lane4, float (&L)[4])
 {
     using Tr = AttTraits<D, BITS>;
-    // four independent accumulation chains: codebook hi/lo, QJL hi/lo
-    float ch[4] = {0.f, 0.f, 0.f, 0.f}, cl[4] = {0.f, 0.f, 0.f, 0.f};
-    float sh[4] = {0.f, 0.f, 0.f, 0.f}, sl[4] = {0.f, 0.f, 0.f, 0.f};
+    // -rho of tokens g and g+8 in both fp16 halves (A rows g and g+8)
+    const uint32_t nr_g = __byte_perm(td.kn.x, 0u, 0x3232) | 0x80008000u;
+    const uint32_t nr_h = __byte_perm(td.kn.y, 0u, 0x3232) | 0x80008000u;
+    // two accumulation chains: hi and lo parts of the B operands; each takes
+    // the codebook product and the rho-weighted QJL product of every k-step
+    float ah[4], al[4];
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
         const uint4 bc = qf.fc(kk, lane);
@@ -363,22 +433,25 @@ __device__ __forceinline__ void tile_logits(const TileData<D, BITS>& td, const Q
         for (int r = 0; r < 4; ++r) {
             const int p = 4 * kk + r;
             ak[r] = lut_load(lutk, lut_off(td.s, Tr::KF * p, Tr::KF, lane4));
-            as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15);
+            as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
         }
-        mma_16816(ch, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
-        mma_16816(cl, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
-        mma_16816(sh, as[0], as[1], as[2], as[3], bs.x, bs.y);
-        mma_16816(sl, as[0], as[1], as[2], as[3], bs.z, bs.w);
+        if (kk == 0) {
+            mma_16816_first(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
+            mma_16816_first(al, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+        } else {
+            mma_16816(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
+            mma_16816(al, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+        }
+        mma_16816(ah, as[0], as[1], as[2], as[3], bs.x, bs.y);
+        mma_16816(al, as[0], as[1], as[2], as[3], bs.z, bs.w);
     }
-    const float kn_g = half_bits_to_float((uint16_t)(td.kn.x & 0xffff)) * (1.0f / 128.0f);
-    const float rho_g = half_bits_to_float((uint16_t)(td.kn.x >> 16));
-    const float kn_h = half_bits_to_float((uint16_t)(td.kn.y & 0xffff)) * (1.0f / 128.0f);
-    const float rho_h = half_bits_to_float((uint16_t)(td.kn.y >> 16));
-    // the B operands carry a factor 2^7
-    L[0] = kn_g * fmaf(rho_g, sh[0] + sl[0], ch[0] + cl[0]);
-    L[1] = kn_g * fmaf(rho_g, sh[1] + sl[1], ch[1] + cl[1]);
-    L[2] = kn_h * fmaf(rho_h, sh[2] + sl[2], ch[2] + cl[2]);
-    L[3] = kn_h * fmaf(rho_h, sh[3] + sl[3], ch[3] + cl[3]);
+    // |k| of tokens g and g+8 (fp16, low halves); the B operands carry 2^7
+    const float kn_g = __low2float(*reinterpret_cast<const __half2*>(&td.kn.x)) * (1.0f / 128.0f);
+    const float kn_h = __low2float(*reinterpret_cast<const __half2*>(&td.kn.y)) * (1.0f / 128.0f);
+    L[0] = kn_g * (ah[0] + al[0]);
+    L[1] = kn_g * (ah[1] + al[1]);
+    L[2] = kn_h * (ah[2] + al[2]);
+    L[3] = kn_h * (ah[3] + al[3]);
 }
 
 // Online-softmax update and P V for one tile.
@@ -400,7 +473,7 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, BITS>& td, flo
             mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
         }
         const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
-        const float al0 = exp2f(st.m0 - mn0), al1 = exp2f(st.m1 - mn1);
+        const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
         st.l0 *= al0;
         st.l1 *= al1;
 #pragma unroll
@@ -413,13 +486,14 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, BITS>& td, flo
         st.m0 = mn0;
         st.m1 = mn1;
     }
-    const float p0 = exp2f(L[0] - st.m0), p1 = exp2f(L[1] - st.m1);
-    const float p2 = exp2f(L[2] - st.m0), p3 = exp2f(L[3] - st.m1);
+    const float p0 = fast_exp2(L[0] - st.m0), p1 = fast_exp2(L[1] - st.m1);
+    const float p2 = fast_exp2(L[2] - st.m0), p3 = fast_exp2(L[3] - st.m1);
     st.l0 += p0 + p2;
     st.l1 += p1 + p3;
     // slots past seq_len may hold anything (even NaN norms): select, never multiply
-    const float vn_g = v0 ? half_bits_to_float((uint16_t)(td.vn & 0xffff)) : 0.f;
-    const float vn_h = v1 ? half_bits_to_float((uint16_t)(td.vn >> 16)) : 0.f;
+    const float2 vnf = __half22float2(*reinterpret_cast<const __half2*>(&td.vn));
+    const float vn_g = v0 ? vnf.x : 0.f;
+    const float vn_h = v1 ? vnf.y : 0.f;
     const uint32_t b0 = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
     const uint32_t b1 = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
 #pragma unroll
@@ -432,18 +506,26 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, BITS>& td, flo
     }
 }
 
-template <int D, int BITS, bool SCORES>
-__global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables tb, AttendArgs a)
+// Fill the lane-replicated decode tables of a CTA of NT threads.
+template <int D, int BITS, int NT>
+__device__ __forceinline__ void fill_luts(const DevTables& tb, uint32_t* lutk, uint32_t* lutv, int tid)
 {
     using Tr = AttTraits<D, BITS>;
-    constexpr int KK = Tr::KK;
-    constexpr bool kRegQ = D <= 128;
-    // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l, so
-    // the 32 lanes of a warp always hit 32 different banks.
+    for (int e = tid; e < Tr::NLK * 32; e += NT) lutk[e] = __ldg(tb.lut_k + (e >> 5));
+    for (int e = tid; e < Tr::NLV * 32; e += NT) lutv[e] = __ldg(tb.lut_v + (e >> 5));
+}
+
+// Estimated logits alone: one CTA per (batch, kv head, group of 8 query heads,
+// context split), every tile up to max_len, -inf past seq_len.
+template <int D, int BITS>
+__global__ void __launch_bounds__(AttTraits<D, BITS>::NT, AttTraits<D, BITS>::CTAS_PER_SM)
+    attend_scores(DevTables tb, AttendArgs a)
+{
+    using Tr = AttTraits<D, BITS>;
+    constexpr int KK = Tr::KK, WARPS = Tr::WARPS, NT = Tr::NT;
     __shared__ __align__(16) uint32_t lutv[Tr::NLV * 32];
     __shared__ __align__(16) uint32_t lutk[Tr::NLK * 32];
     extern __shared__ uint4 dyn_smem[];
-    float* mrg = reinterpret_cast<float*>(dyn_smem);       // [4][8][D+2] after the tile loop
 
     const int split = blockIdx.x, unit = blockIdx.y, b = blockIdx.z;
     const int groups = a.plan.groups;
@@ -452,85 +534,167 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
     const int g = lane >> 2, t = lane & 3;
     const size_t units = (size_t)a.Hkv * groups;
 
-    for (int e = tid; e < Tr::NLK * 32; e += 128) lutk[e] = __ldg(tb.lut_k + (e >> 5));
-    for (int e = tid; e < Tr::NLV * 32; e += 128) lutv[e] = __ldg(tb.lut_v + (e >> 5));
-    QueryFrags<KK, kRegQ> qf;
+    fill_luts<D, BITS, NT>(tb, lutk, lutv, tid);
+    QueryFrags<KK, NT, Tr::QREG> qf;
     qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64,
-            reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dyn_smem) + Tr::RING_BYTES), lane, tid);
-
-    int seq = a.seq_len[b];
-    const int lim = min(a.max_len, a.capacity);
-    if (seq < 0 || seq > lim) {
-        if (tid == 0 && split == 0 && unit == 0) atomicOr(tb.status, TQ_STATUS_SEQ_LEN);
-        seq = min(max(seq, 0), lim);
-    }
+            reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dyn_smem) + Tr::RING_BYTES), tid);
+    const int seq = min(max(a.seq_len[b], 0), min(a.max_len, a.capacity));
     __syncthreads();
 
-    const int ntiles = SCORES ? a.plan.tiles : (seq + 15) >> 4;
     const int t_begin = split * a.plan.tps;
-    const int t_end = min(t_begin + a.plan.tps, ntiles);
+    const int t_end = min(t_begin + a.plan.tps, a.plan.tiles);
     const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
                                          (size_t)a.tile_bytes;
     const uint32_t lane4 = 4u * lane;
     const int ratio = a.Hq / a.Hkv;
-
-    if constexpr (SCORES) {
-        const int j0 = grp * 8 + 2 * t;
-        TileData<D, BITS> td;
+    const int j0 = grp * 8 + 2 * t;
+    TileData<D, BITS> td;
 #pragma unroll 1
-        for (int tl = t_begin + w; tl < t_end; tl += 4) {
-            const int pos0 = tl * 16 + g, pos1 = pos0 + 8;
-            float L[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-            if (tl * 16 < seq) {   // warp-uniform
-                load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, td);
-                tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
-                if (pos0 >= seq) L[0] = L[1] = -CUDART_INF_F;
-                if (pos1 >= seq) L[2] = L[3] = -CUDART_INF_F;
-            }
+    for (int tl = t_begin + w; tl < t_end; tl += WARPS) {
+        const int pos0 = tl * 16 + g, pos1 = pos0 + 8;
+        float L[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+        if (tl * 16 < seq) {   // warp-uniform
+            load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, td);
+            tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
+            if (pos0 >= seq) L[0] = L[1] = -CUDART_INF_F;
+            if (pos1 >= seq) L[2] = L[3] = -CUDART_INF_F;
+        }
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (j0 + hh >= ratio) continue;
-                float* row = a.out + ((size_t)b * a.Hq + hkv * ratio + j0 + hh) * a.max_len;
-                if (pos0 < a.max_len) row[pos0] = L[hh] * kLn2;
-                if (pos1 < a.max_len) row[pos1] = L[2 + hh] * kLn2;
+        for (int hh = 0; hh < 2; ++hh) {
+            if (j0 + hh >= ratio) continue;
+            float* row = a.out + ((size_t)b * a.Hq + hkv * ratio + j0 + hh) * a.max_len;
+            if (pos0 < a.max_len) row[pos0] = L[hh] * kLn2;
+            if (pos1 < a.max_len) row[pos1] = L[2 + hh] * kLn2;
+        }
+    }
+}
+
+// Split kernel, stream-K: the tiles of all (sequence, kv head, group of 8
+// query heads) units, laid end to end (sequence b's units start at
+// prefix[b]), are cut into gridDim.x equal contiguous ranges, one per CTA, so
+// that one wave of CTAs does equal work whatever the lengths. A CTA walks its
+// range unit by unit; for each piece (segment) its 8 warps stream the tiles
+// round-robin through a per-warp cp.async ring, merge in shared memory and
+// write one partial (m, l, acc per head) to slot CTA + unit, a slot no other
+// segment uses: along the tile order both the CTA index and the unit index
+// are non-decreasing and every new segment raises at least one of them.
+template <int D, int BITS>
+__global__ void __launch_bounds__(AttTraits<D, BITS>::NT, AttTraits<D, BITS>::CTAS_PER_SM)
+    attend_split(DevTables tb, AttendArgs a)
+{
+    using Tr = AttTraits<D, BITS>;
+    constexpr int KK = Tr::KK, WARPS = Tr::WARPS, NT = Tr::NT, S = Tr::STAGES;
+    constexpr int RS = D + 2;
+    // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l, so
+    // the 32 lanes of a warp always hit 32 different banks.
+    __shared__ __align__(16) uint32_t lutv[Tr::NLV * 32];
+    __shared__ __align__(16) uint32_t lutk[Tr::NLK * 32];
+    __shared__ __align__(8) uint64_t bars[WARPS * S];   // one mbarrier per ring slot
+    extern __shared__ uint4 dyn_smem[];
+    float* mrg = reinterpret_cast<float*>(dyn_smem);       // [WARPS][8][D+2] after a segment
+    uint4* qsm = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dyn_smem) + Tr::RING_BYTES);
+
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int c = blockIdx.x;
+    const long long G = gridDim.x;
+    const int groups = a.plan.groups, upb = a.Hkv * groups;
+    const long long W = a.prefix[a.B];
+    const long long x0 = (long long)c * W / G, x1 = (long long)(c + 1) * W / G;
+    if (x0 >= x1) return;   // an empty range (fewer tiles than CTAs): uniform, before any barrier
+
+    fill_luts<D, BITS, NT>(tb, lutk, lutv, tid);
+    const int lim = min(a.max_len, a.capacity);
+    const uint32_t lane4 = 4u * lane;
+    uint8_t* ring = reinterpret_cast<uint8_t*>(dyn_smem) + (size_t)w * S * Tr::STAGE_BYTES;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(bars + w * S);
+    if (lane == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(bar_s + 8 * i, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    // Bulk copies this warp has issued / waited for (warp-uniform): copy n uses
+    // ring slot n % S and completes phase (n / S) & 1 of that slot's barrier.
+    uint32_t issued = 0, consumed = 0;
+    bool stalled = false;   // a wait ran out: no further copies, tiles skipped
+    QueryFrags<KK, NT, Tr::QREG> qf;
+
+    // Each segment re-locates its unit from x, so that only x, x1 and the
+    // partial slot stay live across the tile loop.
+    long long x = x0;
+#pragma unroll 1
+    while (x < x1) {
+        // the sequence holding tile x: the largest b with prefix[b] <= x (it has tiles)
+        int b = 0;
+        {
+            int hi = a.B - 1;
+            while (b < hi) {
+                const int mid = (b + hi + 1) >> 1;
+                if (a.prefix[mid] <= x) b = mid; else hi = mid - 1;
             }
         }
-        return;
-    } else {
+        const long long pb = a.prefix[b];
+        const long long T = (a.prefix[b + 1] - pb) / upb;   // tiles per unit of sequence b
+        const int j = (int)((x - pb) / T);
+        const long long U0 = pb + (long long)j * T;
+        const int sb = (int)(x - U0);
+        const int se = (int)min(T, x1 - U0);
+        const int seq = min(max(a.seq_len[b], 0), lim);
+        const int hkv = j / groups;
+        const size_t u = (size_t)b * upb + j;
+        qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
+        __syncthreads();   // tables (first segment) and query fragments visible
+
+        const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
+                                             (size_t)a.tile_bytes;
         SplitState<D> st;
         st.m0 = st.m1 = -CUDART_INF_F;
         st.l0 = st.l1 = 0.f;
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
 
-        // cp.async pipeline: STAGES - 1 tiles of this warp are in flight while
-        // one is decoded; every lane stages and reads back only its own bytes,
-        // so the only synchronisation is the per-thread wait_group.
-        constexpr int S = Tr::STAGES;
-        uint8_t* ring = reinterpret_cast<uint8_t*>(dyn_smem) + (size_t)w * S * Tr::STAGE_BYTES;
-        const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
-        const int my_first = t_begin + w;
+        // Bulk-copy pipeline: S - 1 tiles of this warp are in flight while one
+        // is decoded. Lane 0 issues each copy into the slot the warp finished
+        // reading one iteration earlier (its values are already used).
+        const int my_first = sb + w;
+        fence_proxy_async();
+        if (!stalled && lane == 0) {
 #pragma unroll
-        for (int i = 0; i < S - 1; ++i) {
-            const int tl = my_first + 4 * i;
-            if (tl < t_end)
-                stage_tile<D, BITS>(ring_s + i * Tr::STAGE_BYTES, sbase + (size_t)tl * (size_t)a.tile_bytes,
-                                    lane, g);
-            cp_async_commit();
+            for (int i = 0; i < S - 1; ++i) {
+                const int tl = my_first + WARPS * i;
+                if (tl < se) {
+                    const uint32_t sl = (issued + i) % S;
+                    bulk_load(ring_s + sl * Tr::STAGE_BYTES, sbase + (size_t)tl * Tr::TILE_BYTES,
+                              Tr::TILE_BYTES, bar_s + 8 * sl);
+                }
+            }
+        }
+        if (!stalled) {
+#pragma unroll
+            for (int i = 0; i < S - 1; ++i) issued += (my_first + WARPS * i < se) ? 1u : 0u;
         }
         TileData<D, BITS> td;
-        int slot = 0;
 #pragma unroll 1
-        for (int tl = my_first; tl < t_end; tl += 4) {
-            const int tn = tl + 4 * (S - 1);
-            const int nslot = slot == 0 ? S - 1 : slot - 1;   // the slot consumed last iteration
-            if (tn < t_end)
-                stage_tile<D, BITS>(ring_s + nslot * Tr::STAGE_BYTES, sbase + (size_t)tn * (size_t)a.tile_bytes,
-                                    lane, g);
-            cp_async_commit();
-            cp_async_wait<S - 1>();
+        for (int tl = my_first; tl < se && !stalled; tl += WARPS) {
+            const int tn = tl + WARPS * (S - 1);
+            if (tn < se) {
+                fence_proxy_async();
+                if (lane == 0) {
+                    const uint32_t sl = issued % S;
+                    bulk_load(ring_s + sl * Tr::STAGE_BYTES, sbase + (size_t)tn * Tr::TILE_BYTES,
+                              Tr::TILE_BYTES, bar_s + 8 * sl);
+                }
+                ++issued;
+            }
+            const uint32_t slot = consumed % S;
+            if (!mbar_wait(bar_s + 8 * slot, (consumed / S) & 1u)) {
+                stalled = true;
+                if (lane == 0) atomicOr(tb.status, TQ_STATUS_WAIT_TIMEOUT);
+                break;
+            }
+            ++consumed;
             read_stage<D, BITS>(ring + slot * Tr::STAGE_BYTES, lane, td);
-            slot = slot == S - 1 ? 0 : slot + 1;
             float L[4];
             tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
             const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
@@ -538,7 +702,6 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
             if (!v1) L[2] = L[3] = -CUDART_INF_F;
             tile_accumulate<D, BITS>(td, L, v0, v1, lutv, lane4, st);
         }
-        cp_async_wait<0>();
 
         float l0 = st.l0, l1 = st.l1;
 #pragma unroll
@@ -546,8 +709,8 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
             l0 += __shfl_xor_sync(kFull, l0, sh);
             l1 += __shfl_xor_sync(kFull, l1, sh);
         }
+        fence_proxy_async();
         __syncthreads();   // every warp is done with the ring: reuse it for the merge
-        constexpr int RS = D + 2;
         float* mw = mrg + (size_t)w * 8 * RS;
         if (g == 0) {
             mw[(2 * t) * RS] = st.m0;
@@ -563,24 +726,31 @@ __global__ void __launch_bounds__(128, D <= 128 ? 3 : 1) attend_split(DevTables 
             mw[(2 * t + 1) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][3];
         }
         __syncthreads();
-        float* dst = a.partial + (((size_t)b * units + unit) * a.plan.nsplit + split) * 8 * RS;
-        for (int e = tid; e < 8 * RS; e += 128) {
-            const int head = e / RS, c = e % RS;
+        float* dst = a.partial + ((size_t)c + u) * 8 * RS;
+        for (int e = tid; e < 8 * RS; e += NT) {
+            const int head = e / RS, col = e % RS;
             float M = -CUDART_INF_F;
 #pragma unroll
-            for (int ww = 0; ww < 4; ++ww) M = fmaxf(M, mrg[(ww * 8 + head) * RS]);
+            for (int ww = 0; ww < WARPS; ++ww) M = fmaxf(M, mrg[(ww * 8 + head) * RS]);
             float sum = 0.f;
-            if (c == 0) {
+            if (col == 0) {
                 sum = M;
             } else {
 #pragma unroll
-                for (int ww = 0; ww < 4; ++ww) {
+                for (int ww = 0; ww < WARPS; ++ww) {
                     const float mwv = mrg[(ww * 8 + head) * RS];
-                    if (mwv != -CUDART_INF_F) sum += mrg[(ww * 8 + head) * RS + c] * exp2f(mwv - M);
+                    if (mwv != -CUDART_INF_F) sum += mrg[(ww * 8 + head) * RS + col] * exp2f(mwv - M);
                 }
             }
             dst[e] = sum;
         }
+        __syncthreads();   // merge buffer and query fragments free for the next segment
+        x = U0 + se;       // the next unit (or the end of the range)
+    }
+    // after a wait ran out: wait (bounded) for this warp's copies still in flight
+    while (consumed < issued) {
+        if (!mbar_wait(bar_s + 8 * (consumed % S), (consumed / S) & 1u)) break;
+        ++consumed;
     }
 }
 
@@ -603,20 +773,21 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
 {
     using Tr = AttTraits<D, BITS>;
     static unsigned long long done_scores = 0, done_attend = 0;
+    if (a.tile_bytes != Tr::TILE_BYTES) return cudaErrorInvalidValue;   // the bulk copies' size
     const int units = a.Hkv * a.plan.groups;
     attend_prologue<D><<<dim3(units, a.B), 2 * D, 0, st>>>(tb, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const dim3 grid(a.plan.nsplit, units, a.B);
     if (scores) {
-        auto kern = attend_split<D, BITS, true>;
+        auto kern = attend_scores<D, BITS>;
         if ((e = allow_smem(kern, Tr::DYN_SMEM, done_scores)) != cudaSuccess) return e;
-        if (a.plan.tiles > 0) kern<<<grid, 128, Tr::DYN_SMEM, st>>>(tb, a);
+        if (a.plan.tiles > 0)
+            kern<<<dim3(a.plan.nsplit, units, a.B), Tr::NT, Tr::DYN_SMEM, st>>>(tb, a);
         return cudaGetLastError();
     }
-    auto kern = attend_split<D, BITS, false>;
+    auto kern = attend_split<D, BITS>;
     if ((e = allow_smem(kern, Tr::DYN_SMEM, done_attend)) != cudaSuccess) return e;
-    kern<<<grid, 128, Tr::DYN_SMEM, st>>>(tb, a);
+    if (a.plan.tiles > 0) kern<<<a.plan.ctas, Tr::NT, Tr::DYN_SMEM, st>>>(tb, a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attend_reduce<D><<<dim3(a.Hq, a.B), D, 0, st>>>(tb, a);
@@ -639,17 +810,26 @@ AttendPlan plan_attend(int d, int B, int Hq, int Hkv, int max_len, int num_sms)
     p.groups = (ratio + 7) / 8;
     const long long units = (long long)B * Hkv * p.groups;
     p.tiles = (max_len + 15) / 16;
-    const long long target = 8LL * num_sms;           // CTAs of 4 warps: ~2 waves at 4 CTAs/SM
+    // tq_scores: one CTA per (unit, context split), about two waves
+    const long long per_sm = d <= 128 ? AttTraits<128, 4>::CTAS_PER_SM : AttTraits<256, 4>::CTAS_PER_SM;
+    const long long target = 2 * per_sm * num_sms;
     long long ns = (target + units - 1) / units;
-    const long long max_ns = (p.tiles + 7) / 8;        // at least 8 tiles (2 per warp) per split
+    const long long max_ns = (p.tiles + 15) / 16;      // at least 16 tiles (2 per warp) per split
     if (ns > max_ns) ns = max_ns;
     if (ns < 1) ns = 1;
     p.tps = p.tiles > 0 ? (int)((p.tiles + ns - 1) / ns) : 0;
     p.nsplit = p.tps > 0 ? (p.tiles + p.tps - 1) / p.tps : 1;
+    // tq_attend: stream-K, one wave of CTAs (fewer when there are under 16 tiles per CTA)
+    long long ctas = per_sm * num_sms;
+    const long long most = (units * p.tiles + 15) / 16;
+    if (ctas > most) ctas = most;
+    if (ctas < 1) ctas = 1;
+    p.ctas = (int)ctas;
     p.qfrag_bytes = (size_t)units * (d / 16) * 32 * 32;
-    p.partial_bytes = (size_t)units * p.nsplit * 8 * (d + 2) * sizeof(float);
+    p.prefix_bytes = (size_t)(B + 1) * sizeof(long long);
+    p.partial_bytes = (size_t)(ctas + units) * 8 * (d + 2) * sizeof(float);
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    p.total_bytes = up(p.qfrag_bytes) + up(p.partial_bytes);
+    p.total_bytes = up(p.qfrag_bytes) + up(p.prefix_bytes) + up(p.partial_bytes);
     return p;
 }
 

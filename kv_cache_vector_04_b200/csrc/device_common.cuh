@@ -35,6 +35,25 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same product with a zero accumulator (the first k-step of a chain).
+__device__ __forceinline__ void mma_16816_first(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};\n"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// 2^x with the SFU's approximate exponential (relative error ~2^-22;
+// subnormal results flush to 0, which only touches weights below 2^-126).
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Transpose an 8x8 matrix of 16-bit values held in the m8n8 fragment layout
 // (lane 4g+t holds row g, columns 2t and 2t+1).
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x)

@@ -17,13 +17,14 @@ struct QuantizeArgs {
     long long tile_bytes;
 };
 
-// Split-K geometry of one attention call.
+// Geometry of one attention call.
 struct AttendPlan {
     int groups;     // head groups of 8 per kv head: ceil((Hq/Hkv) / 8)
-    int nsplit;     // splits of the context per (b, kv head, group)
     int tiles;      // ceil(max_len / 16)
-    int tps;        // tiles per split
-    size_t qfrag_bytes, partial_bytes, total_bytes;
+    int nsplit;     // tq_scores: splits of the context per (b, kv head, group)
+    int tps;        // tq_scores: tiles per split
+    int ctas;       // tq_attend: CTAs of the stream-K split kernel
+    size_t qfrag_bytes, prefix_bytes, partial_bytes, total_bytes;
 };
 
 struct AttendArgs {
@@ -34,7 +35,8 @@ struct AttendArgs {
     int B, Hq, Hkv, capacity, max_len;
     long long tile_bytes;
     uint32_t* qfrag;          // workspace: [B][Hkv*groups][d/16][32][4] fp16x2 B fragments
-    float* partial;           // workspace: [B][Hkv*groups][nsplit][8][d + 2]
+    long long* prefix;        // workspace: [B + 1] first flattened tile of each sequence's units
+    float* partial;           // workspace: [ctas + B*Hkv*groups][8][d + 2], slot = CTA + unit
     float* out;               // [B][Hq][d] (attend) or scores [B][Hq][max_len]
     AttendPlan plan;
 };

@@ -30,6 +30,19 @@ def test_library_exports_every_declared_symbol():
     assert sorted(binding.EXPORTS) == names
 
 
+def test_binding_constants_equal_header_defines():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    defs = dict(re.findall(r"#define\s+(TQ_[A-Z0-9_]+)\s+\(?(-?(?:0x)?[0-9a-fA-F]+)u?\)?\s*(?:/\*|\n)", src))
+    assert binding.TQ_NOALLOC_SCRATCH_BYTES == 16 << 20 and "(16u << 20)" in src
+    assert len(defs) >= 12
+    for name, val in defs.items():
+        if hasattr(binding, name):
+            assert getattr(binding, name) == int(val, 0), name
+    for name in ("TQ_STATUS_CAPACITY", "TQ_STATUS_SEQ_LEN", "TQ_STATUS_NORM_SAT",
+                 "TQ_STATUS_WAIT_TIMEOUT", "TQ_ERR_WORKSPACE", "TQ_TILE"):
+        assert name in defs and hasattr(binding, name), name
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(ImportError):
         binding._load(str(tmp_path / "libtq.so"))

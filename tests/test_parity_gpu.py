@@ -230,6 +230,34 @@ def test_attend_many_heads_per_group_and_empty_sequence():
     assert P.attn_error(got, ref).max() <= P.ATTN_TOL
 
 
+@pytest.mark.parametrize("d,bits,max_len", [(64, 4, 600), (128, 3, 600), (128, 2, 4096)])
+def test_attend_many_ragged_sequences(d, bits, max_len):
+    # Many sequences of mixed lengths (empty, one token, tile edges, a few
+    # hundred): the split kernel's equal ranges of the laid-out tiles then
+    # start and end inside units, span several units, and (max_len far above
+    # every length) some CTAs get no tiles at all.
+    ctx, tab = ctx_for(d, bits)
+    B, Hkv, Hq = 40, 2, 12
+    rng = np.random.default_rng(d + bits)
+    top = min(max_len, 600)
+    seq = [int(x) for x in rng.choice([0, 1, 15, 16, 17, 33, top], size=B)]
+    seq[:8] = [int(x) for x in rng.integers(0, top + 1, size=8)]
+    seq = [min(s, 40) for s in seq] if max_len > 600 else seq
+    N = max(seq)
+    cap = ((max(max_len, N) + 15) // 16) * 16
+    k, v = kv(B, Hkv, N, d, seed=300 + d + bits)
+    codes = P.oracle_codes(tab, k, v)
+    cache = tq.Cache(P.pack_cache(tab, codes, cap, d, bits), B, Hkv, cap)
+    q = qtensor(B, Hq, d, seed=5)
+    got = run_attend(ctx, tab, cache, q, seq, max_len, Hkv)
+    ref = O.attend_batch(tab, P.q_bits(q), True, P.stack_codes(codes, cap), np.array(seq, np.int32), Hkv)
+    for b in range(B):
+        if seq[b] == 0:
+            assert np.all(got[b] == 0.0)
+    assert P.attn_error(got, ref).max() <= P.ATTN_TOL
+    assert tq.tq_status(ctx) == 0
+
+
 def test_seq_len_out_of_range_is_clamped_and_flagged():
     d, bits = 64, 3
     ctx, tab = ctx_for(d, bits)
