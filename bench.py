@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--layers", type=int, default=None, help="override layer count (development)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the eager launch loop only (no CUDA graph of the step)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args(argv)
 
@@ -274,21 +276,36 @@ def run_tq(args, dist: Dist):
     seq = torch.full((w.B,), N + 1, dtype=torch.int32, device=dev)
     ws = tq.new_workspace(ctx, w.B, w.Hq, w.Hkv, N + 1)
     outs = [torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev) for _ in range(layers)]
-    launches_per_step = layers * (1 + 3)
+    launches_per_step = layers * 3   # per layer: prologue with the append, split, reduce
 
     def step(events=None):
         for L in range(layers):
             nk, nv = news[L]
-            tq.tq_quantize(ctx, nk, nv, start, caches[L])
             if events is not None:
                 events[L][0].record()
-            tq.tq_attend(ctx, qs[L], caches[L], seq, N + 1, out=outs[L], workspace=ws)
+            tq.tq_append_attend(ctx, qs[L], nk, nv, start, caches[L], seq, N + 1, out=outs[L],
+                                workspace=ws)
             if events is not None:
                 events[L][1].record()
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+
+    # ---- the whole step (all layers) as one CUDA graph
+    graph = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
 
     # ---- copy-kernel HBM peak in the same process (1 GiB -> 1 GiB)
     src = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
@@ -319,10 +336,21 @@ def run_tq(args, dist: Dist):
     t_end.record()
     torch.cuda.synchronize()
     dist.barrier()
-    clk = clocks.stop()
-    ms = t_start.elapsed_time(t_end) / args.steps
+    ms_eager = dist.max(t_start.elapsed_time(t_end) / args.steps)
     attend_ms = statistics.mean(a.elapsed_time(b) for row in ev for (a, b) in row)
-    ms = dist.max(ms)
+    ms_graph = None
+    if graph is not None:
+        dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record()
+        for _ in range(args.steps):
+            graph.replay()
+        t_end.record()
+        torch.cuda.synchronize()
+        dist.barrier()
+        ms_graph = dist.max(t_start.elapsed_time(t_end) / args.steps)
+    clk = clocks.stop()
+    ms = ms_graph if ms_graph is not None else ms_eager
     assert tq.tq_status(ctx) == 0
 
     bytes_step = layers * w.B * w.Hkv * (N + 1) * per_tok
@@ -338,16 +366,17 @@ def run_tq(args, dist: Dist):
         q_host = [q.cpu().pin_memory() for q in qs]
         k_host = [(a.cpu().pin_memory(), b.cpu().pin_memory()) for a, b in news]
         out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-        q_dev = [torch.empty_like(q) for q in qs[:1]]
-        kv_dev = [(torch.empty_like(a), torch.empty_like(b)) for a, b in news[:1]]
+        q_dev = torch.empty_like(qs[0])
+        kv_dev = (torch.empty_like(news[0][0]), torch.empty_like(news[0][1]))
 
         def host_step():
             for L in range(layers):
-                kv_dev[0][0].copy_(k_host[L][0], non_blocking=True)
-                kv_dev[0][1].copy_(k_host[L][1], non_blocking=True)
-                tq.tq_quantize(ctx, kv_dev[0][0], kv_dev[0][1], start, caches[L])
-                tq.attend_host(ctx, q_host[L], caches[L], seq, N + 1, out_host[L], ws,
-                               q_dev[0], outs[L])
+                q_dev.copy_(q_host[L], non_blocking=True)
+                kv_dev[0].copy_(k_host[L][0], non_blocking=True)
+                kv_dev[1].copy_(k_host[L][1], non_blocking=True)
+                tq.tq_append_attend(ctx, q_dev, kv_dev[0], kv_dev[1], start, caches[L], seq, N + 1,
+                                    out=outs[L], workspace=ws)
+                out_host[L].copy_(outs[L], non_blocking=True)
 
         for _ in range(max(args.warmup, 3)):
             host_step()
@@ -376,11 +405,16 @@ def run_tq(args, dist: Dist):
         "config": {"workload": w.name, "layers": layers, "batch": w.B, "q_heads": w.Hq,
                    "kv_heads": w.Hkv, "head_dim": w.d, "bits": w.bits, "context": N + 1,
                    "packed_cache_gb": round(layers * w.B * w.Hkv * cap * per_tok / 1e9, 2),
-                   "step": "per layer: tq_quantize (append 1 token) + tq_attend",
+                   "step": "per layer: tq_append_attend (append 1 token, then attend)",
+                   "step_launch": "one CUDA graph per step" if ms_graph is not None else "eager",
                    "l2": "inputs larger than L2 (%.0f MB per layer)" % (bytes_attend / 1e6),
                    "parallelism": "replicas x%d (weak)" % dist.world},
         "pct_of_hbm_peak": round(100.0 * value / dist.world / peak, 1),
-        "roofline": {"bound": "hbm", "kernel": "tq_attend (prologue + split + reduce launches)",
+        "ms_per_step_eager": round(ms_eager, 4),
+        "ms_per_step_graph": round(ms_graph, 4) if ms_graph is not None else None,
+        "ms_per_layer": round(ms / layers, 4),
+        "roofline": {"bound": "hbm",
+                     "kernel": "tq_append_attend per layer (prologue with the append + split + reduce)",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
                      "traffic": profiled_traffic(w.name),

@@ -181,6 +181,27 @@ int tq_attend(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_c
               const int32_t* seq_len, int max_len, float* out, void* workspace,
               size_t workspace_bytes, void* stream);
 
+/* One decode step of a layer: append T new tokens to the cache, then attend.
+ * The result is that of tq_quantize(ctx, k, v, B, Hkv, T, start_pos, cache,
+ * stream) followed by tq_attend(ctx, q, q_dtype, B, Hq, cache, seq_len,
+ * max_len, out, workspace, workspace_bytes, stream), with Hkv = cache->Hkv:
+ *  k, v:      device, fp16 [B][Hkv][T][d], contiguous, 16-byte aligned.
+ *  T:         new tokens per sequence, >= 0.
+ *  start_pos: device, int32[B]: the new tokens go to positions
+ *             [start_pos[b], start_pos[b] + T) (TQ_STATUS_CAPACITY as in
+ *             tq_quantize). seq_len normally equals start_pos + T.
+ * The other arguments are those of tq_attend. For 1 <= T <= 16 the new tokens
+ * are quantized inside the first attention launch, by one CTA per (sequence,
+ * kv head) working on shared-memory copies of the (at most two) tiles they
+ * touch: three launches per call. For T > 16 the quantize kernel runs first.
+ * This is the per-layer decode step the pages' generation-speed measurements
+ * time ("[Benchmark] TurboQuant 實測：KV Cache 3-bit 壓縮，真的零損失？",
+ * §"GB10 速度"). */
+int tq_append_attend(tq_ctx* ctx, const void* q, int q_dtype, const void* k, const void* v, int B,
+                     int Hq, int T, const int32_t* start_pos, const tq_cache* cache,
+                     const int32_t* seq_len, int max_len, float* out, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
 /* The estimated attention logits alone (the "inner product" of the pages'
  * speed test): scores[b][h][n] = l_n for n < seq_len[b], -inf for
  * seq_len[b] <= n < max_len. scores: device fp32 [B][Hq][max_len]. Same

@@ -34,7 +34,7 @@ TQ_DTYPE_BF16 = 1
 # every symbol include/tq.h declares
 EXPORTS = ("tq_init", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
            "tq_build_tables", "tq_quantize", "tq_attend_workspace", "tq_attend", "tq_scores",
-           "tq_attend_noalloc", "tq_status", "tq_copy", "tq_strerror")
+           "tq_attend_noalloc", "tq_append_attend", "tq_status", "tq_copy", "tq_strerror")
 TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -75,6 +75,8 @@ def _load(path: str = LIB_PATH):
         "tq_attend": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, P]),
         "tq_scores": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, P]),
         "tq_attend_noalloc": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P]),
+        "tq_append_attend": (I, [P, P, I, P, P, I, I, I, P, ctypes.POINTER(_Cache), P, I, P, P,
+                                 SZ, P]),
         "tq_status": (I, [P, ctypes.POINTER(ctypes.c_uint32)]),
         "tq_copy": (I, [P, P, SZ, P]),
         "tq_strerror": (ctypes.c_char_p, [I]),
@@ -292,6 +294,35 @@ def tq_attend_noalloc(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torc
                                   _dev(seq_len, "seq_len", torch.int32), int(max_len),
                                   _dev(out, "out", torch.float32),
                                   ctypes.c_void_p(_stream_ptr(stream))), "tq_attend_noalloc")
+    return out
+
+
+def tq_append_attend(ctx: Context, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                     start_pos: torch.Tensor, cache: Cache, seq_len: torch.Tensor, max_len: int,
+                     out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                     stream=None):
+    """One layer's decode step: append k, v (fp16 [B, Hkv, T, d]) at start_pos,
+    then attend q [B, Hq, d] over tokens [0, seq_len[b]) -> fp32 [B, Hq, d]."""
+    if q.dim() != 3 or q.shape[2] != ctx.d:
+        raise ValueError("q must be [B, Hq, d] with d = %d" % ctx.d)
+    if k.dim() != 4 or k.shape != v.shape or k.shape[3] != ctx.d:
+        raise ValueError("k and v must both be [B, Hkv, T, d] with d = %d" % ctx.d)
+    B, Hq, _ = q.shape
+    if k.shape[0] != B or k.shape[1] != cache.Hkv or start_pos.numel() != B:
+        raise ValueError("k, v, start_pos must match q's batch and the cache's kv heads")
+    T = k.shape[2]
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(ctx, B, Hq, cache.Hkv, max_len)
+    c = cache.struct()
+    _check(_lib.tq_append_attend(ctx.handle, _dev(q, "q"), _q_dtype(q), _dev(k, "k", torch.float16),
+                                 _dev(v, "v", torch.float16), B, Hq, T,
+                                 _dev(start_pos, "start_pos", torch.int32), ctypes.byref(c),
+                                 _dev(seq_len, "seq_len", torch.int32), int(max_len),
+                                 _dev(out, "out", torch.float32), _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(),
+                                 ctypes.c_void_p(_stream_ptr(stream))), "tq_append_attend")
     return out
 
 

@@ -157,9 +157,16 @@ int upload_tables(tq_ctx* ctx)
     return TQ_OK;
 }
 
+int quantize_common(tq_ctx* ctx, const void* k, const void* v, int B, int Hkv, int T,
+                    const int32_t* start_pos, const tq_cache* cache, void* stream);
+
+// tq_attend / tq_scores / tq_append_attend. With k != nullptr the T new tokens
+// are appended first: inside the prologue launch when 1 <= T <= 16, else by
+// the quantize kernel launched ahead of the attention launches.
 int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,
                   const int32_t* seq_len, int max_len, float* out, void* ws, size_t ws_bytes,
-                  void* stream, bool scores)
+                  void* stream, bool scores, const void* k = nullptr, const void* v = nullptr,
+                  int T = 0, const int32_t* start_pos = nullptr)
 {
     if (!ctx || !q || !seq_len || !out) return TQ_ERR_INVALID_ARG;
     if (q_dtype != TQ_DTYPE_F16 && q_dtype != TQ_DTYPE_BF16) return TQ_ERR_INVALID_ARG;
@@ -176,8 +183,22 @@ int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const 
     if (!ws || !aligned(ws, 256)) return TQ_ERR_INVALID_ARG;
     if (ws_bytes < plan.total_bytes) return TQ_ERR_WORKSPACE;
     if (!aligned(q, 16) || !aligned(out, 16)) return TQ_ERR_INVALID_ARG;
+    const bool append = k != nullptr;
+    if (append) {
+        if (!v || !start_pos || T < 0) return TQ_ERR_INVALID_ARG;
+        if (!aligned(k, 16) || !aligned(v, 16)) return TQ_ERR_INVALID_ARG;
+        if (T > 16 && (rc = quantize_common(ctx, k, v, B, Hkv, T, start_pos, cache, stream)))
+            return rc;
+    }
     if (scores && max_len == 0) return TQ_OK;
     tq::AttendArgs a{};
+    if (append && T >= 1 && T <= 16) {
+        a.k_new = static_cast<const __half*>(k);
+        a.v_new = static_cast<const __half*>(v);
+        a.start_pos = start_pos;
+        a.T = T;
+        a.cache_w = static_cast<uint8_t*>(cache->data);
+    }
     a.q = q;
     a.q_bf16 = (q_dtype == TQ_DTYPE_BF16);
     a.seq_len = seq_len;
@@ -292,6 +313,26 @@ int tq_get_tables(const tq_ctx* ctx, float* centroids_k, float* bounds_k, float*
 int tq_quantize(tq_ctx* ctx, const void* k, const void* v, int B, int Hkv, int T,
                 const int32_t* start_pos, const tq_cache* cache, void* stream)
 {
+    return quantize_common(ctx, k, v, B, Hkv, T, start_pos, cache, stream);
+}
+
+int tq_append_attend(tq_ctx* ctx, const void* q, int q_dtype, const void* k, const void* v, int B,
+                     int Hq, int T, const int32_t* start_pos, const tq_cache* cache,
+                     const int32_t* seq_len, int max_len, float* out, void* workspace,
+                     size_t workspace_bytes, void* stream)
+{
+    if (!k) return TQ_ERR_INVALID_ARG;
+    return attend_common(ctx, q, q_dtype, B, Hq, cache, seq_len, max_len, out, workspace,
+                         workspace_bytes, stream, false, k, v, T, start_pos);
+}
+
+}  // extern "C"
+
+namespace {
+
+int quantize_common(tq_ctx* ctx, const void* k, const void* v, int B, int Hkv, int T,
+                    const int32_t* start_pos, const tq_cache* cache, void* stream)
+{
     if (!ctx || !k || !v || !start_pos) return TQ_ERR_INVALID_ARG;
     if (B <= 0 || Hkv <= 0 || T < 0 || B > 65535 || Hkv > 65535) return TQ_ERR_INVALID_ARG;
     int rc = check_cache(ctx, cache, B, Hkv);
@@ -313,6 +354,10 @@ int tq_quantize(tq_ctx* ctx, const void* k, const void* v, int B, int Hkv, int T
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
+
+}  // namespace
+
+extern "C" {
 
 int tq_attend_workspace(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_len, size_t* bytes)
 {

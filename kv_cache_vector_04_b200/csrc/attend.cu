@@ -141,11 +141,12 @@ __device__ __forceinline__ void tile_prefix(const DevTables& tb, const AttendArg
 // products carry ~22 significant bits. alpha is the scale that makes the key
 // codebook almost exact in fp16 (chosen on the host).
 template <int D>
-__global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArgs a)
+__device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendArgs& a)
 {
     constexpr int NT = 2 * D;
     __shared__ float qt[D][8];          // rotated queries, [coordinate][head]
-    __shared__ float pp[2][D][8];       // p = S q~, two partial halves over k
+    __shared__ float pp[1][D][8];       // p = S q~
+    __shared__ float es[8];             // per-head power-of-two scale of q~ for the split
     const int unit = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const int groups = a.plan.groups, ratio = a.Hq / a.Hkv;
     const int hkv = unit / groups, grp = unit % groups;
@@ -178,22 +179,43 @@ __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArg
     const float rs = rsqrtf((float)D);
     for (int e = tid; e < 8 * D; e += NT) (&qt[0][0])[e] *= rs;
     __syncthreads();
+    // per head a power of two es with max |q~| es in [64, 128): the hi and lo
+    // fp16 parts of q~ es below then stay clear of overflow and of subnormals
     {
-        const int j = tid % D, half = tid / D;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const int k0 = half * (D / 2);
-#pragma unroll 4
-        for (int k = k0; k < k0 + D / 2; ++k) {
-            const float sv = __ldg(tb.s_t + (size_t)k * D + j);
-            const float4 q0 = *reinterpret_cast<const float4*>(&qt[k][0]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&qt[k][4]);
-            acc[0] = fmaf(sv, q0.x, acc[0]); acc[1] = fmaf(sv, q0.y, acc[1]);
-            acc[2] = fmaf(sv, q0.z, acc[2]); acc[3] = fmaf(sv, q0.w, acc[3]);
-            acc[4] = fmaf(sv, q1.x, acc[4]); acc[5] = fmaf(sv, q1.y, acc[5]);
-            acc[6] = fmaf(sv, q1.z, acc[6]); acc[7] = fmaf(sv, q1.w, acc[7]);
-        }
+        const int w = tid >> 5, lane = tid & 31;
+        for (int h = w; h < 8; h += NT / 32) {
+            float mx = 0.f;
+            for (int c = lane; c < D; c += 32) mx = fmaxf(mx, fabsf(qt[c][h]));
 #pragma unroll
-        for (int h = 0; h < 8; ++h) pp[half][j][h] = acc[h];
+            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+            if (lane == 0) es[h] = (mx > 0.f && mx < 3.0e38f) ? exp2f((float)(6 - ilogbf(mx))) : 1.f;
+        }
+    }
+    __syncthreads();
+    // p^T = q~^T S^T on the tensor cores: A = q~ es (rows = the 8 heads, rows
+    // 8..15 zero) as hi + lo fp16 parts, B = the fp16-exact S^T fragments,
+    // fp32 accumulation; warp w takes n-tiles (8 rows of S each) w, w + NW, ...
+    {
+        const int w = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+        const float sc = es[g];
+        for (int nt = w; nt < D / 8; nt += NT / 32) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int c0 = 16 * kk + 2 * t;
+                const float x0 = qt[c0][g] * sc, x1 = qt[c0 + 1][g] * sc;
+                const float x2 = qt[c0 + 8][g] * sc, x3 = qt[c0 + 9][g] * sc;
+                const float h0 = __half2float(__float2half_rn(x0)), h1 = __half2float(__float2half_rn(x1));
+                const float h2 = __half2float(__float2half_rn(x2)), h3 = __half2float(__float2half_rn(x3));
+                const uint2 bf = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
+                mma_16816(acc, pack_half2(h0, h1), 0u, pack_half2(h2, h3), 0u, bf.x, bf.y);
+                mma_16816(acc, pack_half2(x0 - h0, x1 - h1), 0u, pack_half2(x2 - h2, x3 - h3), 0u,
+                          bf.x, bf.y);
+            }
+            // acc[0], acc[1]: head g, rows 8 nt + 2t and + 1 of S
+            pp[0][8 * nt + 2 * t][g] = acc[0] / sc;
+            pp[0][8 * nt + 2 * t + 1][g] = acc[1] / sc;
+        }
     }
     __syncthreads();
     {
@@ -209,8 +231,7 @@ __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArg
             float hv[4], lv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const float x = q ? (pp[0][idx[u]][col] + pp[1][idx[u]][col]) * scale_s
-                                  : qt[idx[u]][col] * scale_c;
+                const float x = q ? pp[0][idx[u]][col] * scale_s : qt[idx[u]][col] * scale_c;
                 hv[u] = __half2float(__float2half_rn(x));
                 lv[u] = x - hv[u];
             }
@@ -225,6 +246,198 @@ __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArg
         dst[32] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
     }
 }
+
+template <int D>
+__global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArgs a)
+{
+    prologue_body<D>(tb, a);
+}
+
+// ---------------------------------------------------------------- fused append
+// Bit position helpers for one token's codes inside a tile image (the tile
+// layout of tq.h): a lane string is cut into chunks of CB bytes stored
+// chunk-major, so string word sw of lane L sits at tile word
+// ((4 sw / CB) * 32 + L) * CB/4 + (4 sw % CB) / 4.
+template <int CB>
+__device__ __forceinline__ int tile_word(int L, int sw)
+{
+    return (((4 * sw) / CB) * 32 + L) * (CB / 4) + ((4 * sw) % CB) / 4;
+}
+
+// Replace the nb-bit field at string bit `sbit` of lane L's string (a field may
+// straddle two string words). Other tokens' bits in the same words may be
+// written by other warps at the same time, hence the shared-memory atomics.
+template <int CB>
+__device__ __forceinline__ void put_field(uint32_t* img, int L, int sbit, uint32_t val, int nb)
+{
+    const int sw = sbit >> 5, off = sbit & 31;
+    const uint32_t m = (1u << nb) - 1u;
+    uint32_t* w0 = img + tile_word<CB>(L, sw);
+    atomicAnd(w0, ~(m << off));
+    atomicOr(w0, (val & m) << off);
+    if (off + nb > 32) {
+        uint32_t* w1 = img + tile_word<CB>(L, sw + 1);
+        atomicAnd(w1, ~(m >> (32 - off)));
+        atomicOr(w1, (val & m) >> (32 - off));
+    }
+}
+
+// Quantize the T <= 16 new tokens of (sequence b, kv head hkv) exactly as
+// tq_quantize does and write them into the cache: the (at most two) tiles they
+// touch are copied into shared memory; each warp takes one K or V vector at a
+// time (fp64 norm, sign flip, Walsh–Hadamard, cells; for keys the residual and
+// its norm) and sets its bits in the tile images; then thread j computes row j
+// of z = S r for every new key as an fp64 dot product (each S entry is loaded
+// once for all keys) and sets the QJL sign bits s = [z >= 0]; the tiles are
+// written back.
+template <int D, int BITS>
+__device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendArgs& a, int b, int hkv,
+                                              uint8_t* smem)
+{
+    constexpr int NT = 2 * D, NW = NT / 32, VPL = D / 32, M = D;
+    constexpr int BK = BITS - 1, BV = BITS;
+    constexpr int TB = 16 * (BITS * D / 4 + 6);
+    constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;
+    constexpr int SB0 = BK * D / 2, VB0 = (BK + 1) * D / 2;   // first sign / value bit of a string
+    constexpr int NB = 4 * BITS * D;                          // first norm byte of a tile
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int T = a.T, start = a.start_pos[b];
+    if (T <= 0) return;
+    if (start < 0 || (long long)start + T > (long long)a.capacity) {
+        if (tid == 0 && hkv == 0) atomicOr(tb.status, TQ_STATUS_CAPACITY);
+        return;
+    }
+    uint32_t* img = reinterpret_cast<uint32_t*>(smem);                      // [2][TB]
+    double* tabs = reinterpret_cast<double*>(smem + 2 * TB);                // ck[16] tk[16] tv[16]
+    double* rk = tabs + 48;                                                  // [16][D] key residuals
+    double* zp = rk + 16 * D;                                                // [16][M] half-sums of z
+    const int t0 = start / 16, ntile = (start + T - 1) / 16 - t0 + 1;
+    uint8_t* stream = a.cache_w + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity / 16) * TB;
+    for (int e = tid; e < ntile * TB / 16; e += NT)
+        reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(stream + (size_t)t0 * TB)[e];
+    if (tid < (1 << BK)) tabs[tid] = tb.centroids_kd[tid];
+    if (tid < (1 << BK) - 1) tabs[16 + tid] = tb.bounds_k[tid];
+    if (tid < (1 << BV) - 1) tabs[32 + tid] = tb.bounds_v[tid];
+    __syncthreads();
+
+    unsigned sat = 0u;
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+#pragma unroll 1
+    for (int job = w; job < 2 * T; job += NW) {
+        const bool is_key = job < T;
+        const int i = is_key ? job : job - T;
+        const int n = start + i, tau = n & 15, g = tau & 7, half = tau >> 3;
+        uint32_t* tw = img + (n / 16 - t0) * (TB / 4);
+        const __half* src = (is_key ? a.k_new : a.v_new) +
+                            (((size_t)b * a.Hkv + hkv) * (size_t)T + i) * D + lane * VPL;
+        double x[VPL];
+#pragma unroll
+        for (int k = 0; k < VPL; k += 2) {
+            const __half2 p = *reinterpret_cast<const __half2*>(src + k);
+            x[k] = (double)__low2float(p);
+            x[k + 1] = (double)__high2float(p);
+        }
+        double ss = 0.0;
+#pragma unroll
+        for (int k = 0; k < VPL; ++k) {
+            ss += x[k] * x[k];
+            x[k] *= (double)tb.signs[lane * VPL + k];
+        }
+        ss = warp_sum(ss);
+        wht_warp<VPL>(x, lane);
+        const double nrm = sqrt(ss);
+        const double scale = nrm > 0.0 ? inv_sqrt_d / nrm : 0.0;
+        if (is_key) {
+            double rr = 0.0;
+#pragma unroll
+            for (int k = 0; k < VPL; ++k) {
+                const int c = lane * VPL + k;
+                const double y = x[k] * scale;
+                const int idx = encode_cell<BK>(y, tabs + 16);
+                const double r = y - tabs[idx];
+                rk[i * D + c] = r;
+                rr += r * r;
+                // K field: token g + 8 (r & 1), coordinate 16 kk + 8 (r >> 1) + 2 t + e
+                const int kk = c >> 4, t = (c & 7) >> 1, e = c & 1;
+                const int p = 4 * kk + 2 * ((c & 15) >> 3) + half;
+                put_field<CB>(tw, 4 * g + t, 2 * BK * p + e * BK, (uint32_t)idx, BK);
+            }
+            rr = warp_sum(rr);
+            if (lane == 0) {
+                uint16_t* nk = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(tw) + NB + 8 * g + 4 * half);
+                nk[0] = norm_to_half_bits(nrm, sat);
+                nk[1] = norm_to_half_bits(sqrt(rr), sat);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < VPL; ++k) {
+                const int c = lane * VPL + k;
+                const int idx = encode_cell<BV>(x[k] * scale, tabs + 32);
+                // V field: token 2 t + 8 (r >> 1) + e, coordinate 16 kk + g' + 8 (r & 1)
+                const int kk = c >> 4, gc = c & 7, t = (tau & 7) >> 1, e = tau & 1;
+                const int p = 4 * kk + 2 * half + ((c & 15) >> 3);
+                put_field<CB>(tw, 4 * gc + t, VB0 + 2 * BV * p + e * BV, (uint32_t)idx, BV);
+            }
+            if (lane == 0)
+                *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(tw) + NB + 64 + 4 * g + 2 * half) =
+                    norm_to_half_bits(nrm, sat);
+        }
+    }
+    __syncthreads();
+    // QJL signs: threads j and M + j own row j of z = S r for all new keys, each
+    // summing half of the coordinates (NT = 2M); the loads of S are independent,
+    // so many are in flight at once
+    {
+        const int j = tid % M, hf = tid / M;
+        double z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0.0;
+#pragma unroll 16
+        for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); ++c) {
+            const double sv = (double)__ldg(tb.s_t + (size_t)c * M + j);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < T) z[i] = fma(sv, rk[i * D + c], z[i]);
+        }
+        if (hf == 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (i < T) zp[i * M + j] = z[i];
+        }
+        __syncthreads();
+        if (hf == 0) {
+            const int kk = j >> 4, t = (j & 7) >> 1, e = j & 1;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (i >= T) break;
+                const int n = start + i, tau = n & 15;
+                const int p = 4 * kk + 2 * ((j & 15) >> 3) + (tau >> 3);
+                put_field<CB>(img + (n / 16 - t0) * (TB / 4), 4 * (tau & 7) + t,
+                              SB0 + 32 * (p >> 4) + 16 * e + (p & 15),
+                              z[i] + zp[i * M + j] >= 0.0 ? 1u : 0u, 1);
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < ntile * TB / 16; e += NT)
+        reinterpret_cast<uint4*>(stream + (size_t)t0 * TB)[e] = reinterpret_cast<const uint4*>(img)[e];
+    if (sat) atomicOr(tb.status, TQ_STATUS_NORM_SAT);
+}
+
+// Prologue launch of a decode step with new tokens: CTAs (x < units, b) run
+// the query prologue, CTAs (units + h, b) append the new tokens of (b, kv head
+// h), side by side; the split kernel, launched after this one, reads them.
+template <int D, int BITS>
+__global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArgs a)
+{
+    extern __shared__ uint4 app_smem[];
+    const int units = a.Hkv * a.plan.groups;
+    if ((int)blockIdx.x >= units)
+        append_tokens<D, BITS>(tb, a, blockIdx.y, blockIdx.x - units, reinterpret_cast<uint8_t*>(app_smem));
+    else
+        prologue_body<D>(tb, a);
+}
+
 
 // ---------------------------------------------------------------- reduction
 // One CTA per (query head, batch): merges the partials of the CTAs whose
@@ -775,8 +988,18 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
     static unsigned long long done_scores = 0, done_attend = 0;
     if (a.tile_bytes != Tr::TILE_BYTES) return cudaErrorInvalidValue;   // the bulk copies' size
     const int units = a.Hkv * a.plan.groups;
-    attend_prologue<D><<<dim3(units, a.B), 2 * D, 0, st>>>(tb, a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (a.k_new != nullptr && a.T > 0) {
+        static unsigned long long done_append = 0;
+        constexpr int TB = 16 * (BITS * D / 4 + 6);
+        const size_t smem = 2 * (size_t)TB + 8 * (48 + (size_t)16 * D + (size_t)16 * D);
+        auto kern = append_prologue<D, BITS>;
+        if ((e = allow_smem(kern, smem, done_append)) != cudaSuccess) return e;
+        kern<<<dim3(units + a.Hkv, a.B), 2 * D, smem, st>>>(tb, a);
+    } else {
+        attend_prologue<D><<<dim3(units, a.B), 2 * D, 0, st>>>(tb, a);
+    }
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (scores) {
         auto kern = attend_scores<D, BITS>;

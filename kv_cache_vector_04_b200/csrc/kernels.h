@@ -39,6 +39,12 @@ struct AttendArgs {
     float* partial;           // workspace: [ctas + B*Hkv*groups][8][d + 2], slot = CTA + unit
     float* out;               // [B][Hq][d] (attend) or scores [B][Hq][max_len]
     AttendPlan plan;
+    // fused append (tq_append_attend with 1 <= T <= 16; k_new == nullptr otherwise)
+    const __half* k_new;      // [B][Hkv][T][d]
+    const __half* v_new;      // [B][Hkv][T][d]
+    const int32_t* start_pos; // [B]
+    int T;
+    uint8_t* cache_w;         // the cache, writable
 };
 
 cudaError_t launch_quantize(int d, int bits, const DevTables& tb, const QuantizeArgs& a,
