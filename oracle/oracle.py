@@ -62,13 +62,13 @@ def _load():
         "oracle_rotate": (None, [i32, P, P, P]),
         "oracle_rotate_inverse": (None, [i32, P, P, P]),
         "oracle_encode": (i32, [ctypes.c_double, P, i32]),
-        "oracle_quantize_keys": (None, [i32, i32, P, P, P, P, P, i32, P, P, P, P, P, P, P]),
+        "oracle_quantize_keys": (None, [i32, i32, P, P, P, P, P, i32, i32, P, P, P, P, P, P, P]),
         "oracle_quantize_values": (None, [i32, i32, P, P, P, P, i32, P, P, P, P]),
-        "oracle_tile_bytes": (ctypes.c_int64, [i32, i32]),
-        "oracle_pack_stream": (None, [i32, i32, i32, P, P, P, P, P, P, P]),
-        "oracle_unpack_stream": (None, [i32, i32, i32, P, P, P, P, P, P, P]),
-        "oracle_attend_head": (None, [i32, i32, P, i32, P, P, P, P, P, P, P, P, P, P, P, P]),
-        "oracle_attend_batch": (None, [i32, i32, i32, i32, i32, P, P, i32, P, P, P, P,
+        "oracle_tile_bytes": (ctypes.c_int64, [i32, i32, i32, i32]),
+        "oracle_pack_stream": (None, [i32, i32, i32, i32, i32, P, P, P, P, P, P, P]),
+        "oracle_unpack_stream": (None, [i32, i32, i32, i32, i32, P, P, P, P, P, P, P]),
+        "oracle_attend_head": (None, [i32, i32, P, i32, i32, P, P, P, P, P, P, P, P, P, P, P, P]),
+        "oracle_attend_batch": (None, [i32, i32, i32, i32, i32, P, P, i32, i32, P, P, P, P,
                                         P, P, P, P, P, P, P, P]),
         "oracle_distortion_mc": (ctypes.c_double, [i32, i32, i32, u64]),
         "oracle_ip_trials": (None, [i32, i32, i32, u64, P, P, P, P]),
@@ -170,15 +170,30 @@ def encode(y: float, bounds: np.ndarray) -> int:
 
 
 class Tables:
-    """The method's tables for (d, bits, seed), built by the oracle itself."""
+    """The method's tables for (d, bits, seed), built by the oracle itself.
 
-    def __init__(self, d: int, bits: int, seed: int):
+    fmt = (B_K, B_V, qjl): key and value cell bits and whether keys carry the
+    1-bit QJL sketch. The default is TurboQuant at b bits, (b - 1, b, 1); the
+    MSE-only key formats ("nc", [MUNINN §MSE-Only vs QJL]) have qjl = 0."""
+
+    def __init__(self, d: int, bits: int, seed: int, fmt: tuple | None = None):
         self.d, self.bits, self.seed, self.m = d, bits, seed, d
-        self.BK, self.BV = bits - 1, bits
+        self.fmt = fmt_of(bits) if fmt is None else tuple(int(x) for x in fmt)
+        self.BK, self.BV, self.qjl = self.fmt
         self.D = rotation_signs(d, seed)
         self.S = qjl_matrix(d, d, seed)
         self.cK, self.tK = codebook(self.BK, d)
         self.cV, self.tV = codebook(self.BV, d)
+
+
+def fmt_of(x) -> tuple:
+    """(B_K, B_V, qjl) of a format given as b (TurboQuant at b bits), a tuple or Tables."""
+    if isinstance(x, Tables):
+        return x.fmt
+    if isinstance(x, tuple):
+        return tuple(int(v) for v in x)
+    b = int(x)
+    return (b - 1, b, 1)
 
 
 # --------------------------------------------------------------------------
@@ -195,7 +210,7 @@ def quantize_keys(tab: Tables, x: np.ndarray):
         kydist=np.zeros((N, d), np.float64), zabs=np.zeros((N, d), np.float64),
         ksat=np.zeros(N, np.uint8))
     _load().oracle_quantize_keys(d, N, _p(x), _p(tab.D), _p(tab.S), _p(tab.cK), _p(tab.tK),
-                                 tab.BK, _p(out["kidx"]), _p(out["ksign"]), _p(out["knorm"]),
+                                 tab.BK, tab.qjl, _p(out["kidx"]), _p(out["ksign"]), _p(out["knorm"]),
                                  _p(out["rnorm"]), _p(out["kydist"]), _p(out["zabs"]),
                                  _p(out["ksat"]))
     return out
@@ -218,28 +233,32 @@ def quantize(tab: Tables, k: np.ndarray, v: np.ndarray):
     return out
 
 
-def tile_bytes(d: int, b: int) -> int:
-    return int(_load().oracle_tile_bytes(d, b))
+def tile_bytes(d: int, fmt) -> int:
+    """Bytes of a 16-token tile; fmt as for fmt_of (b, (B_K, B_V, qjl) or Tables)."""
+    kb, vb, qjl = fmt_of(fmt)
+    return int(_load().oracle_tile_bytes(d, kb, vb, qjl))
 
 
-def pack_stream(d: int, b: int, codes: dict, N: int | None = None) -> np.ndarray:
+def pack_stream(d: int, fmt, codes: dict, N: int | None = None) -> np.ndarray:
     """Pack tokens [0, N) of one (batch, kv-head) stream into 16-token tiles."""
+    kb, vb, qjl = fmt_of(fmt)
     N = codes["kidx"].shape[0] if N is None else N
     nt = (N + TILE - 1) // TILE
-    out = np.zeros(nt * tile_bytes(d, b), dtype=np.uint8)
+    out = np.zeros(nt * tile_bytes(d, (kb, vb, qjl)), dtype=np.uint8)
     c = {k: np.ascontiguousarray(codes[k]) for k in
          ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm")}
-    _load().oracle_pack_stream(d, b, N, _p(c["kidx"]), _p(c["ksign"]), _p(c["knorm"]),
+    _load().oracle_pack_stream(d, kb, vb, qjl, N, _p(c["kidx"]), _p(c["ksign"]), _p(c["knorm"]),
                                _p(c["rnorm"]), _p(c["vidx"]), _p(c["vnorm"]), _p(out))
     return out
 
 
-def unpack_stream(d: int, b: int, N: int, tiles: np.ndarray) -> dict:
+def unpack_stream(d: int, fmt, N: int, tiles: np.ndarray) -> dict:
     tiles = np.ascontiguousarray(tiles, dtype=np.uint8)
     out = dict(kidx=np.zeros((N, d), np.uint8), ksign=np.zeros((N, d), np.uint8),
                knorm=np.zeros(N, np.uint16), rnorm=np.zeros(N, np.uint16),
                vidx=np.zeros((N, d), np.uint8), vnorm=np.zeros(N, np.uint16))
-    _load().oracle_unpack_stream(d, b, N, _p(tiles), _p(out["kidx"]), _p(out["ksign"]),
+    kb, vb, qjl = fmt_of(fmt)
+    _load().oracle_unpack_stream(d, kb, vb, qjl, N, _p(tiles), _p(out["kidx"]), _p(out["ksign"]),
                                  _p(out["knorm"]), _p(out["rnorm"]), _p(out["vidx"]),
                                  _p(out["vnorm"]))
     return out
@@ -253,7 +272,7 @@ def attend_head(tab: Tables, q_bits: np.ndarray, q_is_bf16: bool, codes: dict, N
     lg = np.zeros(max(N, 1), np.float64)
     c = {k: np.ascontiguousarray(codes[k]) for k in
          ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm")}
-    _load().oracle_attend_head(d, N, _p(q_bits), int(q_is_bf16), _p(tab.D), _p(tab.S),
+    _load().oracle_attend_head(d, N, _p(q_bits), int(q_is_bf16), tab.qjl, _p(tab.D), _p(tab.S),
                                _p(tab.cK), _p(tab.cV), _p(c["kidx"]), _p(c["ksign"]),
                                _p(c["knorm"]), _p(c["rnorm"]), _p(c["vidx"]), _p(c["vnorm"]),
                                _p(o), _p(lg))
@@ -271,7 +290,7 @@ def attend_batch(tab: Tables, q_bits: np.ndarray, q_is_bf16: bool, codes: dict,
     sl = np.ascontiguousarray(seq_len, dtype=np.int32)
     c = {k: np.ascontiguousarray(codes[k]) for k in
          ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm")}
-    _load().oracle_attend_batch(d, B, Hq, Hkv, cap, _p(sl), _p(q_bits), int(q_is_bf16),
+    _load().oracle_attend_batch(d, B, Hq, Hkv, cap, _p(sl), _p(q_bits), int(q_is_bf16), tab.qjl,
                                 _p(tab.D), _p(tab.S), _p(tab.cK), _p(tab.cV), _p(c["kidx"]),
                                 _p(c["ksign"]), _p(c["knorm"]), _p(c["rnorm"]), _p(c["vidx"]),
                                 _p(c["vnorm"]), _p(out), _p(lg) if lg is not None else None)

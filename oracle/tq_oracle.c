@@ -325,9 +325,11 @@ static double rotate_unit(int d, const int8_t* D, const uint16_t* x, double* y)
  * y = Pi (x/||x||), idx_i = encode(y_i) with the (B_K)-bit codebook,
  * r = y - c[idx], rho = ||r||, z = S r, sign bit s_j = [z_j >= 0].
  * Stores ||x|| and rho as fp16. ydist/zabs report how close each decision was
- * to its threshold (for counting boundary cases in parity tests). */
+ * to its threshold (for counting boundary cases in parity tests).
+ * With qjl = 0 (the MSE-only key format, [MUNINN §MSE-Only vs QJL]) only the
+ * cells and ||x|| are produced: signs, rho and zabs are left at 0. */
 void oracle_quantize_keys(int d, int N, const uint16_t* x, const int8_t* D, const double* S,
-                          const float* cK, const float* tK, int BK,
+                          const float* cK, const float* tK, int BK, int qjl,
                           uint8_t* kidx, uint8_t* ksign, uint16_t* knorm, uint16_t* rnorm,
                           double* ydist, double* zabs, uint8_t* sat)
 {
@@ -347,12 +349,13 @@ void oracle_quantize_keys(int d, int N, const uint16_t* x, const int8_t* D, cons
         }
         for (int j = 0; j < m; ++j) {
             double z = 0.0;
-            for (int i = 0; i < d; ++i) z += S[(size_t)j * d + i] * r[i];
-            ksign[(size_t)n * m + j] = (z >= 0.0) ? 1 : 0;
-            if (zabs) zabs[(size_t)n * m + j] = fabs(z);
+            if (qjl)
+                for (int i = 0; i < d; ++i) z += S[(size_t)j * d + i] * r[i];
+            ksign[(size_t)n * m + j] = (qjl && z >= 0.0) ? 1 : 0;
+            if (zabs) zabs[(size_t)n * m + j] = qjl ? fabs(z) : 0.0;
         }
         knorm[n] = norm_to_half(nrm, &s0);
-        rnorm[n] = norm_to_half(sqrt(rr), &s0);
+        rnorm[n] = qjl ? norm_to_half(sqrt(rr), &s0) : 0;
         if (sat) sat[n] = s0;
     }
 }
@@ -379,50 +382,60 @@ void oracle_quantize_values(int d, int N, const uint16_t* x, const int8_t* D,
 }
 
 /* ------------------------------------------------------------------------- */
-/* Packed cache format (this library's own layout; see DESIGN.md "Packed      */
-/* cache format"). A stream of one (batch, kv-head) is a run of 16-token      */
-/* tiles of 16*(b*d/4 + 6) bytes:                                             */
-/*   codes:   4*b*d bytes = 32 lane strings of b*d/8 bytes each, stored as    */
-/*            chunks of C bytes (C = 16, or 8 when b*d/8 is not a multiple   */
-/*            of 16); chunk c of lane l sits at byte (c*32 + l)*C; a lane     */
+/* Packed cache format (this library's own layout). A format is (B_K, B_V,    */
+/* qjl): key cells of B_K bits, value cells of B_V bits, and with qjl = 1 the */
+/* 1-bit QJL sketch of the key residual plus its norm rho. With W = B_K +     */
+/* qjl + B_V, a stream of one (batch, kv-head) is a run of 16-token tiles of  */
+/* 16*(W*d/8 + 4 + 2*qjl) bytes:                                              */
+/*   codes:   2*W*d bytes = 32 lane strings of W*d/16 bytes each, stored as   */
+/*            chunks of C bytes (C = 16, 8 or 4: the largest dividing the    */
+/*            string); chunk c of lane l sits at byte (c*32 + l)*C; a lane    */
 /*            string is its chunks in order, bit k = bit (k%8) of byte k/8.   */
-/*   K norms: 64 bytes; for g = 0..7: fp16 {|k_g|, rho_g, |k_g+8|, rho_g+8}.  */
+/*   K norms: qjl: 64 bytes; for g = 0..7: fp16 {|k_g|, rho_g, |k_g+8|,       */
+/*            rho_g+8}. No qjl: 32 bytes; fp16 {|k_g|, |k_g+8|}.              */
 /*   V norms: 32 bytes; for g = 0..7: fp16 {|v_g|, |v_g+8|}.                  */
 /* Lane l = 4g + t holds, for p = 4kk + r (kk < d/16, r < 4), e in {0,1}:     */
 /*   K code of token g + 8(r&1), coordinate 16kk + 8(r>>1) + 2t + e,          */
 /*        B_K bits at bit 2*B_K*p + e*B_K;                                    */
-/*   sign of the same token for QJL row 16kk + 8(r>>1) + 2t + e,              */
+/*   (qjl) sign of the same token for QJL row 16kk + 8(r>>1) + 2t + e,        */
 /*        at bit B_K*d/2 + 32*(p/16) + 16e + (p%16);                          */
 /*   V code of token 2t + 8(r>>1) + e, coordinate 16kk + g + 8(r&1),          */
-/*        B_V bits at bit (B_K+1)*d/2 + 2*B_V*p + e*B_V.                      */
+/*        B_V bits at bit (B_K+qjl)*d/2 + 2*B_V*p + e*B_V.                    */
+/* The TurboQuant format at b bits is (b-1, b, 1): tiles of 16*(b*d/4 + 6).   */
 /* ------------------------------------------------------------------------- */
 
-int64_t oracle_tile_bytes(int d, int b) { return (int64_t)TQO_TILE * (b * d / 4 + 6); }
-
-static int chunk_bytes(int d, int b) { return ((b * d / 8) % 16 == 0) ? 16 : 8; }
-
-static int64_t lane_bit_addr(int d, int b, int lane, int64_t bit)
+int64_t oracle_tile_bytes(int d, int kb, int vb, int qjl)
 {
-    int C = chunk_bytes(d, b);
+    return (int64_t)TQO_TILE * ((int64_t)(kb + qjl + vb) * d / 8 + 4 + 2 * qjl);
+}
+
+static int chunk_bytes(int d, int kb, int vb, int qjl)
+{
+    int sb = (kb + qjl + vb) * d / 16;
+    return (sb % 16 == 0) ? 16 : (sb % 8 == 0) ? 8 : 4;
+}
+
+static int64_t lane_bit_addr(int C, int lane, int64_t bit)
+{
     int64_t byte = bit >> 3;
     int64_t chunk = byte / C, off = byte % C;
     return ((chunk * 32 + lane) * C + off) * 8 + (bit & 7);
 }
 
-static void put_bits(uint8_t* tile, int d, int b, int lane, int64_t bit, int nbits, unsigned v)
+static void put_bits(uint8_t* tile, int C, int lane, int64_t bit, int nbits, unsigned v)
 {
     for (int k = 0; k < nbits; ++k) {
-        int64_t a = lane_bit_addr(d, b, lane, bit + k);
+        int64_t a = lane_bit_addr(C, lane, bit + k);
         if ((v >> k) & 1) tile[a >> 3] |= (uint8_t)(1u << (a & 7));
         else tile[a >> 3] &= (uint8_t)~(1u << (a & 7));
     }
 }
 
-static unsigned get_bits(const uint8_t* tile, int d, int b, int lane, int64_t bit, int nbits)
+static unsigned get_bits(const uint8_t* tile, int C, int lane, int64_t bit, int nbits)
 {
     unsigned v = 0;
     for (int k = 0; k < nbits; ++k) {
-        int64_t a = lane_bit_addr(d, b, lane, bit + k);
+        int64_t a = lane_bit_addr(C, lane, bit + k);
         v |= (unsigned)((tile[a >> 3] >> (a & 7)) & 1) << k;
     }
     return v;
@@ -435,18 +448,33 @@ static int64_t sign_bit(int p, int e) { return 32LL * (p / 16) + 16 * e + (p % 1
 static void put_half(uint8_t* p, uint16_t h) { p[0] = (uint8_t)(h & 0xff); p[1] = (uint8_t)(h >> 8); }
 static uint16_t get_half(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 
+/* Byte offsets of token slot n (0..15) of a tile: its |k|, its rho (qjl) and its |v|. */
+static void norm_offsets(int d, int kb, int vb, int qjl, int n, int64_t* ok, int64_t* orho,
+                         int64_t* ov)
+{
+    int64_t knoff = 2LL * (kb + qjl + vb) * d, vnoff = knoff + 32 + 32 * qjl;
+    int g = n & 7, h = n >> 3;
+    if (qjl) {
+        *ok = knoff + 8 * g + 4 * h;
+        *orho = *ok + 2;
+    } else {
+        *ok = knoff + 4 * g + 2 * h;
+        *orho = -1;
+    }
+    *ov = vnoff + 4 * g + 2 * h;
+}
+
 /* Pack tokens [0, N) of one stream (codes as produced above) into ceil(N/16)
  * tiles; slots past N in the last tile are zero. */
-void oracle_pack_stream(int d, int b, int N, const uint8_t* kidx, const uint8_t* ksign,
-                        const uint16_t* knorm, const uint16_t* rnorm,
+void oracle_pack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* kidx,
+                        const uint8_t* ksign, const uint16_t* knorm, const uint16_t* rnorm,
                         const uint8_t* vidx, const uint16_t* vnorm, uint8_t* out)
 {
-    int BK = b - 1, BV = b, m = d;
-    int64_t TB = oracle_tile_bytes(d, b);
+    int m = d, C = chunk_bytes(d, kb, vb, qjl);
+    int64_t TB = oracle_tile_bytes(d, kb, vb, qjl);
     int ntiles = (N + TQO_TILE - 1) / TQO_TILE;
     memset(out, 0, (size_t)(TB * ntiles));
-    int64_t sbase = (int64_t)BK * d / 2, vbase = (int64_t)(BK + 1) * d / 2;
-    int64_t knoff = 4LL * b * d, vnoff = knoff + 64;
+    int64_t sbase = (int64_t)kb * d / 2, vbase = (int64_t)(kb + qjl) * d / 2;
     for (int tl = 0; tl < ntiles; ++tl) {
         uint8_t* tile = out + TB * tl;
         for (int lane = 0; lane < 32; ++lane) {
@@ -459,39 +487,39 @@ void oracle_pack_stream(int d, int b, int N, const uint8_t* kidx, const uint8_t*
                     int nv = tl * TQO_TILE + 2 * t + 8 * (r >> 1) + e;
                     int iv = 16 * kk + g + 8 * (r & 1);
                     if (nk < N) {
-                        if (BK > 0)
-                            put_bits(tile, d, b, lane, 2LL * BK * p + e * BK, BK,
-                                     kidx[(size_t)nk * d + ik]);
-                        put_bits(tile, d, b, lane, sbase + sign_bit(p, e), 1,
-                                 ksign[(size_t)nk * m + ik]);
+                        put_bits(tile, C, lane, 2LL * kb * p + e * kb, kb, kidx[(size_t)nk * d + ik]);
+                        if (qjl)
+                            put_bits(tile, C, lane, sbase + sign_bit(p, e), 1,
+                                     ksign[(size_t)nk * m + ik]);
                     }
                     if (nv < N)
-                        put_bits(tile, d, b, lane, vbase + 2LL * BV * p + e * BV, BV,
+                        put_bits(tile, C, lane, vbase + 2LL * vb * p + e * vb, vb,
                                  vidx[(size_t)nv * d + iv]);
                 }
             }
         }
-        for (int g = 0; g < 8; ++g) {
-            for (int h = 0; h < 2; ++h) {
-                int n = tl * TQO_TILE + g + 8 * h;
-                if (n >= N) continue;
-                put_half(tile + knoff + 8 * g + 4 * h, knorm[n]);
-                put_half(tile + knoff + 8 * g + 4 * h + 2, rnorm[n]);
-                put_half(tile + vnoff + 4 * g + 2 * h, vnorm[n]);
-            }
+        for (int n = 0; n < TQO_TILE; ++n) {
+            int tok = tl * TQO_TILE + n;
+            if (tok >= N) continue;
+            int64_t ok, orho, ov;
+            norm_offsets(d, kb, vb, qjl, n, &ok, &orho, &ov);
+            put_half(tile + ok, knorm[tok]);
+            if (qjl) put_half(tile + orho, rnorm[tok]);
+            put_half(tile + ov, vnorm[tok]);
         }
     }
 }
 
-/* Inverse of oracle_pack_stream for tokens [0, N). */
-void oracle_unpack_stream(int d, int b, int N, const uint8_t* in, uint8_t* kidx, uint8_t* ksign,
-                          uint16_t* knorm, uint16_t* rnorm, uint8_t* vidx, uint16_t* vnorm)
+/* Inverse of oracle_pack_stream for tokens [0, N) (signs and rho read as 0
+ * when qjl = 0). */
+void oracle_unpack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* in, uint8_t* kidx,
+                          uint8_t* ksign, uint16_t* knorm, uint16_t* rnorm, uint8_t* vidx,
+                          uint16_t* vnorm)
 {
-    int BK = b - 1, BV = b, m = d;
-    int64_t TB = oracle_tile_bytes(d, b);
+    int m = d, C = chunk_bytes(d, kb, vb, qjl);
+    int64_t TB = oracle_tile_bytes(d, kb, vb, qjl);
     int ntiles = (N + TQO_TILE - 1) / TQO_TILE;
-    int64_t sbase = (int64_t)BK * d / 2, vbase = (int64_t)(BK + 1) * d / 2;
-    int64_t knoff = 4LL * b * d, vnoff = knoff + 64;
+    int64_t sbase = (int64_t)kb * d / 2, vbase = (int64_t)(kb + qjl) * d / 2;
     for (int tl = 0; tl < ntiles; ++tl) {
         const uint8_t* tile = in + TB * tl;
         for (int lane = 0; lane < 32; ++lane) {
@@ -504,25 +532,24 @@ void oracle_unpack_stream(int d, int b, int N, const uint8_t* in, uint8_t* kidx,
                     int nv = tl * TQO_TILE + 2 * t + 8 * (r >> 1) + e;
                     int iv = 16 * kk + g + 8 * (r & 1);
                     if (nk < N) {
-                        kidx[(size_t)nk * d + ik] = (uint8_t)(BK > 0 ?
-                            get_bits(tile, d, b, lane, 2LL * BK * p + e * BK, BK) : 0);
+                        kidx[(size_t)nk * d + ik] = (uint8_t)get_bits(tile, C, lane, 2LL * kb * p + e * kb, kb);
                         ksign[(size_t)nk * m + ik] =
-                            (uint8_t)get_bits(tile, d, b, lane, sbase + sign_bit(p, e), 1);
+                            (uint8_t)(qjl ? get_bits(tile, C, lane, sbase + sign_bit(p, e), 1) : 0);
                     }
                     if (nv < N)
                         vidx[(size_t)nv * d + iv] =
-                            (uint8_t)get_bits(tile, d, b, lane, vbase + 2LL * BV * p + e * BV, BV);
+                            (uint8_t)get_bits(tile, C, lane, vbase + 2LL * vb * p + e * vb, vb);
                 }
             }
         }
-        for (int g = 0; g < 8; ++g) {
-            for (int h = 0; h < 2; ++h) {
-                int n = tl * TQO_TILE + g + 8 * h;
-                if (n >= N) continue;
-                knorm[n] = get_half(tile + knoff + 8 * g + 4 * h);
-                rnorm[n] = get_half(tile + knoff + 8 * g + 4 * h + 2);
-                vnorm[n] = get_half(tile + vnoff + 4 * g + 2 * h);
-            }
+        for (int n = 0; n < TQO_TILE; ++n) {
+            int tok = tl * TQO_TILE + n;
+            if (tok >= N) continue;
+            int64_t ok, orho, ov;
+            norm_offsets(d, kb, vb, qjl, n, &ok, &orho, &ov);
+            knorm[tok] = get_half(tile + ok);
+            rnorm[tok] = qjl ? get_half(tile + orho) : 0;
+            vnorm[tok] = get_half(tile + ov);
         }
     }
 }
@@ -536,8 +563,9 @@ void oracle_unpack_stream(int d, int b, int N, const uint8_t* in, uint8_t* kidx,
  *   q~ = Pi q,  p = S q~,  kappa = sqrt(pi/2)/m,
  *   l_n = |k_n| (<q~, cK[idx_n]> + rho_n kappa <p, 2 s_n - 1>) / sqrt(d),
  *   w = softmax(l),  o = Pi^T sum_n w_n |v_n| cV[vidx_n].
- * N = 0 gives o = 0. logits (if not NULL) receives l. */
-void oracle_attend_head(int d, int N, const uint16_t* q, int q_is_bf16,
+ * With qjl = 0 the QJL term is absent: l_n = |k_n| <q~, cK[idx_n]> / sqrt(d),
+ * the MSE-only estimate. N = 0 gives o = 0. logits (if not NULL) receives l. */
+void oracle_attend_head(int d, int N, const uint16_t* q, int q_is_bf16, int qjl,
                         const int8_t* D, const double* S, const float* cK, const float* cV,
                         const uint8_t* kidx, const uint8_t* ksign, const uint16_t* knorm,
                         const uint16_t* rnorm, const uint8_t* vidx, const uint16_t* vnorm,
@@ -559,8 +587,10 @@ void oracle_attend_head(int d, int N, const uint16_t* q, int q_is_bf16,
     for (int n = 0; n < N; ++n) {
         double ct = 0.0, st = 0.0;
         for (int i = 0; i < d; ++i) ct += qt[i] * (double)cK[kidx[(size_t)n * d + i]];
-        for (int j = 0; j < m; ++j) st += (ksign[(size_t)n * m + j] ? 1.0 : -1.0) * p[j];
-        double kn = oracle_half_to_double(knorm[n]), rn = oracle_half_to_double(rnorm[n]);
+        if (qjl)
+            for (int j = 0; j < m; ++j) st += (ksign[(size_t)n * m + j] ? 1.0 : -1.0) * p[j];
+        double kn = oracle_half_to_double(knorm[n]);
+        double rn = qjl ? oracle_half_to_double(rnorm[n]) : 0.0;
         l[n] = kn * (ct + rn * kappa * st) * inv_sqrt_d;
         if (l[n] > lmax) lmax = l[n];
         if (logits) logits[n] = l[n];
@@ -579,7 +609,7 @@ void oracle_attend_head(int d, int N, const uint16_t* q, int q_is_bf16,
 /* Batched form over (b, query head): codes are stored per (b, kv head) with a
  * stride of `cap` tokens; query head h reads kv head h / (Hq / Hkv). */
 void oracle_attend_batch(int d, int B, int Hq, int Hkv, int cap, const int32_t* seq_len,
-                         const uint16_t* q, int q_is_bf16, const int8_t* D, const double* S,
+                         const uint16_t* q, int q_is_bf16, int qjl, const int8_t* D, const double* S,
                          const float* cK, const float* cV,
                          const uint8_t* kidx, const uint8_t* ksign, const uint16_t* knorm,
                          const uint16_t* rnorm, const uint8_t* vidx, const uint16_t* vnorm,
@@ -591,7 +621,7 @@ void oracle_attend_batch(int d, int B, int Hq, int Hkv, int cap, const int32_t* 
         for (int h = 0; h < Hq; ++h) {
             size_t s = (size_t)b * Hkv + h / g;
             size_t base = s * cap;
-            oracle_attend_head(d, seq_len[b], q + ((size_t)b * Hq + h) * d, q_is_bf16, D, S, cK, cV,
+            oracle_attend_head(d, seq_len[b], q + ((size_t)b * Hq + h) * d, q_is_bf16, qjl, D, S, cK, cV,
                                kidx + base * d, ksign + base * m, knorm + base, rnorm + base,
                                vidx + base * d, vnorm + base, out + ((size_t)b * Hq + h) * d,
                                logits ? logits + ((size_t)b * Hq + h) * cap : NULL);

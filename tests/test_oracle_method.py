@@ -57,6 +57,27 @@ def test_quantize_keys_brute_force_small():
         assert out["rnorm"][n] == np.float16(np.linalg.norm(r)).view(np.uint16)
 
 
+@pytest.mark.parametrize("fmt", [(3, 3, 0), (2, 4, 0)])
+def test_quantize_keys_mse_only_brute_force_small(fmt):
+    # the MSE-only key format: nearest B_K-bit cell, |k| stored, no sketch
+    d = 8
+    tab = O.Tables(d, 3, seed=4, fmt=fmt)
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((40, d)) * 2).astype(np.float16)
+    out = O.quantize(tab, x, x)
+    H = np.array([[(-1) ** bin(i & j).count("1") for j in range(d)] for i in range(d)], float)
+    for n in range(x.shape[0]):
+        xv = x[n].astype(np.float64)
+        y = H @ (tab.D * xv) / math.sqrt(d) / np.linalg.norm(xv)
+        kid = np.array([np.argmin(np.abs(yi - tab.cK.astype(np.float64))) for yi in y])
+        vid = np.array([np.argmin(np.abs(yi - tab.cV.astype(np.float64))) for yi in y])
+        assert np.array_equal(out["kidx"][n], kid)
+        assert np.array_equal(out["vidx"][n], vid)
+        assert kid.max() < (1 << fmt[0]) and vid.max() < (1 << fmt[1])
+        assert not out["ksign"][n].any() and out["rnorm"][n] == 0
+        assert out["knorm"][n] == np.float16(np.linalg.norm(xv)).view(np.uint16)
+
+
 def test_exact_cancellation_meets_the_tie_rule():
     # D o x = (1, 1, 0, ...) gives Walsh-Hadamard sums 1 + (-1)^(i&1): every
     # odd coordinate of the rotated vector is exactly 0, which the strict '>'
@@ -154,6 +175,68 @@ def test_pack_round_trip(d, b):
                 assert np.unpackbits(blk).mean() > 0.4
 
 
+FORMATS = [(1, 2, 1), (2, 3, 1), (3, 4, 1), (2, 2, 0), (3, 3, 0), (4, 4, 0), (3, 4, 0)]
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_pack_round_trip_formats(d, fmt):
+    kb, vb, qjl = fmt
+    rng = np.random.default_rng(d + 7 * kb + vb)
+    for N in (1, 17, 32):
+        codes = dict(
+            kidx=rng.integers(0, 1 << kb, (N, d), dtype=np.uint8),
+            ksign=rng.integers(0, 2, (N, d), dtype=np.uint8) * qjl,
+            knorm=rng.integers(0, 0x7BFF, N, dtype=np.uint16),
+            rnorm=rng.integers(0, 0x7BFF, N, dtype=np.uint16) * qjl,
+            vidx=rng.integers(0, 1 << vb, (N, d), dtype=np.uint8),
+            vnorm=rng.integers(0, 0x7BFF, N, dtype=np.uint16))
+        tiles = O.pack_stream(d, fmt, codes)
+        # per head-token: key cells + sketch + |k| (+ rho), value cells + |v|
+        per_token = (kb + qjl) * d / 8 + 2 + 2 * qjl + vb * d / 8 + 2
+        assert tiles.size == ((N + 15) // 16) * 16 * per_token
+        back = O.unpack_stream(d, fmt, N, tiles)
+        for key in codes:
+            assert np.array_equal(back[key], codes[key]), (key, N)
+
+
+@pytest.mark.parametrize("fmt", FORMATS)
+def test_pack_fields_tile_the_tile(fmt):
+    # Packing one field at a time: every field sets exactly its own bits, no
+    # two fields share a bit, and together they cover the whole tile.
+    d = 64
+    kb, vb, qjl = fmt
+    N = 16
+    zero = dict(kidx=np.zeros((N, d), np.uint8), ksign=np.zeros((N, d), np.uint8),
+                knorm=np.zeros(N, np.uint16), rnorm=np.zeros(N, np.uint16),
+                vidx=np.zeros((N, d), np.uint8), vnorm=np.zeros(N, np.uint16))
+    TB = O.tile_bytes(d, fmt)
+    owner = np.full(TB * 8, -1)
+    fields = [("kidx", (1 << kb) - 1, kb), ("vidx", (1 << vb) - 1, vb)]
+    if qjl:
+        fields.append(("ksign", 1, 1))
+    fid = 0
+    for name, val, width in fields:
+        for n in range(N):
+            for i in range(d):
+                c = {k: v.copy() for k, v in zero.items()}
+                c[name][n, i] = val
+                bits = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+                assert bits.size == width
+                assert np.all(owner[bits] == -1)
+                owner[bits] = fid
+                fid += 1
+    for name in ("knorm", "vnorm") + (("rnorm",) if qjl else ()):
+        for n in range(N):
+            c = {k: v.copy() for k, v in zero.items()}
+            c[name][n] = 0xFFFF
+            bits = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+            assert bits.size == 16 and np.all(owner[bits] == -1)
+            owner[bits] = fid
+            fid += 1
+    assert np.all(owner >= 0)
+
+
 def test_pack_sizes_match_pages(golden):
     vals = {r[0]: float(r[1]) for r in golden("pages_numbers.txt")}
     d = 128
@@ -182,9 +265,11 @@ def _random_codes(tab, N, seed, kscale=1.0):
     return O.quantize(tab, k, v)
 
 
-@pytest.mark.parametrize("d,bits", [(64, 2), (128, 3), (256, 4)])
-def test_attention_equals_sdpa_over_reconstructed(d, bits):
-    tab = O.Tables(d, bits, seed=5)
+@pytest.mark.parametrize("d,bits,fmt", [(64, 2, None), (128, 3, None), (256, 4, None),
+                                        (128, 3, (3, 3, 0)), (64, 4, (3, 4, 0))])
+def test_attention_equals_sdpa_over_reconstructed(d, bits, fmt):
+    # with fmt (B_K, B_V, 0) the keys are the MSE-only reconstructions
+    tab = O.Tables(d, bits, seed=5, fmt=fmt)
     N = 77
     codes = _random_codes(tab, N, seed=d + bits, kscale=2.0)
     kh, vh = O.reconstruct(tab, codes, N)
