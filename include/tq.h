@@ -70,15 +70,16 @@ typedef struct tq_ctx tq_ctx; /* opaque: the codebook, rotation and QJL tables o
 /* Sizes of the packed cache (see "Packed cache format" below). */
 typedef struct {
     int32_t d;                 /* head dimension: 64, 128 or 256                          */
-    int32_t bits;              /* b: 2, 3 or 4 bits per coordinate (K: b-1 + 1 QJL; V: b) */
+    int32_t bits;              /* b = B_V (TurboQuant at b bits: K b-1 + 1 QJL; V b)      */
     int32_t m;                 /* QJL rows, = d                                           */
-    int32_t kbits, vbits;      /* B_K = b - 1, B_V = b                                    */
+    int32_t kbits, vbits;      /* B_K, B_V: key and value cell bits                       */
     int32_t tile;              /* TQ_TILE                                                 */
-    int64_t k_bytes_per_token; /* b*d/8 + 4: codes + signs + fp16 |k| + fp16 |r|          */
-    int64_t v_bytes_per_token; /* b*d/8 + 2: codes + fp16 |v|                             */
+    int64_t k_bytes_per_token; /* (B_K+qjl)*d/8 + 2 + 2*qjl: codes, signs, |k|, rho       */
+    int64_t v_bytes_per_token; /* B_V*d/8 + 2: codes + fp16 |v|                           */
     int64_t tile_bytes;        /* TQ_TILE * (k_bytes_per_token + v_bytes_per_token)       */
-    int64_t code_bytes;        /* 4*b*d: the code region at the start of each tile         */
-    int32_t chunk_bytes;       /* 16, or 8 when b*d/8 is not a multiple of 16             */
+    int64_t code_bytes;        /* 2*W*d, W = B_K + qjl + B_V: the tile's code region      */
+    int32_t chunk_bytes;       /* 16, 8 or 4: the largest dividing a lane string (W*d/16)  */
+    int32_t qjl;               /* 1: keys carry the QJL sketch and rho; 0: MSE-only keys  */
 } tq_layout;
 
 /* A packed cache of B sequences x Hkv kv heads x `capacity` token slots.
@@ -92,23 +93,26 @@ typedef struct {
 } tq_cache;
 
 /*
- * Packed cache format (one 16-token tile of one (batch, kv head)):
- *  bytes [0, 4bd): the code region. It holds 32 "lane strings" of b*d/8 bytes,
+ * Packed cache format (one 16-token tile of one (batch, kv head)). A format is
+ * (B_K, B_V, qjl); TurboQuant at b bits is (b-1, b, 1), where W = B_K + qjl +
+ * B_V = 2b, so that the code region is 4bd bytes and a lane string b*d/8 bytes:
+ *  bytes [0, 2Wd): the code region. It holds 32 "lane strings" of W*d/16 bytes,
  *    stored in chunks of chunk_bytes: chunk c of lane l is at byte
  *    (c*32 + l)*chunk_bytes; a lane string is its chunks in order and bit k of
  *    it is bit k%8 of its byte k/8. Lane l = 4g + t (g < 8, t < 4) holds, for
  *    p = 4kk + r (kk < d/16, r < 4) and e in {0, 1}:
  *      K code of token g + 8(r&1), coordinate 16kk + 8(r>>1) + 2t + e:
  *        B_K bits at 2*B_K*p + e*B_K;
- *      QJL sign bit of the same token, row 16kk + 8(r>>1) + 2t + e:
+ *      (qjl = 1) QJL sign bit of the same token, row 16kk + 8(r>>1) + 2t + e:
  *        at B_K*d/2 + 32*(p/16) + 16e + (p%16)  (1 = S r >= 0);
  *      V code of token 2t + 8(r>>1) + e, coordinate 16kk + g + 8(r&1):
- *        B_V bits at (B_K+1)*d/2 + 2*B_V*p + e*B_V.
+ *        B_V bits at (B_K+qjl)*d/2 + 2*B_V*p + e*B_V.
  *    (Lane l's bits are exactly the operands that lane l of a warp needs for
  *    the m16n8k16 tensor-core fragments of the attention kernel, so each lane
  *    streams its own bytes with 128-bit coalesced loads.)
- *  bytes [4bd, 4bd+64): K norms; for g = 0..7, fp16 {|k_g|, rho_g, |k_g+8|, rho_g+8}.
- *  bytes [4bd+64, 4bd+96): V norms; for g = 0..7, fp16 {|v_g|, |v_g+8|}.
+ *  then the K norms: qjl = 1: 64 bytes, for g = 0..7, fp16 {|k_g|, rho_g,
+ *    |k_g+8|, rho_g+8}; qjl = 0: 32 bytes, fp16 {|k_g|, |k_g+8|};
+ *  then the V norms: 32 bytes; for g = 0..7, fp16 {|v_g|, |v_g+8|}.
  * Codes are cell indices of the sorted codebook (0 = most negative). Norms are
  * fp16, round to nearest even, saturating at 65504.
  */
@@ -127,6 +131,17 @@ typedef struct {
  * *out receives a new context (owned by the caller; free with tq_destroy).
  * Allocates a small device block (< 600 KB) and synchronizes. */
 int tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
+
+/* tq_init for any built format (B_K = kbits, B_V = vbits, QJL sketch on keys
+ * iff qjl = 1); tq_init(d, b, ...) is tq_init_ex(d, b - 1, b, 1, ...). Built:
+ * qjl = 1 with kbits = vbits - 1 and vbits in {2, 3, 4} (TurboQuant), and the
+ * MSE-only key formats qjl = 0 with (kbits, vbits) in {(2,2), (3,3), (4,4),
+ * (3,4)}: the "nc" and k3v4-nc variants of the method table in the vLLM
+ * section ("vLLM 工程師的實測") of turboquant-kvquant-vllm-benchmark, read as
+ * "no QJL correction" ([MUNINN] §"MSE-Only vs QJL" contrasts the two). Without
+ * QJL the logit is |k| <Pi q, cK[idx]> / sqrt(d), the biased MSE-only
+ * estimate. Other formats return TQ_ERR_UNSUPPORTED. */
+int tq_init_ex(int d, int kbits, int vbits, int qjl, uint64_t seed, tq_ctx** out);
 
 /* Free a context and its device tables. NULL is ignored. */
 void tq_destroy(tq_ctx* ctx);

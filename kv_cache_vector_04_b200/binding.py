@@ -32,7 +32,7 @@ TQ_DTYPE_F16 = 0
 TQ_DTYPE_BF16 = 1
 
 # every symbol include/tq.h declares
-EXPORTS = ("tq_init", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
+EXPORTS = ("tq_init", "tq_init_ex", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
            "tq_build_tables", "tq_quantize", "tq_attend_workspace", "tq_attend", "tq_scores",
            "tq_attend_noalloc", "tq_append_attend", "tq_status", "tq_copy", "tq_strerror")
 TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -49,7 +49,7 @@ class _Layout(ctypes.Structure):
                 ("kbits", ctypes.c_int32), ("vbits", ctypes.c_int32), ("tile", ctypes.c_int32),
                 ("k_bytes_per_token", ctypes.c_int64), ("v_bytes_per_token", ctypes.c_int64),
                 ("tile_bytes", ctypes.c_int64), ("code_bytes", ctypes.c_int64),
-                ("chunk_bytes", ctypes.c_int32)]
+                ("chunk_bytes", ctypes.c_int32), ("qjl", ctypes.c_int32)]
 
 
 class _Cache(ctypes.Structure):
@@ -65,6 +65,7 @@ def _load(path: str = LIB_PATH):
     P, I, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
     sig = {
         "tq_init": (I, [I, I, U64, ctypes.POINTER(P)]),
+        "tq_init_ex": (I, [I, I, I, I, U64, ctypes.POINTER(P)]),
         "tq_destroy": (None, [P]),
         "tq_cache_layout": (I, [P, ctypes.POINTER(_Layout)]),
         "tq_cache_bytes": (I, [P, I, I, I, ctypes.POINTER(SZ)]),
@@ -125,11 +126,14 @@ def _dev(t: torch.Tensor, name: str, dtype=None):
 # ------------------------------------------------------------------ context
 
 class Context:
-    """Handle of a tq_ctx: the tables of one (d, bits, seed) on one device."""
+    """Handle of a tq_ctx: the tables of one (d, format, seed) on one device.
+    fmt = (B_K, B_V, qjl); TurboQuant at b bits is (b - 1, b, 1)."""
 
-    def __init__(self, handle: int, d: int, bits: int, seed: int, device: int):
+    def __init__(self, handle: int, d: int, bits: int, seed: int, device: int,
+                 fmt: tuple | None = None):
         self._h = ctypes.c_void_p(handle)
         self.d, self.bits, self.seed, self.device = d, bits, seed, device
+        self.fmt = (bits - 1, bits, 1) if fmt is None else tuple(fmt)
 
     @property
     def handle(self):
@@ -163,6 +167,15 @@ def tq_init(d: int, bits: int, seed: int) -> Context:
     h = ctypes.c_void_p()
     _check(_lib.tq_init(int(d), int(bits), ctypes.c_uint64(seed), ctypes.byref(h)), "tq_init")
     return Context(h.value, d, bits, seed, torch.cuda.current_device())
+
+
+def tq_init_ex(d: int, kbits: int, vbits: int, qjl: int, seed: int) -> Context:
+    """A context of any built format: (kbits, vbits, qjl) = (B_K, B_V, QJL on keys)."""
+    h = ctypes.c_void_p()
+    _check(_lib.tq_init_ex(int(d), int(kbits), int(vbits), int(qjl), ctypes.c_uint64(seed),
+                           ctypes.byref(h)), "tq_init_ex")
+    return Context(h.value, d, vbits, seed, torch.cuda.current_device(),
+                   fmt=(int(kbits), int(vbits), int(qjl)))
 
 
 def tq_destroy(ctx: Context):

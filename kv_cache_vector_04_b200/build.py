@@ -18,8 +18,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["api.cu", "quantize.cu", "attend.cu", "noalloc.cu", "tables.cpp"]
-HEADERS = ["device_common.cuh", "kernels.h", "tables.h"]
+SOURCES = ["api.cu", "quantize.cu", "attend.cu", "attend_d64.cu", "attend_d128.cu",
+           "attend_d256.cu", "noalloc.cu", "tables.cpp"]
+HEADERS = ["device_common.cuh", "kernels.h", "tables.h", "attend_impl.cuh"]
 
 
 def nvcc_path() -> str:
@@ -44,20 +45,36 @@ def is_stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object (in parallel: the kernel templates are
+    instantiated for every format), then link libtq.so."""
     if not force and not is_stale():
         return LIB
+    import concurrent.futures
+    import tempfile
     nvcc = nvcc_path()
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc, "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-ffp-contract=off",
-           "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-           "-I", INCLUDE, "-I", CSRC, "-o", tmp]
+    flags = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-ffp-contract=off",
+             "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-I", INCLUDE, "-I", CSRC]
     if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    cmd += ["-lcudart"]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+        flags += ["-Xptxas", "-v"]
+    with tempfile.TemporaryDirectory(prefix="tq_build_") as tmpdir:
+        def compile_one(src):
+            obj = os.path.join(tmpdir, src + ".o")
+            r = subprocess.run([nvcc] + flags + ["-c", os.path.join(CSRC, src), "-o", obj],
+                               stdout=subprocess.PIPE, stderr=subprocess.STDOUT, text=True)
+            return src, obj, r.returncode, r.stdout
+        workers = max(1, min(len(SOURCES), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+            results = list(ex.map(compile_one, SOURCES))
+        failed = [r for r in results if r[2] != 0]
+        for src, _, rc, out in results:
+            if out and (verbose or rc != 0):
+                sys.stdout.write(out)
+        if failed:
+            raise subprocess.CalledProcessError(failed[0][2], "nvcc -c " + failed[0][0])
+        tmp = LIB + ".tmp%d" % os.getpid()
+        subprocess.run([nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp]
+                       + [r[1] for r in results] + ["-lcudart"], check=True)
+        os.replace(tmp, LIB)
     return LIB
 
 

@@ -14,7 +14,7 @@
 #include "tq.h"
 
 struct tq_ctx {
-    int d = 0, bits = 0, device = 0, num_sms = 148;
+    int d = 0, bits = 0, kbits = 0, vbits = 0, qjl = 1, device = 0, num_sms = 148;
     tq::HostTables host;
     void* dev_block = nullptr;
     tq::DevTables tables{};
@@ -22,9 +22,15 @@ struct tq_ctx {
 
 namespace {
 
-bool supported(int d, int bits)
+// The built formats (B_K, B_V, qjl): TurboQuant at 2, 3, 4 bits, and the
+// MSE-only key formats 2/2, 3/3, 4/4 and 3/4 bits.
+bool supported(int d, int kbits, int vbits, int qjl)
 {
-    return (d == 64 || d == 128 || d == 256) && bits >= 2 && bits <= 4;
+    if (d != 64 && d != 128 && d != 256) return false;
+    if (qjl == 1) return vbits >= 2 && vbits <= 4 && kbits == vbits - 1;
+    if (qjl == 0)
+        return (kbits == vbits && kbits >= 2 && kbits <= 4) || (kbits == 3 && vbits == 4);
+    return false;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -45,22 +51,29 @@ int check_device(const tq_ctx* ctx)
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-tq_layout make_layout(int d, int bits)
+tq_layout make_layout(int d, int kbits, int vbits, int qjl)
 {
     tq_layout L{};
+    const int w = kbits + qjl + vbits;   // bits per coordinate pair-slot of a lane string
     L.d = d;
-    L.bits = bits;
+    L.bits = vbits;
     L.m = d;
-    L.kbits = bits - 1;
-    L.vbits = bits;
+    L.kbits = kbits;
+    L.vbits = vbits;
     L.tile = TQ_TILE;
-    L.k_bytes_per_token = bits * d / 8 + 4;
-    L.v_bytes_per_token = bits * d / 8 + 2;
+    L.k_bytes_per_token = (int64_t)(kbits + qjl) * d / 8 + 2 + 2 * qjl;
+    L.v_bytes_per_token = (int64_t)vbits * d / 8 + 2;
     L.tile_bytes = TQ_TILE * (L.k_bytes_per_token + L.v_bytes_per_token);
-    L.code_bytes = 4LL * bits * d;
-    L.chunk_bytes = ((bits * d / 8) % 16 == 0) ? 16 : 8;
+    L.code_bytes = 2LL * w * d;
+    const int sb = w * d / 16;
+    L.chunk_bytes = (sb % 16 == 0) ? 16 : (sb % 8 == 0) ? 8 : 4;
+    L.qjl = qjl;
     return L;
 }
+
+tq_layout ctx_layout(const tq_ctx* ctx) { return make_layout(ctx->d, ctx->kbits, ctx->vbits, ctx->qjl); }
+
+tq::Format ctx_format(const tq_ctx* ctx) { return tq::Format{ctx->d, ctx->kbits, ctx->vbits, ctx->qjl}; }
 
 int check_cache(const tq_ctx* ctx, const tq_cache* c, int B, int Hkv)
 {
@@ -179,7 +192,7 @@ int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const 
     if (B > 65535 || (long long)Hkv * ((Hq / Hkv + 7) / 8) > 65535 || Hq > 65535)
         return TQ_ERR_INVALID_ARG;
     if ((rc = check_device(ctx))) return rc;
-    const tq::AttendPlan plan = tq::plan_attend(ctx->d, B, Hq, Hkv, max_len, ctx->num_sms);
+    const tq::AttendPlan plan = tq::plan_attend(ctx_format(ctx), B, Hq, Hkv, max_len, ctx->num_sms);
     if (!ws || !aligned(ws, 256)) return TQ_ERR_INVALID_ARG;
     if (ws_bytes < plan.total_bytes) return TQ_ERR_WORKSPACE;
     if (!aligned(q, 16) || !aligned(out, 16)) return TQ_ERR_INVALID_ARG;
@@ -208,14 +221,14 @@ int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const 
     a.Hkv = Hkv;
     a.capacity = cache->capacity;
     a.max_len = max_len;
-    a.tile_bytes = make_layout(ctx->d, ctx->bits).tile_bytes;
+    a.tile_bytes = ctx_layout(ctx).tile_bytes;
     a.qfrag = static_cast<uint32_t*>(ws);
     a.prefix = reinterpret_cast<long long*>(static_cast<uint8_t*>(ws) + align256(plan.qfrag_bytes));
     a.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(plan.qfrag_bytes) +
                                          align256(plan.prefix_bytes));
     a.out = out;
     a.plan = plan;
-    const cudaError_t e = tq::launch_attend(ctx->d, ctx->bits, ctx->tables, a, scores,
+    const cudaError_t e = tq::launch_attend(ctx_format(ctx), ctx->tables, a, scores,
                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
@@ -227,9 +240,9 @@ extern "C" {
 int tq_build_tables(int d, int bits, uint64_t seed, float* centroids_k, float* bounds_k,
                     float* centroids_v, float* bounds_v, int8_t* signs, float* S)
 {
-    if (!supported(d, bits)) return TQ_ERR_UNSUPPORTED;
+    if (!supported(d, bits - 1, bits, 1)) return TQ_ERR_UNSUPPORTED;
     tq::HostTables t;
-    if (!tq::build_host_tables(d, bits, seed, t)) return TQ_ERR_CUDA;
+    if (!tq::build_host_tables(d, bits - 1, bits, 1, seed, t)) return TQ_ERR_CUDA;
     if (centroids_k) std::memcpy(centroids_k, t.centroids_k.data(), t.centroids_k.size() * 4);
     if (bounds_k) std::memcpy(bounds_k, t.bounds_k.data(), t.bounds_k.size() * 4);
     if (centroids_v) std::memcpy(centroids_v, t.centroids_v.data(), t.centroids_v.size() * 4);
@@ -241,14 +254,22 @@ int tq_build_tables(int d, int bits, uint64_t seed, float* centroids_k, float* b
 
 int tq_init(int d, int bits, uint64_t seed, tq_ctx** out)
 {
+    return tq_init_ex(d, bits - 1, bits, 1, seed, out);
+}
+
+int tq_init_ex(int d, int kbits, int vbits, int qjl, uint64_t seed, tq_ctx** out)
+{
     if (!out) return TQ_ERR_INVALID_ARG;
     *out = nullptr;
-    if (!supported(d, bits)) return TQ_ERR_UNSUPPORTED;
+    if (!supported(d, kbits, vbits, qjl)) return TQ_ERR_UNSUPPORTED;
     tq_ctx* ctx = new (std::nothrow) tq_ctx();
     if (!ctx) return TQ_ERR_INVALID_ARG;
     ctx->d = d;
-    ctx->bits = bits;
-    if (!tq::build_host_tables(d, bits, seed, ctx->host)) {
+    ctx->bits = vbits;
+    ctx->kbits = kbits;
+    ctx->vbits = vbits;
+    ctx->qjl = qjl;
+    if (!tq::build_host_tables(d, kbits, vbits, qjl, seed, ctx->host)) {
         delete ctx;
         return TQ_ERR_CUDA;
     }
@@ -284,7 +305,7 @@ void tq_destroy(tq_ctx* ctx)
 int tq_cache_layout(const tq_ctx* ctx, tq_layout* out)
 {
     if (!ctx || !out) return TQ_ERR_INVALID_ARG;
-    *out = make_layout(ctx->d, ctx->bits);
+    *out = ctx_layout(ctx);
     return TQ_OK;
 }
 
@@ -292,7 +313,7 @@ int tq_cache_bytes(const tq_ctx* ctx, int B, int Hkv, int capacity, size_t* byte
 {
     if (!ctx || !bytes || B <= 0 || Hkv <= 0 || capacity <= 0 || capacity % TQ_TILE)
         return TQ_ERR_INVALID_ARG;
-    *bytes = size_t(B) * Hkv * (capacity / TQ_TILE) * size_t(make_layout(ctx->d, ctx->bits).tile_bytes);
+    *bytes = size_t(B) * Hkv * (capacity / TQ_TILE) * size_t(ctx_layout(ctx).tile_bytes);
     return TQ_OK;
 }
 
@@ -349,8 +370,8 @@ int quantize_common(tq_ctx* ctx, const void* k, const void* v, int B, int Hkv, i
     a.Hkv = Hkv;
     a.T = T;
     a.capacity = cache->capacity;
-    a.tile_bytes = make_layout(ctx->d, ctx->bits).tile_bytes;
-    const cudaError_t e = tq::launch_quantize(ctx->d, ctx->bits, ctx->tables, a,
+    a.tile_bytes = ctx_layout(ctx).tile_bytes;
+    const cudaError_t e = tq::launch_quantize(ctx_format(ctx), ctx->tables, a,
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
@@ -363,7 +384,7 @@ int tq_attend_workspace(const tq_ctx* ctx, int B, int Hq, int Hkv, int max_len, 
 {
     if (!ctx || !bytes || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || max_len < 0)
         return TQ_ERR_INVALID_ARG;
-    *bytes = tq::plan_attend(ctx->d, B, Hq, Hkv, max_len, ctx->num_sms).total_bytes;
+    *bytes = tq::plan_attend(ctx_format(ctx), B, Hq, Hkv, max_len, ctx->num_sms).total_bytes;
     return TQ_OK;
 }
 

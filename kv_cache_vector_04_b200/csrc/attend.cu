@@ -1,1021 +1,10 @@
-// tq_attend / tq_scores: split-K flash decoding straight from the packed cache.
-//
-// The logit of query head h against cached token n is the QJL-corrected
-// estimate ("[Benchmark] TurboQuant 實測：KV Cache 3-bit 壓縮，真的零損失？",
-// ai-muninn.com, §"TurboQuant 是什麼：30 秒懶人包": the QJL step makes the
-// attention score unbiased):
-//   l_n = |k_n| (<q~, cK[idx_n]> + rho_n sqrt(pi/2)/m <S q~, 2 s_n - 1>) / sqrt(d),
-// with q~ = Pi q; values stay in the rotated domain and are rotated back once
-// per output: o = Pi^T sum_n softmax(l)_n |v_n| cV[vidx_n].
-//
-// Three kernels:
-//  prologue  q~ = H (D o q) / sqrt(d) and p = S q~ per group of 8 query heads,
-//            written as fp16 m16n8k16 B fragments (hi/lo; log2(e) and the
-//            norms' scales folded in);
-//  split     one CTA per (batch, kv head, group of 8 query heads, context
-//            split); each warp streams 16-token tiles with 128-bit loads of its
-//            own lane string, decodes codes to fp16 tensor-core A fragments
-//            through a lane-replicated shared-memory table (2 ALU ops + 1 LDS
-//            per fp16x2) and sign pairs with 2 ALU ops, and runs
-//              logits: [16 tok x d] x [d x 8 heads]  (codebook term)
-//                      [16 tok x m] x [m x 8 heads]  (QJL sign term)
-//              PV:     [d x 16 tok] x [16 tok x 8 heads]
-//            on mma.sync with fp32 accumulation, with an online softmax per
-//            head in registers; the 8 warps of a CTA merge in shared memory;
-//  reduce    merges the splits per query head and applies Pi^T (fp32 WHT).
-// Operands come from registers because every A fragment is decoded on the
-// fly; the contraction is skinny (N = 8 heads), so the legacy register-fed
-// MMA fits better here than shared-memory/TMEM-fed tcgen05 tiles.
-#include <cuda_runtime.h>
-#include <math_constants.h>
-
-#include "device_common.cuh"
-#include "kernels.h"
+// Host side of the attention launches: the work plan, the dispatch to the
+// per-head-dim launch tables, and the streaming copy kernel that measures HBM
+// bandwidth in the same process.
+#include "attend_impl.cuh"
 
 namespace tq {
 namespace {
-
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
-
-template <int D, int BITS>
-struct AttTraits {
-    static constexpr int BK = BITS - 1, BV = BITS;
-    static constexpr int KF = 2 * BK, VF = 2 * BV;          // field widths
-    static constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;
-    static constexpr int SBW = BK * D / 64;                  // first sign word
-    static constexpr int VB = (BK + 1) * D / 2;              // first value bit
-    static constexpr int KK = D / 16;                        // k-steps / coordinate blocks
-    static constexpr int NLK = 1 << KF, NLV = 1 << VF;       // LUT entries
-    static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
-    // d <= 128: CTAs of 4 warps, 3 per SM, query fragments in registers;
-    // d = 256: CTAs of 8 warps, 1 per SM, query fragments in shared memory
-    static constexpr bool QREG = D <= 128;
-    static constexpr int WARPS = QREG ? 4 : 8, NT = 32 * WARPS, CTAS_PER_SM = QREG ? 3 : 1;
-    static constexpr size_t MERGE_BYTES = (size_t)WARPS * 8 * (D + 2) * 4;
-    // staging ring: per warp STAGES images of whole tiles, each brought in by
-    // one bulk copy
-    static constexpr int STAGES = 3;
-    static constexpr int NCH = BITS * D / 8 / CB;
-    static constexpr int TILE_BYTES = 16 * (BITS * D / 4 + 6);
-    static constexpr int STAGE_BYTES = TILE_BYTES;
-    static constexpr size_t RING_BYTES = (size_t)WARPS * STAGES * STAGE_BYTES;
-    static constexpr size_t QF_SMEM = QREG ? 0 : QF_BYTES;
-    static constexpr size_t LOOP_BYTES = RING_BYTES + QF_SMEM;
-    static constexpr size_t DYN_SMEM = LOOP_BYTES > MERGE_BYTES ? LOOP_BYTES : MERGE_BYTES;
-};
-
-// Offset, inside a lane-replicated table, of the entry selected by the F-bit
-// field at bit `pos` of the lane string: field * 128 + 4 * lane, built with one
-// funnel (or plain) shift and one LOP3 (lane4 = 4 * lane occupies bits 2..6,
-// the field bits 7 and up). The table's own shared address is added by the
-// load as an immediate, so no alignment of the table is assumed: shared
-// memory does not start at address 0 of the window, and declared alignments
-// above 1 KB are not honoured there.
-__device__ __forceinline__ uint32_t lut_off(const uint32_t* s, int pos, int F, uint32_t lane4)
-{
-    const int wi = pos >> 5, o = pos & 31;
-    const uint32_t mask = ((1u << F) - 1u) << 7;
-    uint32_t v;
-    if (o + F <= 32)
-        v = (o >= 7) ? (s[wi] >> (o - 7)) : (s[wi] << (7 - o));
-    else
-        v = __funnelshift_r(s[wi], s[wi + 1], o - 7);
-    return (v & mask) | lane4;
-}
-
-__device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t byte_off)
-{
-    return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(table) + byte_off);
-}
-
-// fp16x2 (+-rho, +-rho) from sign pair p: element 0 at bit p%16, element 1 at
-// bit 16 + p%16 of sign word p/16 (bit 1 = +); nrho2 holds -rho in both halves.
-// The residual norm rho rides on the sign operand, so the QJL products land in
-// the same accumulators as the codebook products.
-__device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q, uint32_t nrho2)
-{
-    const uint32_t x = word << (15 - q);
-    return (x & 0x80008000u) ^ nrho2;
-}
-
-// ---------------------------------------------------------------- prologue
-// Warp 0 of CTA (0, 0) also lays the units' tiles end to end for the split
-// kernel: prefix[b] = sum over sequences b' < b of ceil(seq'/16) x units per
-// sequence (seq clamped to [0, min(max_len, capacity)], flagging a clamp),
-// prefix[B] = the total.
-__device__ __forceinline__ void tile_prefix(const DevTables& tb, const AttendArgs& a, int lane)
-{
-    const int lim = min(a.max_len, a.capacity);
-    const long long upb = (long long)a.Hkv * a.plan.groups;
-    long long run = 0;
-    bool bad = false;
-    for (int b0 = 0; b0 < a.B; b0 += 32) {
-        const int b = b0 + lane;
-        long long v = 0;
-        if (b < a.B) {
-            int s = a.seq_len[b];
-            if (s < 0 || s > lim) {
-                bad = true;
-                s = min(max(s, 0), lim);
-            }
-            v = (long long)((s + 15) >> 4) * upb;
-        }
-        long long incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const long long y = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (b < a.B) a.prefix[b] = run + incl - v;
-        run += __shfl_sync(kFull, incl, 31);
-    }
-    if (lane == 0) a.prefix[a.B] = run;
-    if (__any_sync(kFull, bad) && lane == 0) atomicOr(tb.status, TQ_STATUS_SEQ_LEN);
-}
-
-// One CTA per (batch, kv head, group of 8 query heads): q~ = H (D o q) / sqrt(d)
-// and p = S q~ for the 8 heads (S is read once per CTA), written as the fp16 B
-// fragments of [log2(e) 2^7 q~ / (d alpha)] and [log2(e) 2^7 kappa p / sqrt(d)],
-// each as a hi part and a lo part (x - hi), so that the two tensor-core
-// products carry ~22 significant bits. alpha is the scale that makes the key
-// codebook almost exact in fp16 (chosen on the host).
-template <int D>
-__device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendArgs& a)
-{
-    constexpr int NT = 2 * D;
-    __shared__ float qt[D][8];          // rotated queries, [coordinate][head]
-    __shared__ float pp[1][D][8];       // p = S q~
-    __shared__ float es[8];             // per-head power-of-two scale of q~ for the split
-    const int unit = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-    const int groups = a.plan.groups, ratio = a.Hq / a.Hkv;
-    const int hkv = unit / groups, grp = unit % groups;
-    const size_t units = (size_t)a.Hkv * groups;
-    if (unit == 0 && b == 0 && tid < 32) tile_prefix(tb, a, tid);
-
-    for (int e = tid; e < 8 * D; e += NT) {
-        const int h = e / D, i = e % D, j = grp * 8 + h;
-        float x = 0.f;
-        if (j < ratio) {
-            const size_t off = ((size_t)b * a.Hq + hkv * ratio + j) * D + i;
-            x = a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[off])
-                         : __half2float(reinterpret_cast<const __half*>(a.q)[off]);
-            x *= tb.signs[i];
-        }
-        qt[i][h] = x;
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int st = 1; st < D; st <<= 1) {            // Walsh-Hadamard butterflies, 8 heads
-        for (int e = tid; e < 4 * D; e += NT) {
-            const int h = e & 7, bf = e >> 3;
-            const int i = (bf / st) * 2 * st + (bf % st);
-            const float x0 = qt[i][h], x1 = qt[i + st][h];
-            qt[i][h] = x0 + x1;
-            qt[i + st][h] = x0 - x1;
-        }
-        __syncthreads();
-    }
-    const float rs = rsqrtf((float)D);
-    for (int e = tid; e < 8 * D; e += NT) (&qt[0][0])[e] *= rs;
-    __syncthreads();
-    // per head a power of two es with max |q~| es in [64, 128): the hi and lo
-    // fp16 parts of q~ es below then stay clear of overflow and of subnormals
-    {
-        const int w = tid >> 5, lane = tid & 31;
-        for (int h = w; h < 8; h += NT / 32) {
-            float mx = 0.f;
-            for (int c = lane; c < D; c += 32) mx = fmaxf(mx, fabsf(qt[c][h]));
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-            if (lane == 0) es[h] = (mx > 0.f && mx < 3.0e38f) ? exp2f((float)(6 - ilogbf(mx))) : 1.f;
-        }
-    }
-    __syncthreads();
-    // p^T = q~^T S^T on the tensor cores: A = q~ es (rows = the 8 heads, rows
-    // 8..15 zero) as hi + lo fp16 parts, B = the fp16-exact S^T fragments,
-    // fp32 accumulation; warp w takes n-tiles (8 rows of S each) w, w + NW, ...
-    {
-        const int w = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-        const float sc = es[g];
-        for (int nt = w; nt < D / 8; nt += NT / 32) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const int c0 = 16 * kk + 2 * t;
-                const float x0 = qt[c0][g] * sc, x1 = qt[c0 + 1][g] * sc;
-                const float x2 = qt[c0 + 8][g] * sc, x3 = qt[c0 + 9][g] * sc;
-                const float h0 = __half2float(__float2half_rn(x0)), h1 = __half2float(__float2half_rn(x1));
-                const float h2 = __half2float(__float2half_rn(x2)), h3 = __half2float(__float2half_rn(x3));
-                const uint2 bf = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
-                mma_16816(acc, pack_half2(h0, h1), 0u, pack_half2(h2, h3), 0u, bf.x, bf.y);
-                mma_16816(acc, pack_half2(x0 - h0, x1 - h1), 0u, pack_half2(x2 - h2, x3 - h3), 0u,
-                          bf.x, bf.y);
-            }
-            // acc[0], acc[1]: head g, rows 8 nt + 2t and + 1 of S
-            pp[0][8 * nt + 2 * t][g] = acc[0] / sc;
-            pp[0][8 * nt + 2 * t + 1][g] = acc[1] / sc;
-        }
-    }
-    __syncthreads();
-    {
-        // one fragment entry (k-step, thread-in-group, head column) per thread
-        const int e = tid, col = e & 7, t = (e >> 3) & 3, kk = e >> 5;
-        const int c0 = 16 * kk + 2 * t;
-        const int idx[4] = {c0, c0 + 1, c0 + 8, c0 + 9};
-        const float scale_c = kLog2e * 128.0f / ((float)D * tb.alpha_k);
-        const float scale_s = kLog2e * 128.0f * 1.2533141373155003f / ((float)D * sqrtf((float)D));
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            float hv[4], lv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float x = q ? pp[0][idx[u]][col] * scale_s : qt[idx[u]][col] * scale_c;
-                hv[u] = __half2float(__float2half_rn(x));
-                lv[u] = x - hv[u];
-            }
-            hi[2 * q] = pack_half2(hv[0], hv[1]);
-            hi[2 * q + 1] = pack_half2(hv[2], hv[3]);
-            lo[2 * q] = pack_half2(lv[0], lv[1]);
-            lo[2 * q + 1] = pack_half2(lv[2], lv[3]);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(a.qfrag) +
-                     (((size_t)b * units + unit) * (D / 16) + kk) * 64 + col * 4 + t;
-        dst[0] = make_uint4(hi[0], hi[1], lo[0], lo[1]);    // codebook term: b0,b1 hi; b0,b1 lo
-        dst[32] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
-    }
-}
-
-template <int D>
-__global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArgs a)
-{
-    prologue_body<D>(tb, a);
-}
-
-// ---------------------------------------------------------------- fused append
-// Bit position helpers for one token's codes inside a tile image (the tile
-// layout of tq.h): a lane string is cut into chunks of CB bytes stored
-// chunk-major, so string word sw of lane L sits at tile word
-// ((4 sw / CB) * 32 + L) * CB/4 + (4 sw % CB) / 4.
-template <int CB>
-__device__ __forceinline__ int tile_word(int L, int sw)
-{
-    return (((4 * sw) / CB) * 32 + L) * (CB / 4) + ((4 * sw) % CB) / 4;
-}
-
-// Replace the nb-bit field at string bit `sbit` of lane L's string (a field may
-// straddle two string words). Other tokens' bits in the same words may be
-// written by other warps at the same time, hence the shared-memory atomics.
-template <int CB>
-__device__ __forceinline__ void put_field(uint32_t* img, int L, int sbit, uint32_t val, int nb)
-{
-    const int sw = sbit >> 5, off = sbit & 31;
-    const uint32_t m = (1u << nb) - 1u;
-    uint32_t* w0 = img + tile_word<CB>(L, sw);
-    atomicAnd(w0, ~(m << off));
-    atomicOr(w0, (val & m) << off);
-    if (off + nb > 32) {
-        uint32_t* w1 = img + tile_word<CB>(L, sw + 1);
-        atomicAnd(w1, ~(m >> (32 - off)));
-        atomicOr(w1, (val & m) >> (32 - off));
-    }
-}
-
-// Quantize the T <= 16 new tokens of (sequence b, kv head hkv) exactly as
-// tq_quantize does and write them into the cache: the (at most two) tiles they
-// touch are copied into shared memory; each warp takes one K or V vector at a
-// time (fp64 norm, sign flip, Walsh–Hadamard, cells; for keys the residual and
-// its norm) and sets its bits in the tile images; then thread j computes row j
-// of z = S r for every new key as an fp64 dot product (each S entry is loaded
-// once for all keys) and sets the QJL sign bits s = [z >= 0]; the tiles are
-// written back.
-template <int D, int BITS>
-__device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendArgs& a, int b, int hkv,
-                                              uint8_t* smem)
-{
-    constexpr int NT = 2 * D, NW = NT / 32, VPL = D / 32, M = D;
-    constexpr int BK = BITS - 1, BV = BITS;
-    constexpr int TB = 16 * (BITS * D / 4 + 6);
-    constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;
-    constexpr int SB0 = BK * D / 2, VB0 = (BK + 1) * D / 2;   // first sign / value bit of a string
-    constexpr int NB = 4 * BITS * D;                          // first norm byte of a tile
-    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int T = a.T, start = a.start_pos[b];
-    if (T <= 0) return;
-    if (start < 0 || (long long)start + T > (long long)a.capacity) {
-        if (tid == 0 && hkv == 0) atomicOr(tb.status, TQ_STATUS_CAPACITY);
-        return;
-    }
-    uint32_t* img = reinterpret_cast<uint32_t*>(smem);                      // [2][TB]
-    double* tabs = reinterpret_cast<double*>(smem + 2 * TB);                // ck[16] tk[16] tv[16]
-    double* rk = tabs + 48;                                                  // [16][D] key residuals
-    double* zp = rk + 16 * D;                                                // [16][M] half-sums of z
-    const int t0 = start / 16, ntile = (start + T - 1) / 16 - t0 + 1;
-    uint8_t* stream = a.cache_w + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity / 16) * TB;
-    for (int e = tid; e < ntile * TB / 16; e += NT)
-        reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(stream + (size_t)t0 * TB)[e];
-    if (tid < (1 << BK)) tabs[tid] = tb.centroids_kd[tid];
-    if (tid < (1 << BK) - 1) tabs[16 + tid] = tb.bounds_k[tid];
-    if (tid < (1 << BV) - 1) tabs[32 + tid] = tb.bounds_v[tid];
-    __syncthreads();
-
-    unsigned sat = 0u;
-    const double inv_sqrt_d = 1.0 / sqrt((double)D);
-#pragma unroll 1
-    for (int job = w; job < 2 * T; job += NW) {
-        const bool is_key = job < T;
-        const int i = is_key ? job : job - T;
-        const int n = start + i, tau = n & 15, g = tau & 7, half = tau >> 3;
-        uint32_t* tw = img + (n / 16 - t0) * (TB / 4);
-        const __half* src = (is_key ? a.k_new : a.v_new) +
-                            (((size_t)b * a.Hkv + hkv) * (size_t)T + i) * D + lane * VPL;
-        double x[VPL];
-#pragma unroll
-        for (int k = 0; k < VPL; k += 2) {
-            const __half2 p = *reinterpret_cast<const __half2*>(src + k);
-            x[k] = (double)__low2float(p);
-            x[k + 1] = (double)__high2float(p);
-        }
-        double ss = 0.0;
-#pragma unroll
-        for (int k = 0; k < VPL; ++k) {
-            ss += x[k] * x[k];
-            x[k] *= (double)tb.signs[lane * VPL + k];
-        }
-        ss = warp_sum(ss);
-        wht_warp<VPL>(x, lane);
-        const double nrm = sqrt(ss);
-        const double scale = nrm > 0.0 ? inv_sqrt_d / nrm : 0.0;
-        if (is_key) {
-            double rr = 0.0;
-#pragma unroll
-            for (int k = 0; k < VPL; ++k) {
-                const int c = lane * VPL + k;
-                const double y = x[k] * scale;
-                const int idx = encode_cell<BK>(y, tabs + 16);
-                const double r = y - tabs[idx];
-                rk[i * D + c] = r;
-                rr += r * r;
-                // K field: token g + 8 (r & 1), coordinate 16 kk + 8 (r >> 1) + 2 t + e
-                const int kk = c >> 4, t = (c & 7) >> 1, e = c & 1;
-                const int p = 4 * kk + 2 * ((c & 15) >> 3) + half;
-                put_field<CB>(tw, 4 * g + t, 2 * BK * p + e * BK, (uint32_t)idx, BK);
-            }
-            rr = warp_sum(rr);
-            if (lane == 0) {
-                uint16_t* nk = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(tw) + NB + 8 * g + 4 * half);
-                nk[0] = norm_to_half_bits(nrm, sat);
-                nk[1] = norm_to_half_bits(sqrt(rr), sat);
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < VPL; ++k) {
-                const int c = lane * VPL + k;
-                const int idx = encode_cell<BV>(x[k] * scale, tabs + 32);
-                // V field: token 2 t + 8 (r >> 1) + e, coordinate 16 kk + g' + 8 (r & 1)
-                const int kk = c >> 4, gc = c & 7, t = (tau & 7) >> 1, e = tau & 1;
-                const int p = 4 * kk + 2 * half + ((c & 15) >> 3);
-                put_field<CB>(tw, 4 * gc + t, VB0 + 2 * BV * p + e * BV, (uint32_t)idx, BV);
-            }
-            if (lane == 0)
-                *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(tw) + NB + 64 + 4 * g + 2 * half) =
-                    norm_to_half_bits(nrm, sat);
-        }
-    }
-    __syncthreads();
-    // QJL signs: threads j and M + j own row j of z = S r for all new keys, each
-    // summing half of the coordinates (NT = 2M); the loads of S are independent,
-    // so many are in flight at once
-    {
-        const int j = tid % M, hf = tid / M;
-        double z[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0.0;
-#pragma unroll 16
-        for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); ++c) {
-            const double sv = (double)__ldg(tb.s_t + (size_t)c * M + j);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < T) z[i] = fma(sv, rk[i * D + c], z[i]);
-        }
-        if (hf == 1) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < T) zp[i * M + j] = z[i];
-        }
-        __syncthreads();
-        if (hf == 0) {
-            const int kk = j >> 4, t = (j & 7) >> 1, e = j & 1;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                if (i >= T) break;
-                const int n = start + i, tau = n & 15;
-                const int p = 4 * kk + 2 * ((j & 15) >> 3) + (tau >> 3);
-                put_field<CB>(img + (n / 16 - t0) * (TB / 4), 4 * (tau & 7) + t,
-                              SB0 + 32 * (p >> 4) + 16 * e + (p & 15),
-                              z[i] + zp[i * M + j] >= 0.0 ? 1u : 0u, 1);
-            }
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < ntile * TB / 16; e += NT)
-        reinterpret_cast<uint4*>(stream + (size_t)t0 * TB)[e] = reinterpret_cast<const uint4*>(img)[e];
-    if (sat) atomicOr(tb.status, TQ_STATUS_NORM_SAT);
-}
-
-// Prologue launch of a decode step with new tokens: CTAs (x < units, b) run
-// the query prologue, CTAs (units + h, b) append the new tokens of (b, kv head
-// h), side by side; the split kernel, launched after this one, reads them.
-template <int D, int BITS>
-__global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArgs a)
-{
-    extern __shared__ uint4 app_smem[];
-    const int units = a.Hkv * a.plan.groups;
-    if ((int)blockIdx.x >= units)
-        append_tokens<D, BITS>(tb, a, blockIdx.y, blockIdx.x - units, reinterpret_cast<uint8_t*>(app_smem));
-    else
-        prologue_body<D>(tb, a);
-}
-
-
-// ---------------------------------------------------------------- reduction
-// One CTA per (query head, batch): merges the partials of the CTAs whose
-// ranges cover the head's unit (the range of CTA c is [c W / G, (c+1) W / G)
-// of the W tiles, so tile x lies in CTA ((x + 1) G - 1) / W), then applies
-// Pi^T with an fp32 Walsh-Hadamard transform.
-template <int D>
-__global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
-{
-    __shared__ float os[D];
-    const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
-    const int ratio = a.Hq / a.Hkv, groups = a.plan.groups;
-    const int hkv = hq / ratio, jh = hq % ratio, grp = jh >> 3, col = jh & 7;
-    const int upb = a.Hkv * groups, ju = hkv * groups + grp;
-    const size_t u = (size_t)b * upb + ju;
-    constexpr int RS = D + 2;
-    const long long W = a.prefix[a.B], pb = a.prefix[b];
-    const long long T = (a.prefix[b + 1] - pb) / upb;
-    const long long G = a.plan.ctas;
-    float M = -CUDART_INF_F, L = 0.f, acc = 0.f;
-    if (T > 0) {
-        const long long U0 = pb + ju * T, U1 = U0 + T;
-        const int cf = (int)(((U0 + 1) * G - 1) / W), cl = (int)((U1 * G - 1) / W);
-        for (int c = cf; c <= cl; ++c) {
-            if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;   // empty range
-            M = fmaxf(M, a.partial[((size_t)c + u) * 8 * RS + col * RS]);
-        }
-        if (M != -CUDART_INF_F) {
-            for (int c = cf; c <= cl; ++c) {
-                if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;
-                const float* ps = a.partial + ((size_t)c + u) * 8 * RS + col * RS;
-                const float ms = ps[0];
-                if (ms == -CUDART_INF_F) continue;
-                const float f = exp2f(ms - M);
-                L = fmaf(ps[1], f, L);
-                acc = fmaf(ps[2 + i], f, acc);
-            }
-        }
-    }
-    os[i] = (L > 0.f) ? acc / L : 0.f;
-    __syncthreads();
-#pragma unroll
-    for (int s = 1; s < D; s <<= 1) {
-        const float mine = os[i], other = os[i ^ s];
-        __syncthreads();
-        os[i] = (i & s) ? (other - mine) : (mine + other);
-        __syncthreads();
-    }
-    // Pi^T = D H / sqrt(d), and the value table carries a factor sqrt(d)
-    a.out[((size_t)b * a.Hq + hq) * D + i] = os[i] * tb.signs[i] * (1.0f / (float)D);
-}
-
-// ---------------------------------------------------------------- split kernel
-// mbarrier + bulk-copy helpers (shared addresses are 32-bit).
-constexpr int kWaitLimit = 1 << 22;   // bounded waits: give up and flag TQ_STATUS_WAIT_TIMEOUT
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init()
-{
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-}
-// Orders this thread's earlier generic-proxy accesses of shared memory before
-// later async-proxy (bulk copy) writes to it.
-__device__ __forceinline__ void fence_proxy_async()
-{
-    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-}
-// One bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
-// from global memory into this CTA's shared memory, completing on `bar`,
-// whose expected transaction count is raised by the same amount.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
-                 : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-// Wait for phase `parity` of `bar` to complete; false after kWaitLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
-{
-    for (int i = 0; i < kWaitLimit; ++i) {
-        uint32_t ok;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-            " selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok) return true;
-    }
-    return false;
-}
-
-template <int D, int BITS>
-struct TileData {
-    uint32_t s[BITS * D / 32];   // this lane's string of the tile
-    uint2 kn;                    // fp16 {|k_g|, rho_g, |k_g+8|, rho_g+8}
-    uint32_t vn;                 // fp16 {|v_g|, |v_g+8|}
-};
-
-template <int D, int BITS>
-__device__ __forceinline__ void load_tile(const uint8_t* tp, int lane, int g, TileData<D, BITS>& td)
-{
-    using Tr = AttTraits<D, BITS>;
-    constexpr int CB = Tr::CB, NCH = BITS * D / 8 / CB;
-#pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        const uint8_t* src = tp + ((size_t)c * 32 + lane) * CB;
-        if constexpr (CB == 16) {
-            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src));
-            td.s[4 * c] = v.x; td.s[4 * c + 1] = v.y; td.s[4 * c + 2] = v.z; td.s[4 * c + 3] = v.w;
-        } else {
-            const uint2 v = __ldcs(reinterpret_cast<const uint2*>(src));
-            td.s[2 * c] = v.x; td.s[2 * c + 1] = v.y;
-        }
-    }
-    td.kn = __ldcs(reinterpret_cast<const uint2*>(tp + 4 * BITS * D + 8 * g));
-    td.vn = __ldcs(reinterpret_cast<const uint32_t*>(tp + 4 * BITS * D + 64 + 4 * g));
-}
-
-// Read this lane's bytes of a tile image in shared memory (the image has the
-// cache's own layout: chunk-major lane strings, then K norms, then V norms).
-template <int D, int BITS>
-__device__ __forceinline__ void read_stage(const uint8_t* slot, int lane, TileData<D, BITS>& td)
-{
-    using Tr = AttTraits<D, BITS>;
-#pragma unroll
-    for (int c = 0; c < Tr::NCH; ++c) {
-        const uint8_t* src = slot + (c * 32 + lane) * Tr::CB;
-        if constexpr (Tr::CB == 16) {
-            const uint4 v = *reinterpret_cast<const uint4*>(src);
-            td.s[4 * c] = v.x; td.s[4 * c + 1] = v.y; td.s[4 * c + 2] = v.z; td.s[4 * c + 3] = v.w;
-        } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(src);
-            td.s[2 * c] = v.x; td.s[2 * c + 1] = v.y;
-        }
-    }
-    constexpr int nb = 4 * BITS * D;
-    const int g = lane >> 2;
-    td.kn = *reinterpret_cast<const uint2*>(slot + nb + 8 * g);
-    td.vn = *reinterpret_cast<const uint32_t*>(slot + nb + 64 + 4 * g);
-}
-
-// Query B fragments of one k-step: x,y = hi (b0, b1), z,w = lo, for the
-// codebook term (c) and the QJL term (s). Held in registers (they do not
-// change from tile to tile) or, where registers are short, in shared memory.
-template <int KK, int NT, bool IN_REGS>
-struct QueryFrags;
-
-template <int KK, int NT>
-struct QueryFrags<KK, NT, true> {
-    uint4 c[KK], s[KK];
-    __device__ __forceinline__ void load(const uint4* src, uint4*, int tid)
-    {
-        const int lane = tid & 31;
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-            c[kk] = src[kk * 64 + lane];
-            s[kk] = src[kk * 64 + 32 + lane];
-        }
-    }
-    __device__ __forceinline__ uint4 fc(int kk, int) const { return c[kk]; }
-    __device__ __forceinline__ uint4 fs(int kk, int) const { return s[kk]; }
-};
-
-template <int KK, int NT>
-struct QueryFrags<KK, NT, false> {
-    const uint4* sm;
-    __device__ __forceinline__ void load(const uint4* src, uint4* smem, int tid)
-    {
-        for (int e = tid; e < KK * 64; e += NT) smem[e] = src[e];
-        sm = smem;
-    }
-    __device__ __forceinline__ uint4 fc(int kk, int lane) const { return sm[kk * 64 + lane]; }
-    __device__ __forceinline__ uint4 fs(int kk, int lane) const { return sm[kk * 64 + 32 + lane]; }
-};
-
-template <int D>
-struct SplitState {
-    float m0, m1, l0, l1;
-    float acc[D / 16][4];
-};
-
-// Logits of one tile (log2 units) for tokens g, g+8 and heads 2t, 2t+1.
-template <int D, int BITS, typename QF>
-__device__ __forceinline__ void tile_logits(const TileData<D, BITS>& td, const QF& qf, int lane,
-                                            const uint32_t* lutk, uint32_t lane4, float (&L)[4])
-{
-    using Tr = AttTraits<D, BITS>;
-    // -rho of tokens g and g+8 in both fp16 halves (A rows g and g+8)
-    const uint32_t nr_g = __byte_perm(td.kn.x, 0u, 0x3232) | 0x80008000u;
-    const uint32_t nr_h = __byte_perm(td.kn.y, 0u, 0x3232) | 0x80008000u;
-    // two accumulation chains: hi and lo parts of the B operands; each takes
-    // the codebook product and the rho-weighted QJL product of every k-step
-    float ah[4], al[4];
-#pragma unroll
-    for (int kk = 0; kk < Tr::KK; ++kk) {
-        const uint4 bc = qf.fc(kk, lane);
-        const uint4 bs = qf.fs(kk, lane);
-        uint32_t ak[4], as[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int p = 4 * kk + r;
-            ak[r] = lut_load(lutk, lut_off(td.s, Tr::KF * p, Tr::KF, lane4));
-            as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
-        }
-        if (kk == 0) {
-            mma_16816_first(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
-            mma_16816_first(al, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
-        } else {
-            mma_16816(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
-            mma_16816(al, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
-        }
-        mma_16816(ah, as[0], as[1], as[2], as[3], bs.x, bs.y);
-        mma_16816(al, as[0], as[1], as[2], as[3], bs.z, bs.w);
-    }
-    // |k| of tokens g and g+8 (fp16, low halves); the B operands carry 2^7
-    const float kn_g = __low2float(*reinterpret_cast<const __half2*>(&td.kn.x)) * (1.0f / 128.0f);
-    const float kn_h = __low2float(*reinterpret_cast<const __half2*>(&td.kn.y)) * (1.0f / 128.0f);
-    L[0] = kn_g * (ah[0] + al[0]);
-    L[1] = kn_g * (ah[1] + al[1]);
-    L[2] = kn_h * (ah[2] + al[2]);
-    L[3] = kn_h * (ah[3] + al[3]);
-}
-
-// Online-softmax update and P V for one tile.
-template <int D, int BITS>
-__device__ __forceinline__ void tile_accumulate(const TileData<D, BITS>& td, float (&L)[4], bool v0,
-                                                bool v1, const uint32_t* lutv, uint32_t lane4,
-                                                SplitState<D>& st)
-{
-    using Tr = AttTraits<D, BITS>;
-    // The running max only moves when some logit exceeds it (rarely, after the
-    // first tiles): only then reduce across the 8 token lanes and rescale.
-    // Otherwise every p = exp2(L - m) <= 1, which also keeps p*|v| in fp16 range.
-    const bool above = (L[0] > st.m0) || (L[2] > st.m0) || (L[1] > st.m1) || (L[3] > st.m1);
-    if (__any_sync(kFull, above)) {
-        float mx0 = fmaxf(L[0], L[2]), mx1 = fmaxf(L[1], L[3]);
-#pragma unroll
-        for (int sh = 4; sh <= 16; sh <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
-        }
-        const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
-        const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
-        st.l0 *= al0;
-        st.l1 *= al1;
-#pragma unroll
-        for (int kk = 0; kk < Tr::KK; ++kk) {
-            st.acc[kk][0] *= al0;
-            st.acc[kk][1] *= al1;
-            st.acc[kk][2] *= al0;
-            st.acc[kk][3] *= al1;
-        }
-        st.m0 = mn0;
-        st.m1 = mn1;
-    }
-    const float p0 = fast_exp2(L[0] - st.m0), p1 = fast_exp2(L[1] - st.m1);
-    const float p2 = fast_exp2(L[2] - st.m0), p3 = fast_exp2(L[3] - st.m1);
-    st.l0 += p0 + p2;
-    st.l1 += p1 + p3;
-    // slots past seq_len may hold anything (even NaN norms): select, never multiply
-    const float2 vnf = __half22float2(*reinterpret_cast<const __half2*>(&td.vn));
-    const float vn_g = v0 ? vnf.x : 0.f;
-    const float vn_h = v1 ? vnf.y : 0.f;
-    const uint32_t b0 = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
-    const uint32_t b1 = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
-#pragma unroll
-    for (int kk = 0; kk < Tr::KK; ++kk) {
-        uint32_t av[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-            av[r] = lut_load(lutv, lut_off(td.s, Tr::VB + Tr::VF * (4 * kk + r), Tr::VF, lane4));
-        mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0, b1);
-    }
-}
-
-// Fill the lane-replicated decode tables of a CTA of NT threads.
-template <int D, int BITS, int NT>
-__device__ __forceinline__ void fill_luts(const DevTables& tb, uint32_t* lutk, uint32_t* lutv, int tid)
-{
-    using Tr = AttTraits<D, BITS>;
-    for (int e = tid; e < Tr::NLK * 32; e += NT) lutk[e] = __ldg(tb.lut_k + (e >> 5));
-    for (int e = tid; e < Tr::NLV * 32; e += NT) lutv[e] = __ldg(tb.lut_v + (e >> 5));
-}
-
-// Estimated logits alone: one CTA per (batch, kv head, group of 8 query heads,
-// context split), every tile up to max_len, -inf past seq_len.
-template <int D, int BITS>
-__global__ void __launch_bounds__(AttTraits<D, BITS>::NT, AttTraits<D, BITS>::CTAS_PER_SM)
-    attend_scores(DevTables tb, AttendArgs a)
-{
-    using Tr = AttTraits<D, BITS>;
-    constexpr int KK = Tr::KK, WARPS = Tr::WARPS, NT = Tr::NT;
-    __shared__ __align__(16) uint32_t lutv[Tr::NLV * 32];
-    __shared__ __align__(16) uint32_t lutk[Tr::NLK * 32];
-    extern __shared__ uint4 dyn_smem[];
-
-    const int split = blockIdx.x, unit = blockIdx.y, b = blockIdx.z;
-    const int groups = a.plan.groups;
-    const int hkv = unit / groups, grp = unit % groups;
-    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const size_t units = (size_t)a.Hkv * groups;
-
-    fill_luts<D, BITS, NT>(tb, lutk, lutv, tid);
-    QueryFrags<KK, NT, Tr::QREG> qf;
-    qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64,
-            reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dyn_smem) + Tr::RING_BYTES), tid);
-    const int seq = min(max(a.seq_len[b], 0), min(a.max_len, a.capacity));
-    __syncthreads();
-
-    const int t_begin = split * a.plan.tps;
-    const int t_end = min(t_begin + a.plan.tps, a.plan.tiles);
-    const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
-                                         (size_t)a.tile_bytes;
-    const uint32_t lane4 = 4u * lane;
-    const int ratio = a.Hq / a.Hkv;
-    const int j0 = grp * 8 + 2 * t;
-    TileData<D, BITS> td;
-#pragma unroll 1
-    for (int tl = t_begin + w; tl < t_end; tl += WARPS) {
-        const int pos0 = tl * 16 + g, pos1 = pos0 + 8;
-        float L[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-        if (tl * 16 < seq) {   // warp-uniform
-            load_tile<D, BITS>(sbase + (size_t)tl * (size_t)a.tile_bytes, lane, g, td);
-            tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
-            if (pos0 >= seq) L[0] = L[1] = -CUDART_INF_F;
-            if (pos1 >= seq) L[2] = L[3] = -CUDART_INF_F;
-        }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            if (j0 + hh >= ratio) continue;
-            float* row = a.out + ((size_t)b * a.Hq + hkv * ratio + j0 + hh) * a.max_len;
-            if (pos0 < a.max_len) row[pos0] = L[hh] * kLn2;
-            if (pos1 < a.max_len) row[pos1] = L[2 + hh] * kLn2;
-        }
-    }
-}
-
-// Split kernel, stream-K: the tiles of all (sequence, kv head, group of 8
-// query heads) units, laid end to end (sequence b's units start at
-// prefix[b]), are cut into gridDim.x equal contiguous ranges, one per CTA, so
-// that one wave of CTAs does equal work whatever the lengths. A CTA walks its
-// range unit by unit; for each piece (segment) its 8 warps stream the tiles
-// round-robin through a per-warp cp.async ring, merge in shared memory and
-// write one partial (m, l, acc per head) to slot CTA + unit, a slot no other
-// segment uses: along the tile order both the CTA index and the unit index
-// are non-decreasing and every new segment raises at least one of them.
-template <int D, int BITS>
-__global__ void __launch_bounds__(AttTraits<D, BITS>::NT, AttTraits<D, BITS>::CTAS_PER_SM)
-    attend_split(DevTables tb, AttendArgs a)
-{
-    using Tr = AttTraits<D, BITS>;
-    constexpr int KK = Tr::KK, WARPS = Tr::WARPS, NT = Tr::NT, S = Tr::STAGES;
-    constexpr int RS = D + 2;
-    // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l, so
-    // the 32 lanes of a warp always hit 32 different banks.
-    __shared__ __align__(16) uint32_t lutv[Tr::NLV * 32];
-    __shared__ __align__(16) uint32_t lutk[Tr::NLK * 32];
-    __shared__ __align__(8) uint64_t bars[WARPS * S];   // one mbarrier per ring slot
-    extern __shared__ uint4 dyn_smem[];
-    float* mrg = reinterpret_cast<float*>(dyn_smem);       // [WARPS][8][D+2] after a segment
-    uint4* qsm = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(dyn_smem) + Tr::RING_BYTES);
-
-    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int c = blockIdx.x;
-    const long long G = gridDim.x;
-    const int groups = a.plan.groups, upb = a.Hkv * groups;
-    const long long W = a.prefix[a.B];
-    const long long x0 = (long long)c * W / G, x1 = (long long)(c + 1) * W / G;
-    if (x0 >= x1) return;   // an empty range (fewer tiles than CTAs): uniform, before any barrier
-
-    fill_luts<D, BITS, NT>(tb, lutk, lutv, tid);
-    const int lim = min(a.max_len, a.capacity);
-    const uint32_t lane4 = 4u * lane;
-    uint8_t* ring = reinterpret_cast<uint8_t*>(dyn_smem) + (size_t)w * S * Tr::STAGE_BYTES;
-    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
-    const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(bars + w * S);
-    if (lane == 0) {
-        for (int i = 0; i < S; ++i) mbar_init(bar_s + 8 * i, 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-    // Bulk copies this warp has issued / waited for (warp-uniform): copy n uses
-    // ring slot n % S and completes phase (n / S) & 1 of that slot's barrier.
-    uint32_t issued = 0, consumed = 0;
-    bool stalled = false;   // a wait ran out: no further copies, tiles skipped
-    QueryFrags<KK, NT, Tr::QREG> qf;
-
-    // Each segment re-locates its unit from x, so that only x, x1 and the
-    // partial slot stay live across the tile loop.
-    long long x = x0;
-#pragma unroll 1
-    while (x < x1) {
-        // the sequence holding tile x: the largest b with prefix[b] <= x (it has tiles)
-        int b = 0;
-        {
-            int hi = a.B - 1;
-            while (b < hi) {
-                const int mid = (b + hi + 1) >> 1;
-                if (a.prefix[mid] <= x) b = mid; else hi = mid - 1;
-            }
-        }
-        const long long pb = a.prefix[b];
-        const long long T = (a.prefix[b + 1] - pb) / upb;   // tiles per unit of sequence b
-        const int j = (int)((x - pb) / T);
-        const long long U0 = pb + (long long)j * T;
-        const int sb = (int)(x - U0);
-        const int se = (int)min(T, x1 - U0);
-        const int seq = min(max(a.seq_len[b], 0), lim);
-        const int hkv = j / groups;
-        const size_t u = (size_t)b * upb + j;
-        qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
-        __syncthreads();   // tables (first segment) and query fragments visible
-
-        const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
-                                             (size_t)a.tile_bytes;
-        SplitState<D> st;
-        st.m0 = st.m1 = -CUDART_INF_F;
-        st.l0 = st.l1 = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
-
-        // Bulk-copy pipeline: S - 1 tiles of this warp are in flight while one
-        // is decoded. Lane 0 issues each copy into the slot the warp finished
-        // reading one iteration earlier (its values are already used).
-        const int my_first = sb + w;
-        fence_proxy_async();
-        if (!stalled && lane == 0) {
-#pragma unroll
-            for (int i = 0; i < S - 1; ++i) {
-                const int tl = my_first + WARPS * i;
-                if (tl < se) {
-                    const uint32_t sl = (issued + i) % S;
-                    bulk_load(ring_s + sl * Tr::STAGE_BYTES, sbase + (size_t)tl * Tr::TILE_BYTES,
-                              Tr::TILE_BYTES, bar_s + 8 * sl);
-                }
-            }
-        }
-        if (!stalled) {
-#pragma unroll
-            for (int i = 0; i < S - 1; ++i) issued += (my_first + WARPS * i < se) ? 1u : 0u;
-        }
-        TileData<D, BITS> td;
-#pragma unroll 1
-        for (int tl = my_first; tl < se && !stalled; tl += WARPS) {
-            const int tn = tl + WARPS * (S - 1);
-            if (tn < se) {
-                fence_proxy_async();
-                if (lane == 0) {
-                    const uint32_t sl = issued % S;
-                    bulk_load(ring_s + sl * Tr::STAGE_BYTES, sbase + (size_t)tn * Tr::TILE_BYTES,
-                              Tr::TILE_BYTES, bar_s + 8 * sl);
-                }
-                ++issued;
-            }
-            const uint32_t slot = consumed % S;
-            if (!mbar_wait(bar_s + 8 * slot, (consumed / S) & 1u)) {
-                stalled = true;
-                if (lane == 0) atomicOr(tb.status, TQ_STATUS_WAIT_TIMEOUT);
-                break;
-            }
-            ++consumed;
-            read_stage<D, BITS>(ring + slot * Tr::STAGE_BYTES, lane, td);
-            float L[4];
-            tile_logits<D, BITS>(td, qf, lane, lutk, lane4, L);
-            const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
-            if (!v0) L[0] = L[1] = -CUDART_INF_F;
-            if (!v1) L[2] = L[3] = -CUDART_INF_F;
-            tile_accumulate<D, BITS>(td, L, v0, v1, lutv, lane4, st);
-        }
-
-        float l0 = st.l0, l1 = st.l1;
-#pragma unroll
-        for (int sh = 4; sh <= 16; sh <<= 1) {
-            l0 += __shfl_xor_sync(kFull, l0, sh);
-            l1 += __shfl_xor_sync(kFull, l1, sh);
-        }
-        fence_proxy_async();
-        __syncthreads();   // every warp is done with the ring: reuse it for the merge
-        float* mw = mrg + (size_t)w * 8 * RS;
-        if (g == 0) {
-            mw[(2 * t) * RS] = st.m0;
-            mw[(2 * t) * RS + 1] = l0;
-            mw[(2 * t + 1) * RS] = st.m1;
-            mw[(2 * t + 1) * RS + 1] = l1;
-        }
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-            mw[(2 * t) * RS + 2 + 16 * kk + g] = st.acc[kk][0];
-            mw[(2 * t + 1) * RS + 2 + 16 * kk + g] = st.acc[kk][1];
-            mw[(2 * t) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][2];
-            mw[(2 * t + 1) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][3];
-        }
-        __syncthreads();
-        float* dst = a.partial + ((size_t)c + u) * 8 * RS;
-        for (int e = tid; e < 8 * RS; e += NT) {
-            const int head = e / RS, col = e % RS;
-            float M = -CUDART_INF_F;
-#pragma unroll
-            for (int ww = 0; ww < WARPS; ++ww) M = fmaxf(M, mrg[(ww * 8 + head) * RS]);
-            float sum = 0.f;
-            if (col == 0) {
-                sum = M;
-            } else {
-#pragma unroll
-                for (int ww = 0; ww < WARPS; ++ww) {
-                    const float mwv = mrg[(ww * 8 + head) * RS];
-                    if (mwv != -CUDART_INF_F) sum += mrg[(ww * 8 + head) * RS + col] * exp2f(mwv - M);
-                }
-            }
-            dst[e] = sum;
-        }
-        __syncthreads();   // merge buffer and query fragments free for the next segment
-        x = U0 + se;       // the next unit (or the end of the range)
-    }
-    // after a wait ran out: wait (bounded) for this warp's copies still in flight
-    while (consumed < issued) {
-        if (!mbar_wait(bar_s + 8 * (consumed % S), (consumed / S) & 1u)) break;
-        ++consumed;
-    }
-}
-
-// cudaFuncSetAttribute once per (kernel, device).
-template <typename K>
-cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long& done_mask)
-{
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (__atomic_load_n(&done_mask, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) __atomic_fetch_or(&done_mask, bit, __ATOMIC_ACQ_REL);
-    return e;
-}
-
-template <int D, int BITS>
-cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool scores, cudaStream_t st)
-{
-    using Tr = AttTraits<D, BITS>;
-    static unsigned long long done_scores = 0, done_attend = 0;
-    if (a.tile_bytes != Tr::TILE_BYTES) return cudaErrorInvalidValue;   // the bulk copies' size
-    const int units = a.Hkv * a.plan.groups;
-    cudaError_t e;
-    if (a.k_new != nullptr && a.T > 0) {
-        static unsigned long long done_append = 0;
-        constexpr int TB = 16 * (BITS * D / 4 + 6);
-        const size_t smem = 2 * (size_t)TB + 8 * (48 + (size_t)16 * D + (size_t)16 * D);
-        auto kern = append_prologue<D, BITS>;
-        if ((e = allow_smem(kern, smem, done_append)) != cudaSuccess) return e;
-        kern<<<dim3(units + a.Hkv, a.B), 2 * D, smem, st>>>(tb, a);
-    } else {
-        attend_prologue<D><<<dim3(units, a.B), 2 * D, 0, st>>>(tb, a);
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (scores) {
-        auto kern = attend_scores<D, BITS>;
-        if ((e = allow_smem(kern, Tr::DYN_SMEM, done_scores)) != cudaSuccess) return e;
-        if (a.plan.tiles > 0)
-            kern<<<dim3(a.plan.nsplit, units, a.B), Tr::NT, Tr::DYN_SMEM, st>>>(tb, a);
-        return cudaGetLastError();
-    }
-    auto kern = attend_split<D, BITS>;
-    if ((e = allow_smem(kern, Tr::DYN_SMEM, done_attend)) != cudaSuccess) return e;
-    if (a.plan.tiles > 0) kern<<<a.plan.ctas, Tr::NT, Tr::DYN_SMEM, st>>>(tb, a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    attend_reduce<D><<<dim3(a.Hq, a.B), D, 0, st>>>(tb, a);
-    return cudaGetLastError();
-}
 
 __global__ void copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n)
 {
@@ -1026,15 +15,25 @@ __global__ void copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ d
 
 }  // namespace
 
-AttendPlan plan_attend(int d, int B, int Hq, int Hkv, int max_len, int num_sms)
+int attend_ctas_per_sm(const Format& f)
 {
+#define TQ_C(DD, KB, VB, QJ) \
+    if (f.d == DD && f.kb == KB && f.vb == VB && f.qjl == QJ) return AttTraits<DD, KB, VB, QJ>::CTAS_PER_SM;
+    TQ_FORMATS(TQ_C)
+#undef TQ_C
+    return 1;
+}
+
+AttendPlan plan_attend(const Format& f, int B, int Hq, int Hkv, int max_len, int num_sms)
+{
+    const int d = f.d;
     AttendPlan p{};
     const int ratio = Hq / Hkv;
     p.groups = (ratio + 7) / 8;
     const long long units = (long long)B * Hkv * p.groups;
     p.tiles = (max_len + 15) / 16;
     // tq_scores: one CTA per (unit, context split), about two waves
-    const long long per_sm = d <= 128 ? AttTraits<128, 4>::CTAS_PER_SM : AttTraits<256, 4>::CTAS_PER_SM;
+    const long long per_sm = attend_ctas_per_sm(f);
     const long long target = 2 * per_sm * num_sms;
     long long ns = (target + units - 1) / units;
     const long long max_ns = (p.tiles + 15) / 16;      // at least 16 tiles (2 per warp) per split
@@ -1056,16 +55,15 @@ AttendPlan plan_attend(int d, int B, int Hq, int Hkv, int max_len, int num_sms)
     return p;
 }
 
-cudaError_t launch_attend(int d, int bits, const DevTables& tb, const AttendArgs& a, bool scores,
+cudaError_t launch_attend(const Format& f, const DevTables& tb, const AttendArgs& a, bool scores,
                           cudaStream_t st)
 {
-#define TQ_A(DD, BB) \
-    if (d == DD && bits == BB) return launch_attend_t<DD, BB>(tb, a, scores, st);
-    TQ_A(64, 2) TQ_A(64, 3) TQ_A(64, 4)
-    TQ_A(128, 2) TQ_A(128, 3) TQ_A(128, 4)
-    TQ_A(256, 2) TQ_A(256, 3) TQ_A(256, 4)
-#undef TQ_A
-    return cudaErrorInvalidValue;
+    switch (f.d) {
+    case 64: return launch_attend_d64(f, tb, a, scores, st);
+    case 128: return launch_attend_d128(f, tb, a, scores, st);
+    case 256: return launch_attend_d256(f, tb, a, scores, st);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st)

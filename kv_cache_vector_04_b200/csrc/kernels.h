@@ -8,6 +8,11 @@ namespace tq {
 
 struct DevTables;
 
+// A cache format: head dim, key cell bits, value cell bits, QJL sketch on keys.
+struct Format {
+    int d, kb, vb, qjl;
+};
+
 struct QuantizeArgs {
     const __half* k;          // [B][Hkv][T][d]
     const __half* v;          // [B][Hkv][T][d]
@@ -47,12 +52,25 @@ struct AttendArgs {
     uint8_t* cache_w;         // the cache, writable
 };
 
-cudaError_t launch_quantize(int d, int bits, const DevTables& tb, const QuantizeArgs& a,
+cudaError_t launch_quantize(const Format& f, const DevTables& tb, const QuantizeArgs& a,
                             cudaStream_t st);
-cudaError_t launch_attend(int d, int bits, const DevTables& tb, const AttendArgs& a,
+cudaError_t launch_attend(const Format& f, const DevTables& tb, const AttendArgs& a,
                           bool scores, cudaStream_t st);
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t st);
+cudaError_t launch_attend_d64(const Format& f, const DevTables& tb, const AttendArgs& a, bool scores,
+                             cudaStream_t st);
+cudaError_t launch_attend_d128(const Format& f, const DevTables& tb, const AttendArgs& a, bool scores,
+                              cudaStream_t st);
+cudaError_t launch_attend_d256(const Format& f, const DevTables& tb, const AttendArgs& a, bool scores,
+                              cudaStream_t st);
 
-AttendPlan plan_attend(int d, int B, int Hq, int Hkv, int max_len, int num_sms);
+AttendPlan plan_attend(const Format& f, int B, int Hq, int Hkv, int max_len, int num_sms);
+// Split CTAs resident per SM for a format (its shared memory and registers).
+int attend_ctas_per_sm(const Format& f);
+
+// Every built format, for the launch tables: X(D, KB, VB, QJL).
+#define TQ_FORMATS_D(X, D) \
+    X(D, 1, 2, 1) X(D, 2, 3, 1) X(D, 3, 4, 1) X(D, 2, 2, 0) X(D, 3, 3, 0) X(D, 4, 4, 0) X(D, 3, 4, 0)
+#define TQ_FORMATS(X) TQ_FORMATS_D(X, 64) TQ_FORMATS_D(X, 128) TQ_FORMATS_D(X, 256)
 
 }  // namespace tq

@@ -28,16 +28,22 @@
 namespace tq {
 namespace {
 
-template <int D, int BITS>
+// Format (KB, VB, QJ): key cells of KB bits, value cells of VB bits, QJL
+// sketch of the key residual (and rho) iff QJ = 1.
+template <int D, int KB, int VB, int QJ>
 struct QuantTraits {
-    static constexpr int BK = BITS - 1, BV = BITS, M = D;
+    static constexpr int BK = KB, BV = VB, M = D;
+    static constexpr int W = KB + QJ + VB;             // lane-string bits per pair slot
     static constexpr int VPL = D / 32;                 // coordinates per lane per vector
-    static constexpr int CB = ((BITS * D / 8) % 16 == 0) ? 16 : 8;  // chunk bytes
-    static constexpr int NCH = BITS * D / 8 / CB;      // chunks per lane string
+    static constexpr int SBYTES = W * D / 16;          // bytes of a lane string
+    static constexpr int CB = SBYTES % 16 == 0 ? 16 : SBYTES % 8 == 0 ? 8 : 4;  // chunk bytes
+    static constexpr int NCH = SBYTES / CB;            // chunks per lane string
     static constexpr int CW = CB / 4;                  // words per chunk
     static constexpr int KF = 2 * BK, VF = 2 * BV;     // field widths (two codes each)
     static constexpr int SBW = BK * D / 64;            // first sign word of a lane string
-    static constexpr int VBW = (BK + 1) * D / 64;      // first value word
+    static constexpr int VBW = (BK + QJ) * D / 64;     // first value word
+    static constexpr int CODE_BYTES = 2 * W * D;       // code region of a tile
+    static constexpr int KNB = 32 + 32 * QJ;           // K norm bytes of a tile
     static constexpr int NT = M / 8;                   // n-tiles of z = S r
     static constexpr int NTW = NT / 4;                 // n-tiles per warp
 };
@@ -63,10 +69,10 @@ struct QuantSmem {
     uint16_t nk[16], nr[16], nv[16];  // fp16 norms
 };
 
-template <int D, int BITS>
+template <int D, int KB, int VB, int QJ>
 __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArgs a)
 {
-    using Tr = QuantTraits<D, BITS>;
+    using Tr = QuantTraits<D, KB, VB, QJ>;
     constexpr int BK = Tr::BK, BV = Tr::BV, M = Tr::M, VPL = Tr::VPL;
 
     extern __shared__ __align__(16) unsigned char quant_smem_raw[];
@@ -115,7 +121,7 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
         const int n = w + 4 * (it & 3);
         const bool is_key = it < 4;
         if (n < lo_slot || n >= hi_slot) {
-            if (is_key) {
+            if (QJ && is_key) {
 #pragma unroll
                 for (int k = 0; k < VPL / 2; ++k) {
                     rh[n][lane * (VPL / 2) + k] = 0u;
@@ -154,7 +160,11 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
         wht_warp<VPL>(x, lane);
         const double nrm = sqrt(ss);
         const double scale = nrm > 0.0 ? inv_sqrt_d / nrm : 0.0;
-        if (is_key) {
+        if (is_key && !QJ) {
+#pragma unroll
+            for (int k = 0; k < VPL; ++k) kc[n][lane * VPL + k] = (uint8_t)encode_cell<BK>(x[k] * scale, tk_s);
+            if (lane == 0) nk[n] = norm_to_half_bits(nrm, sat);
+        } else if (is_key) {
             double r[VPL], rr = 0.0;
 #pragma unroll
             for (int k = 0; k < VPL; ++k) {
@@ -192,7 +202,7 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
     __syncthreads();
 
     // ---------------- 2. z = S r on the tensor cores ----------------
-    {
+    if constexpr (QJ) {
         const int g = lane >> 2, t = lane & 3;
         float acc[Tr::NTW][4];
 #pragma unroll
@@ -309,7 +319,11 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
                 mask[q] = msk;
             }
             uint8_t* dst = tile_ptr + ((size_t)c * 32 + L) * Tr::CB;
-            if constexpr (Tr::CW == 4) {
+            if constexpr (Tr::CW == 1) {
+                uint32_t v = word[0];
+                if (!full) v = (*reinterpret_cast<const uint32_t*>(dst) & ~mask[0]) | (v & mask[0]);
+                *reinterpret_cast<uint32_t*>(dst) = v;
+            } else if constexpr (Tr::CW == 4) {
                 uint4 v = make_uint4(word[0], word[1], word[2], word[3]);
                 if (!full) {
                     const uint4 o = *reinterpret_cast<const uint4*>(dst);
@@ -329,21 +343,27 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
                 *reinterpret_cast<uint2*>(dst) = v;
             }
         }
-        // norms: 32 halves of |k|, rho then 16 halves of |v|
-        if (tid < 48) {
-            const size_t base = (size_t)4 * BITS * D;
+        // norms: QJ: 32 halves of |k|, rho, else 16 halves of |k|; then 16 of |v|
+        constexpr int NKH = 16 + 16 * QJ;
+        if (tid < NKH + 16) {
+            const size_t base = (size_t)Tr::CODE_BYTES;
             int tok, off;
             uint16_t v16;
-            if (tid < 32) {
+            if (QJ && tid < 32) {
                 const int g2 = tid >> 2, s = tid & 3;
                 tok = g2 + 8 * (s >> 1);
                 v16 = (s & 1) ? nr[tok] : nk[tok];
                 off = 8 * g2 + 2 * s;
+            } else if (!QJ && tid < 16) {
+                const int g2 = tid >> 1, s = tid & 1;
+                tok = g2 + 8 * s;
+                v16 = nk[tok];
+                off = 4 * g2 + 2 * s;
             } else {
-                const int u = tid - 32, g2 = u >> 1, s = u & 1;
+                const int u = tid - NKH, g2 = u >> 1, s = u & 1;
                 tok = g2 + 8 * s;
                 v16 = nv[tok];
-                off = 64 + 4 * g2 + 2 * s;
+                off = Tr::KNB + 4 * g2 + 2 * s;
             }
             if (is_new(tok)) *reinterpret_cast<uint16_t*>(tile_ptr + base + off) = v16;
         }
@@ -351,34 +371,35 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
     if (sat) atomicOr(tb.status, TQ_STATUS_NORM_SAT);
 }
 
-template <int D, int BITS>
+template <int D, int KB, int VB, int QJ>
 cudaError_t launch_quantize_t(const DevTables& tb, const QuantizeArgs& a, cudaStream_t st)
 {
     const int tiles = (a.T + 15) / 16 + 1;
     dim3 grid(tiles, a.Hkv, a.B);
     const size_t smem = sizeof(QuantSmem<D>);
-    static bool attr_set = false;   // one attribute call per instantiation
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(quantize_kernel<D, BITS>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)smem);
+    auto kern = quantize_kernel<D, KB, VB, QJ>;
+    static unsigned long long done = 0;   // one attribute call per (instantiation, device)
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(__atomic_load_n(&done, __ATOMIC_ACQUIRE) & bit)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        __atomic_fetch_or(&done, bit, __ATOMIC_ACQ_REL);
     }
-    quantize_kernel<D, BITS><<<grid, 128, smem, st>>>(tb, a);
+    kern<<<grid, 128, smem, st>>>(tb, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_quantize(int d, int bits, const DevTables& tb, const QuantizeArgs& a,
+cudaError_t launch_quantize(const Format& f, const DevTables& tb, const QuantizeArgs& a,
                             cudaStream_t st)
 {
-#define TQ_Q(DD, BB) \
-    if (d == DD && bits == BB) return launch_quantize_t<DD, BB>(tb, a, st);
-    TQ_Q(64, 2) TQ_Q(64, 3) TQ_Q(64, 4)
-    TQ_Q(128, 2) TQ_Q(128, 3) TQ_Q(128, 4)
-    TQ_Q(256, 2) TQ_Q(256, 3) TQ_Q(256, 4)
+#define TQ_Q(DD, KB, VB, QJ) \
+    if (f.d == DD && f.kb == KB && f.vb == VB && f.qjl == QJ) return launch_quantize_t<DD, KB, VB, QJ>(tb, a, st);
+    TQ_FORMATS(TQ_Q)
 #undef TQ_Q
     return cudaErrorInvalidValue;
 }

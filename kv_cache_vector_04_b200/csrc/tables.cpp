@@ -170,13 +170,14 @@ float choose_decode_scale(const float* centroids, int n, int d)
     return float(best);
 }
 
-bool build_host_tables(int d, int bits, uint64_t seed, HostTables& t)
+bool build_host_tables(int d, int kbits, int vbits, int qjl, uint64_t seed, HostTables& t)
 {
     t.d = d;
-    t.bits = bits;
+    t.bits = vbits;
     t.m = d;
-    t.kbits = bits - 1;
-    t.vbits = bits;
+    t.kbits = kbits;
+    t.vbits = vbits;
+    t.qjl = qjl;
     t.centroids_k.assign(1u << t.kbits, 0.f);
     t.bounds_k.assign((1u << t.kbits) - 1, 0.f);
     t.centroids_v.assign(1u << t.vbits, 0.f);

@@ -6,7 +6,7 @@
 namespace tq {
 
 struct HostTables {
-    int d = 0, bits = 0, m = 0, kbits = 0, vbits = 0;
+    int d = 0, bits = 0, m = 0, kbits = 0, vbits = 0, qjl = 1;
     std::vector<float> centroids_k, bounds_k;  // 2^kbits levels, 2^kbits - 1 edges (fp32)
     std::vector<float> centroids_v, bounds_v;  // 2^vbits levels, 2^vbits - 1 edges (fp32)
     std::vector<int8_t> signs;                 // D: d entries of +-1
@@ -20,7 +20,8 @@ struct HostTables {
 bool build_codebook(int B, int d, float* centroids, float* bounds);
 void build_rotation_signs(int d, uint64_t seed, int8_t* signs);
 void build_qjl_matrix(int m, int d, uint64_t seed, float* S);
-bool build_host_tables(int d, int bits, uint64_t seed, HostTables& t);
+// Tables of the format (kbits, vbits, qjl); TurboQuant at b bits is (b-1, b, 1).
+bool build_host_tables(int d, int kbits, int vbits, int qjl, uint64_t seed, HostTables& t);
 // Scale in [1, 2) that puts alpha * sqrt(d) * c_j closest to fp16 values for
 // the n/2 positive levels c_j (the kernel's decode table precision).
 float choose_decode_scale(const float* centroids, int n, int d);

@@ -102,11 +102,11 @@ def stack_codes(codes, cap: int):
 def pack_cache(tab: O.Tables, codes, cap: int, d: int, bits: int) -> torch.Tensor:
     """Oracle-packed cache bytes for [B][Hkv] code streams, as a CUDA tensor."""
     B, Hkv = len(codes), len(codes[0])
-    tb = O.tile_bytes(d, bits)
+    tb = O.tile_bytes(d, tab)   # the context's format (tab.fmt)
     host = np.zeros(B * Hkv * (cap // 16) * tb, np.uint8)
     for b in range(B):
         for h in range(Hkv):
-            s = O.pack_stream(d, bits, codes[b][h])
+            s = O.pack_stream(d, tab, codes[b][h])
             s0 = (b * Hkv + h) * (cap // 16) * tb
             host[s0: s0 + s.size] = s
     return torch.from_numpy(host).cuda()

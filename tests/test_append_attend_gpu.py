@@ -22,8 +22,8 @@ pytestmark = pytest.mark.gpu
 DB = [(d, b) for d in (64, 128, 256) for b in (2, 3, 4)]
 
 
-def _run(d, bits, T, starts, Hq=8, seed=0):
-    ctx, tab = ctx_for(d, bits)
+def _run(d, bits, T, starts, Hq=8, seed=0, fmt=None):
+    ctx, tab = ctx_for(d, bits, fmt=fmt)
     B, Hkv, cap = len(starts), 2, 96
     pre = max(starts)
     cache = tq.new_cache(ctx, B, Hkv, cap)
@@ -53,8 +53,8 @@ def _run(d, bits, T, starts, Hq=8, seed=0):
         row = []
         for h in range(Hkv):
             s0 = (b * Hkv + h) * per
-            new = O.unpack_stream(d, bits, cap, after[s0: s0 + per])
-            old = O.unpack_stream(d, bits, cap, before[s0: s0 + per])
+            new = O.unpack_stream(d, tab, cap, after[s0: s0 + per])
+            old = O.unpack_stream(d, tab, cap, before[s0: s0 + per])
             sel = np.zeros(cap, bool)
             sel[starts[b]: starts[b] + T] = True
             for key in new:

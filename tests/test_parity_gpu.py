@@ -16,10 +16,16 @@ DB = [(d, b) for d in (64, 128, 256) for b in (2, 3, 4)]
 _ctx_cache = {}
 
 
-def ctx_for(d, bits, seed=1):
-    key = (d, bits, seed)
+def ctx_for(d, bits, seed=1, fmt=None):
+    """(library context, oracle tables) of TurboQuant at `bits`, or of the
+    format fmt = (B_K, B_V, qjl) when given."""
+    key = (d, bits, seed, fmt)
     if key not in _ctx_cache:
-        _ctx_cache[key] = (tq.tq_init(d, bits, seed), O.Tables(d, bits, seed))
+        if fmt is None:
+            _ctx_cache[key] = (tq.tq_init(d, bits, seed), O.Tables(d, bits, seed))
+        else:
+            _ctx_cache[key] = (tq.tq_init_ex(d, fmt[0], fmt[1], fmt[2], seed),
+                               O.Tables(d, fmt[1], seed, fmt=fmt))
     return _ctx_cache[key]
 
 
@@ -43,7 +49,7 @@ def check_quantize(ctx, tab, k, v, cache, start=0, stats=None):
     for b in range(B):
         for h in range(Hkv):
             sb = P.stream_bytes(host, lay["tile_bytes"], cache.capacity, Hkv, b, h, start + T)
-            gpu = O.unpack_stream(d, tab.bits, start + T, sb)
+            gpu = O.unpack_stream(d, tab, start + T, sb)
             gpu = {kk: vv[start:] for kk, vv in gpu.items()}
             P.compare_stream(tab, gpu, codes[b][h], T, st)
     if stats is None:
