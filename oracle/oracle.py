@@ -59,6 +59,10 @@ def _load():
         "oracle_lloyd_max_unit": (i32, [i32, P, P]),
         "oracle_quantizer_mse_unit": (ctypes.c_double, [i32, P]),
         "oracle_codebook": (i32, [i32, i32, P, P]),
+        "oracle_beta_marginal_pdf": (ctypes.c_double, [i32, ctypes.c_double]),
+        "oracle_lloyd_max_beta": (i32, [i32, i32, P]),
+        "oracle_quantizer_mse_beta": (ctypes.c_double, [i32, i32, P]),
+        "oracle_codebook_beta": (i32, [i32, i32, P, P]),
         "oracle_rotate": (None, [i32, P, P, P]),
         "oracle_rotate_inverse": (None, [i32, P, P, P]),
         "oracle_encode": (i32, [ctypes.c_double, P, i32]),
@@ -140,12 +144,32 @@ def quantizer_mse_unit(B: int, c: np.ndarray) -> float:
     return float(_load().oracle_quantizer_mse_unit(B, _p(c)))
 
 
-def codebook(B: int, d: int):
+def codebook(B: int, d: int, kind: str = "gauss"):
+    """fp32 centroids and boundaries of the B-bit codebook for head dim d:
+    kind "gauss" models a rotated coordinate as N(0, 1/d); "beta" uses its
+    exact marginal (beta_marginal_pdf)."""
     c = np.zeros(1 << B, dtype=np.float32)
     t = np.zeros(max((1 << B) - 1, 1), dtype=np.float32)
-    rc = _load().oracle_codebook(B, d, _p(c), _p(t))
+    fn = _load().oracle_codebook if kind == "gauss" else _load().oracle_codebook_beta
+    rc = fn(B, d, _p(c), _p(t))
     assert rc == 0
     return c, t[: (1 << B) - 1]
+
+
+def beta_marginal_pdf(d: int, y: float) -> float:
+    return float(_load().oracle_beta_marginal_pdf(d, float(y)))
+
+
+def lloyd_max_beta(d: int, B: int):
+    c = np.zeros(1 << B, dtype=np.float64)
+    rc = _load().oracle_lloyd_max_beta(d, B, _p(c))
+    return c, rc
+
+
+def quantizer_mse_beta(d: int, B: int, c: np.ndarray) -> float:
+    """MSE under the exact marginal of the quantizer with centroids c."""
+    c = np.ascontiguousarray(c, dtype=np.float64)
+    return float(_load().oracle_quantizer_mse_beta(d, B, _p(c)))
 
 
 def rotate(D: np.ndarray, u: np.ndarray) -> np.ndarray:
@@ -176,14 +200,16 @@ class Tables:
     1-bit QJL sketch. The default is TurboQuant at b bits, (b - 1, b, 1); the
     MSE-only key formats ("nc", [MUNINN §MSE-Only vs QJL]) have qjl = 0."""
 
-    def __init__(self, d: int, bits: int, seed: int, fmt: tuple | None = None):
+    def __init__(self, d: int, bits: int, seed: int, fmt: tuple | None = None,
+                 kind: str = "gauss"):
         self.d, self.bits, self.seed, self.m = d, bits, seed, d
         self.fmt = fmt_of(bits) if fmt is None else tuple(int(x) for x in fmt)
         self.BK, self.BV, self.qjl = self.fmt
+        self.kind = kind   # the codebooks' coordinate model (see codebook)
         self.D = rotation_signs(d, seed)
         self.S = qjl_matrix(d, d, seed)
-        self.cK, self.tK = codebook(self.BK, d)
-        self.cV, self.tV = codebook(self.BV, d)
+        self.cK, self.tK = codebook(self.BK, d, kind)
+        self.cV, self.tV = codebook(self.BV, d, kind)
 
 
 def fmt_of(x) -> tuple:

@@ -252,6 +252,115 @@ int oracle_codebook(int B, int d, float* centroids, float* bounds)
 }
 
 /* ------------------------------------------------------------------------- */
+/* Exact coordinate marginal [WISELY §TurboQuant 是什麼, step 1: a random      */
+/* rotation concentrates the coordinates as a Beta distribution]              */
+/* ------------------------------------------------------------------------- */
+
+/* Density of one coordinate y of a uniformly random unit vector in R^d, d >= 3:
+ *   f_d(y) = Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2)) (1 - y^2)^((d-3)/2),  |y| < 1,
+ * i.e. (1 + y)/2 ~ Beta((d-1)/2, (d-1)/2). N(0, 1/d) is its large-d limit. */
+double oracle_beta_marginal_pdf(int d, double y)
+{
+    if (!(y > -1.0 && y < 1.0)) return 0.0;
+    double logc = lgamma(0.5 * d) - 0.5 * log(M_PI) - lgamma(0.5 * (d - 1));
+    return exp(logc + 0.5 * (d - 3) * log1p(-y * y));
+}
+
+/* Moments m_k = integral over [lo, hi] of y^k f_d(y) dy, k = 0, 1, 2, by
+ * composite Simpson in theta with y = sin(theta): the integrand becomes
+ * c_d sin^k(theta) cos^(d-2)(theta), smooth up to the ends of [-1, 1]. */
+static void beta_moments(int d, double lo, double hi, double* m0, double* m1, double* m2)
+{
+    *m0 = *m1 = *m2 = 0.0;
+    if (lo < -1.0) lo = -1.0;
+    if (hi > 1.0) hi = 1.0;
+    if (!(hi > lo)) return;
+    const int n = 20000;   /* panels, even */
+    double a = asin(lo), b = asin(hi), h = (b - a) / n;
+    double logc = lgamma(0.5 * d) - 0.5 * log(M_PI) - lgamma(0.5 * (d - 1));
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0;
+    for (int i = 0; i <= n; ++i) {
+        double th = a + i * h, w = (i == 0 || i == n) ? 1.0 : ((i & 1) ? 4.0 : 2.0);
+        double cs = cos(th), sn = sin(th);
+        double f = (cs > 0.0) ? w * exp(logc + (d - 2) * log(cs)) : 0.0;
+        s0 += f;
+        s1 += f * sn;
+        s2 += f * sn * sn;
+    }
+    *m0 = s0 * h / 3.0;
+    *m1 = s1 * h / 3.0;
+    *m2 = s2 * h / 3.0;
+}
+
+/* Lloyd–Max for f_d with L = 2^B levels: midpoint boundaries, centroids the
+ * conditional means m1/m0 of their cells. Starts from the N(0,1/d) codebook
+ * (d >= 16) or from the uniform quantizer on [-1, 1], and stops like the
+ * Gaussian iteration (at the fp64/quadrature noise floor). Symmetrised. */
+int oracle_lloyd_max_beta(int d, int B, double* c)
+{
+    int L = 1 << B;
+    if (d >= 16) {
+        double g[16];
+        oracle_lloyd_max_unit(B, g, NULL);
+        for (int j = 0; j < L; ++j) c[j] = g[j] / sqrt((double)d);
+    } else {
+        for (int j = 0; j < L; ++j) c[j] = -1.0 + (2.0 * j + 1.0) / L;
+    }
+    double nc[16], prev = INFINITY;
+    int ok = -1;
+    for (int it = 0; it < 100000; ++it) {
+        double delta = 0.0;
+        for (int j = 0; j < L; ++j) {
+            double lo = (j == 0) ? -1.0 : 0.5 * (c[j - 1] + c[j]);
+            double hi = (j == L - 1) ? 1.0 : 0.5 * (c[j] + c[j + 1]);
+            double m0, m1, m2;
+            beta_moments(d, lo, hi, &m0, &m1, &m2);
+            nc[j] = m1 / m0;
+            double dd = fabs(nc[j] - c[j]);
+            if (dd > delta) delta = dd;
+        }
+        memcpy(c, nc, sizeof(double) * L);
+        if (delta == 0.0 || (delta < 1e-13 && delta >= prev)) { ok = 0; break; }
+        prev = delta;
+    }
+    for (int j = 0; j < L / 2; ++j) {
+        double s = 0.5 * (c[L - 1 - j] - c[j]);
+        c[j] = -s;
+        c[L - 1 - j] = s;
+    }
+    return ok;
+}
+
+/* Mean squared error, under f_d, of the quantizer with centroids c (any scale:
+ * these are coordinates of a unit vector) and midpoint cells. */
+double oracle_quantizer_mse_beta(int d, int B, const double* c)
+{
+    int L = 1 << B;
+    double mse = 0.0;
+    for (int j = 0; j < L; ++j) {
+        double lo = (j == 0) ? -1.0 : 0.5 * (c[j - 1] + c[j]);
+        double hi = (j == L - 1) ? 1.0 : 0.5 * (c[j] + c[j + 1]);
+        double m0, m1, m2;
+        beta_moments(d, lo, hi, &m0, &m1, &m2);
+        mse += m2 - 2.0 * c[j] * m1 + c[j] * c[j] * m0;
+    }
+    return mse;
+}
+
+/* The exact-marginal codebook: oracle_lloyd_max_beta rounded once to fp32,
+ * boundaries the fp32 midpoints (the same rounding as oracle_codebook). */
+int oracle_codebook_beta(int B, int d, float* centroids, float* bounds)
+{
+    double c[16];
+    int rc = oracle_lloyd_max_beta(d, B, c);
+    int L = 1 << B;
+    for (int j = 0; j < L; ++j) centroids[j] = (float)c[j];
+    for (int j = 0; j + 1 < L; ++j)
+        bounds[j] = (float)(0.5 * ((double)centroids[j] + (double)centroids[j + 1]));
+    return rc;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Rotation [DIGIPUB opening; MUNINN §30 秒懶人包; WISELY step 1]              */
 /* ------------------------------------------------------------------------- */
 
