@@ -154,7 +154,7 @@ def profiled_traffic(workload: str):
     was taken on this workload and on the kernel source as it is now (else None)."""
     import hashlib
     prof = os.path.join(ROOT, "profiles", "attend_split_llama70b_32k.md")
-    src = os.path.join(ROOT, "kv_cache_vector_04_b200", "csrc", "attend.cu")
+    src = os.path.join(ROOT, "kv_cache_vector_04_b200", "csrc", "attend_impl.cuh")
     if workload != DEFAULT_WORKLOAD or not os.path.exists(prof):
         return None
     fields = {}

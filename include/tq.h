@@ -62,6 +62,9 @@ extern "C" {
 #define TQ_TILE 16 /* tokens per packed tile */
 
 /* dtypes of query input */
+#define TQ_CODEBOOK_GAUSS 0 /* Lloyd–Max for N(0, 1/d), the pages' coordinate model */
+#define TQ_CODEBOOK_BETA 1  /* Lloyd–Max for the exact marginal: (1 + y)/2 ~ Beta((d-1)/2, (d-1)/2) */
+
 #define TQ_DTYPE_F16 0
 #define TQ_DTYPE_BF16 1
 
@@ -141,7 +144,15 @@ int tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
  * "no QJL correction" ([MUNINN] §"MSE-Only vs QJL" contrasts the two). Without
  * QJL the logit is |k| <Pi q, cK[idx]> / sqrt(d), the biased MSE-only
  * estimate. Other formats return TQ_ERR_UNSUPPORTED. */
-int tq_init_ex(int d, int kbits, int vbits, int qjl, uint64_t seed, tq_ctx** out);
+int tq_init_ex(int d, int kbits, int vbits, int qjl, int codebook, uint64_t seed, tq_ctx** out);
+/* codebook (tq_init_ex): TQ_CODEBOOK_GAUSS, or TQ_CODEBOOK_BETA for the exact
+ * distribution of a rotated unit-vector coordinate, which the N(0, 1/d) model
+ * approximates (turboquant-kvquant-vllm-benchmark, "TurboQuant 是什麼", step
+ * 1: the rotation concentrates the coordinates as a Beta distribution). */
+
+/* One codebook alone, on the host (no device, no context): B in 1..4 bits,
+ * d >= 3; fp32 centroids[2^B] and boundaries[2^B - 1] (fp32 midpoints). */
+int tq_build_codebook(int B, int d, int codebook, float* centroids, float* bounds);
 
 /* Free a context and its device tables. NULL is ignored. */
 void tq_destroy(tq_ctx* ctx);
@@ -153,7 +164,7 @@ int tq_cache_layout(const tq_ctx* ctx, tq_layout* out);
 int tq_cache_bytes(const tq_ctx* ctx, int B, int Hkv, int capacity, size_t* bytes);
 
 /* Host copies of the tables, for checking (any pointer may be NULL):
- * centroids_k[2^(b-1)], bounds_k[2^(b-1)-1], centroids_v[2^b], bounds_v[2^b-1]
+ * centroids_k[2^B_K], bounds_k[2^B_K-1], centroids_v[2^B_V], bounds_v[2^B_V-1]
  * (fp32), signs[d] (int8 ±1), S[m*d] (fp32, row-major, fp16-exact values). */
 int tq_get_tables(const tq_ctx* ctx, float* centroids_k, float* bounds_k, float* centroids_v,
                   float* bounds_v, int8_t* signs, float* S);

@@ -28,11 +28,13 @@ TQ_STATUS_SEQ_LEN = 0x2
 TQ_STATUS_NORM_SAT = 0x4
 TQ_STATUS_WAIT_TIMEOUT = 0x8
 TQ_TILE = 16
+TQ_CODEBOOK_GAUSS = 0
+TQ_CODEBOOK_BETA = 1
 TQ_DTYPE_F16 = 0
 TQ_DTYPE_BF16 = 1
 
 # every symbol include/tq.h declares
-EXPORTS = ("tq_init", "tq_init_ex", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
+EXPORTS = ("tq_init", "tq_init_ex", "tq_build_codebook", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
            "tq_build_tables", "tq_quantize", "tq_attend_workspace", "tq_attend", "tq_scores",
            "tq_attend_noalloc", "tq_append_attend", "tq_status", "tq_copy", "tq_strerror")
 TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -65,7 +67,8 @@ def _load(path: str = LIB_PATH):
     P, I, U64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
     sig = {
         "tq_init": (I, [I, I, U64, ctypes.POINTER(P)]),
-        "tq_init_ex": (I, [I, I, I, I, U64, ctypes.POINTER(P)]),
+        "tq_init_ex": (I, [I, I, I, I, I, U64, ctypes.POINTER(P)]),
+        "tq_build_codebook": (I, [I, I, I, P, P]),
         "tq_destroy": (None, [P]),
         "tq_cache_layout": (I, [P, ctypes.POINTER(_Layout)]),
         "tq_cache_bytes": (I, [P, I, I, I, ctypes.POINTER(SZ)]),
@@ -169,13 +172,25 @@ def tq_init(d: int, bits: int, seed: int) -> Context:
     return Context(h.value, d, bits, seed, torch.cuda.current_device())
 
 
-def tq_init_ex(d: int, kbits: int, vbits: int, qjl: int, seed: int) -> Context:
-    """A context of any built format: (kbits, vbits, qjl) = (B_K, B_V, QJL on keys)."""
+def tq_init_ex(d: int, kbits: int, vbits: int, qjl: int, seed: int,
+               codebook: int = TQ_CODEBOOK_GAUSS) -> Context:
+    """A context of any built format: (kbits, vbits, qjl) = (B_K, B_V, QJL on
+    keys); codebook TQ_CODEBOOK_GAUSS or TQ_CODEBOOK_BETA (exact marginal)."""
     h = ctypes.c_void_p()
-    _check(_lib.tq_init_ex(int(d), int(kbits), int(vbits), int(qjl), ctypes.c_uint64(seed),
-                           ctypes.byref(h)), "tq_init_ex")
+    _check(_lib.tq_init_ex(int(d), int(kbits), int(vbits), int(qjl), int(codebook),
+                           ctypes.c_uint64(seed), ctypes.byref(h)), "tq_init_ex")
     return Context(h.value, d, vbits, seed, torch.cuda.current_device(),
                    fmt=(int(kbits), int(vbits), int(qjl)))
+
+
+def tq_build_codebook(B: int, d: int, codebook: int = TQ_CODEBOOK_GAUSS):
+    """Host-only codebook: (fp32 centroids [2^B], fp32 boundaries [2^B - 1])."""
+    import numpy as np
+    c = np.zeros(1 << B, np.float32)
+    t = np.zeros(max((1 << B) - 1, 1), np.float32)
+    _check(_lib.tq_build_codebook(int(B), int(d), int(codebook), c.ctypes.data_as(ctypes.c_void_p),
+                                  t.ctypes.data_as(ctypes.c_void_p)), "tq_build_codebook")
+    return c, t[: (1 << B) - 1]
 
 
 def tq_destroy(ctx: Context):
@@ -202,26 +217,28 @@ def new_cache(ctx: Context, B: int, Hkv: int, capacity: int, device=None) -> Cac
     return Cache(torch.zeros(n, dtype=torch.uint8, device=dev), B, Hkv, capacity)
 
 
-def _tables(fn, d: int, bits: int, args_prefix):
+def _tables(fn, d: int, kbits: int, vbits: int, args_prefix):
     import numpy as np
-    ck = np.zeros(1 << (bits - 1), np.float32)
-    tk = np.zeros(max((1 << (bits - 1)) - 1, 1), np.float32)
-    cv = np.zeros(1 << bits, np.float32)
-    tv = np.zeros((1 << bits) - 1, np.float32)
+    ck = np.zeros(1 << kbits, np.float32)
+    tk = np.zeros(max((1 << kbits) - 1, 1), np.float32)
+    cv = np.zeros(1 << vbits, np.float32)
+    tv = np.zeros((1 << vbits) - 1, np.float32)
     sg = np.zeros(d, np.int8)
     S = np.zeros((d, d), np.float32)
     p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
     _check(fn(*args_prefix, p(ck), p(tk), p(cv), p(tv), p(sg), p(S)), fn.__name__)
-    return dict(centroids_k=ck, bounds_k=tk[: (1 << (bits - 1)) - 1], centroids_v=cv,
+    return dict(centroids_k=ck, bounds_k=tk[: (1 << kbits) - 1], centroids_v=cv,
                 bounds_v=tv, signs=sg, S=S)
 
 
 def tq_get_tables(ctx: Context) -> dict:
-    return _tables(_lib.tq_get_tables, ctx.d, ctx.bits, (ctx.handle,))
+    """Host copies of a context's tables (arrays sized by its format)."""
+    return _tables(_lib.tq_get_tables, ctx.d, ctx.fmt[0], ctx.fmt[1], (ctx.handle,))
 
 
 def tq_build_tables(d: int, bits: int, seed: int) -> dict:
-    return _tables(_lib.tq_build_tables, d, bits, (int(d), int(bits), ctypes.c_uint64(seed)))
+    """TurboQuant tables at b = bits computed on the host only."""
+    return _tables(_lib.tq_build_tables, d, bits - 1, bits, (int(d), int(bits), ctypes.c_uint64(seed)))
 
 
 # ------------------------------------------------------------------ quantize / attend

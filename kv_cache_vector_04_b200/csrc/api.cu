@@ -237,12 +237,22 @@ int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const 
 
 extern "C" {
 
+int tq_build_codebook(int B, int d, int codebook, float* centroids, float* bounds)
+{
+    if (B < 1 || B > 4 || d < 3 || d > 4096 || !centroids || !bounds) return TQ_ERR_INVALID_ARG;
+    if (codebook == TQ_CODEBOOK_GAUSS)
+        return tq::build_codebook(B, d, centroids, bounds) ? TQ_OK : TQ_ERR_CUDA;
+    if (codebook == TQ_CODEBOOK_BETA)
+        return tq::build_codebook_beta(B, d, centroids, bounds) ? TQ_OK : TQ_ERR_CUDA;
+    return TQ_ERR_UNSUPPORTED;
+}
+
 int tq_build_tables(int d, int bits, uint64_t seed, float* centroids_k, float* bounds_k,
                     float* centroids_v, float* bounds_v, int8_t* signs, float* S)
 {
     if (!supported(d, bits - 1, bits, 1)) return TQ_ERR_UNSUPPORTED;
     tq::HostTables t;
-    if (!tq::build_host_tables(d, bits - 1, bits, 1, seed, t)) return TQ_ERR_CUDA;
+    if (!tq::build_host_tables(d, bits - 1, bits, 1, TQ_CODEBOOK_GAUSS, seed, t)) return TQ_ERR_CUDA;
     if (centroids_k) std::memcpy(centroids_k, t.centroids_k.data(), t.centroids_k.size() * 4);
     if (bounds_k) std::memcpy(bounds_k, t.bounds_k.data(), t.bounds_k.size() * 4);
     if (centroids_v) std::memcpy(centroids_v, t.centroids_v.data(), t.centroids_v.size() * 4);
@@ -254,14 +264,15 @@ int tq_build_tables(int d, int bits, uint64_t seed, float* centroids_k, float* b
 
 int tq_init(int d, int bits, uint64_t seed, tq_ctx** out)
 {
-    return tq_init_ex(d, bits - 1, bits, 1, seed, out);
+    return tq_init_ex(d, bits - 1, bits, 1, TQ_CODEBOOK_GAUSS, seed, out);
 }
 
-int tq_init_ex(int d, int kbits, int vbits, int qjl, uint64_t seed, tq_ctx** out)
+int tq_init_ex(int d, int kbits, int vbits, int qjl, int codebook, uint64_t seed, tq_ctx** out)
 {
     if (!out) return TQ_ERR_INVALID_ARG;
     *out = nullptr;
     if (!supported(d, kbits, vbits, qjl)) return TQ_ERR_UNSUPPORTED;
+    if (codebook != TQ_CODEBOOK_GAUSS && codebook != TQ_CODEBOOK_BETA) return TQ_ERR_UNSUPPORTED;
     tq_ctx* ctx = new (std::nothrow) tq_ctx();
     if (!ctx) return TQ_ERR_INVALID_ARG;
     ctx->d = d;
@@ -269,7 +280,7 @@ int tq_init_ex(int d, int kbits, int vbits, int qjl, uint64_t seed, tq_ctx** out
     ctx->kbits = kbits;
     ctx->vbits = vbits;
     ctx->qjl = qjl;
-    if (!tq::build_host_tables(d, kbits, vbits, qjl, seed, ctx->host)) {
+    if (!tq::build_host_tables(d, kbits, vbits, qjl, codebook, seed, ctx->host)) {
         delete ctx;
         return TQ_ERR_CUDA;
     }

@@ -110,7 +110,99 @@ bool gaussian_lloyd_max(int B, double* level)
     return converged;
 }
 
+// Regularized incomplete beta I_x(p, p) for x <= 1/2, by the continued
+// fraction of the incomplete beta function (Abramowitz & Stegun 26.5.8)
+// evaluated with the modified Lentz method.
+double incomplete_beta_sym(double p, double x)
+{
+    if (x <= 0.0) return 0.0;
+    const double a = p, b = p, tiny = 1e-300;
+    // I_x(a, b) = x^a (1-x)^b / (a B(a, b)) / g with
+    // g = 1 + e1 / (1 + e2 / (1 + ...)), e_{2m+1} = -(a+m)(a+b+m)x / ((a+2m)(a+2m+1)),
+    // e_{2m} = m(b-m)x / ((a+2m-1)(a+2m)); Lentz: f = g, C and Dn the running ratios.
+    double f = 1.0, C = 1.0, Dn = 0.0;
+    for (int i = 1; i <= 100000; ++i) {
+        const int m = i / 2;
+        const double e = (i & 1) ? -(a + m) * (a + b + m) * x / ((a + 2 * m) * (a + 2 * m + 1))
+                                 : m * (b - m) * x / ((a + 2 * m - 1) * (a + 2 * m));
+        Dn = 1.0 + e * Dn;
+        if (std::fabs(Dn) < tiny) Dn = tiny;
+        C = 1.0 + e / C;
+        if (std::fabs(C) < tiny) C = tiny;
+        Dn = 1.0 / Dn;
+        const double step = C * Dn;
+        f *= step;
+        if (std::fabs(step - 1.0) < 1e-16) break;
+    }
+    const double front = std::exp(std::lgamma(a + b) - std::lgamma(a) - std::lgamma(b) +
+                                  a * std::log(x) + b * std::log1p(-x));
+    return front / (a * f);
+}
+
 }  // namespace
+
+// Lloyd–Max for the exact marginal of one coordinate of a random unit vector
+// in R^d: (1 + y)/2 ~ Beta(p, p), p = (d-1)/2, density c_d (1 - y^2)^((d-3)/2).
+// Cell mass from the incomplete beta function (by symmetry always evaluated on
+// the lower half), first moment in closed form:
+//   int y (1-y^2)^al dy = -(1-y^2)^(al+1) / (2 (al+1)),  al = (d-3)/2.
+// Starting point and stopping rule as for the Gaussian iteration.
+bool beta_lloyd_max(int B, int d, double* level)
+{
+    const int n = 1 << B;
+    const double p = 0.5 * (d - 1), al = 0.5 * (d - 3);
+    const double logc = std::lgamma(0.5 * d) - 0.5 * std::log(M_PI) - std::lgamma(0.5 * (d - 1));
+    auto lower = [&](double t) {   // P(y <= t) for t <= 0
+        return incomplete_beta_sym(p, 0.5 * (1.0 + t));
+    };
+    auto mass = [&](double lo, double hi) {   // P(lo < y < hi), -1 <= lo < hi <= 1
+        if (hi <= 0.0) return lower(hi) - lower(lo);
+        if (lo >= 0.0) return lower(-lo) - lower(-hi);
+        return (0.5 - lower(lo)) + (0.5 - lower(-hi));
+    };
+    auto first = [&](double lo, double hi) {   // E[y; lo < y < hi]
+        const double plo = std::exp(logc + (al + 1.0) * std::log1p(-lo * lo));
+        const double phi = std::exp(logc + (al + 1.0) * std::log1p(-hi * hi));
+        return (plo - phi) / (2.0 * (al + 1.0));
+    };
+    if (d >= 16) {
+        gaussian_lloyd_max(B, level);
+        for (int j = 0; j < n; ++j) level[j] /= std::sqrt(double(d));
+    } else {
+        for (int j = 0; j < n; ++j) level[j] = -1.0 + (2.0 * j + 1.0) / n;
+    }
+    bool converged = false;
+    double last_step = INFINITY;
+    for (int iter = 0; iter < 100000 && !converged; ++iter) {
+        double moved = 0.0, next[16];
+        for (int j = 0; j < n; ++j) {
+            const double lo = (j == 0) ? -1.0 : 0.5 * (level[j - 1] + level[j]);
+            const double hi = (j == n - 1) ? 1.0 : 0.5 * (level[j] + level[j + 1]);
+            next[j] = first(lo, hi) / mass(lo, hi);
+            moved = std::fmax(moved, std::fabs(next[j] - level[j]));
+        }
+        for (int j = 0; j < n; ++j) level[j] = next[j];
+        converged = moved == 0.0 || (moved < 1e-13 && moved >= last_step);
+        last_step = moved;
+    }
+    for (int j = 0; j < n / 2; ++j) {
+        const double a = 0.5 * (level[n - 1 - j] - level[j]);
+        level[j] = -a;
+        level[n - 1 - j] = a;
+    }
+    return converged;
+}
+
+bool build_codebook_beta(int B, int d, float* centroids, float* bounds)
+{
+    double level[16];
+    const bool ok = beta_lloyd_max(B, d, level);
+    const int n = 1 << B;
+    for (int j = 0; j < n; ++j) centroids[j] = float(level[j]);
+    for (int j = 0; j + 1 < n; ++j)
+        bounds[j] = float((double(centroids[j]) + double(centroids[j + 1])) * 0.5);
+    return ok;
+}
 
 bool build_codebook(int B, int d, float* centroids, float* bounds)
 {
@@ -170,7 +262,8 @@ float choose_decode_scale(const float* centroids, int n, int d)
     return float(best);
 }
 
-bool build_host_tables(int d, int kbits, int vbits, int qjl, uint64_t seed, HostTables& t)
+bool build_host_tables(int d, int kbits, int vbits, int qjl, int codebook, uint64_t seed,
+                       HostTables& t)
 {
     t.d = d;
     t.bits = vbits;
@@ -184,8 +277,10 @@ bool build_host_tables(int d, int kbits, int vbits, int qjl, uint64_t seed, Host
     t.bounds_v.assign((1u << t.vbits) - 1, 0.f);
     t.signs.assign(d, 1);
     t.S.assign(size_t(t.m) * d, 0.f);
-    bool ok = build_codebook(t.kbits, d, t.centroids_k.data(), t.bounds_k.data());
-    ok = build_codebook(t.vbits, d, t.centroids_v.data(), t.bounds_v.data()) && ok;
+    auto cb = codebook == 1 ? build_codebook_beta : build_codebook;
+    t.codebook = codebook;
+    bool ok = cb(t.kbits, d, t.centroids_k.data(), t.bounds_k.data());
+    ok = cb(t.vbits, d, t.centroids_v.data(), t.bounds_v.data()) && ok;
     build_rotation_signs(d, seed, t.signs.data());
     build_qjl_matrix(t.m, d, seed, t.S.data());
     t.alpha_k = choose_decode_scale(t.centroids_k.data(), 1 << t.kbits, d);

@@ -105,3 +105,30 @@ def test_scores_match_oracle_logits(d, fmt):
 @pytest.mark.parametrize("d,fmt", [(64, (2, 2, 0)), (128, (3, 4, 0)), (256, (3, 3, 0))])
 def test_append_one_token_then_attend(d, fmt):
     run_append(d, fmt[1], 1, [32, 37, 47], seed=d + fmt[0], fmt=fmt)
+
+
+# ---------------------------------------------------------------- exact-marginal codebooks
+
+BETA = [(64, (1, 2, 1)), (128, (3, 4, 1)), (128, (3, 3, 0)), (256, (2, 3, 1))]
+
+
+@pytest.mark.parametrize("d,fmt", BETA)
+def test_beta_codebook_tables_quantize_and_attend(d, fmt):
+    # The exact Beta-marginal codebooks ride on the same kernels: the device
+    # tables hold the oracle's codebooks, quantization and attention match.
+    ctx, tab = ctx_for(d, fmt[1], fmt=fmt, kind="beta")
+    t = tq.tq_get_tables(ctx)
+    assert np.array_equal(t["centroids_k"], tab.cK) and np.array_equal(t["centroids_v"], tab.cV)
+    assert np.array_equal(t["bounds_k"], tab.tK) and np.array_equal(t["bounds_v"], tab.tV)
+    stats = P.QuantStats()
+    k, v = kv(2, 2, 97, d, seed=d + fmt[1], dist="spiky_tokens")
+    cache = P.quantize_on_gpu(ctx, k, v, capacity=112)
+    codes = check_quantize(ctx, tab, k, v, cache, stats=stats)
+    stats.check()
+    q = qtensor(2, 8, d, seed=4)
+    seq = [97, 40]
+    got = tq.tq_attend(ctx, q.cuda(), cache, torch.tensor(seq, dtype=torch.int32).cuda(), 97)
+    torch.cuda.synchronize()
+    ref = O.attend_batch(tab, P.q_bits(q), True, P.stack_codes(codes, 112), np.array(seq, np.int32), 2)
+    assert P.attn_error(got.cpu().numpy().astype(np.float64), ref).max() <= P.ATTN_TOL
+    assert tq.tq_status(ctx) == 0

@@ -46,9 +46,10 @@ def test_binding_constants_equal_header_defines():
 def test_unsupported_formats_are_refused_before_any_cuda_call():
     h = ctypes.c_void_p()
     for f in ((2, 4, 1), (5, 5, 0), (4, 3, 0), (1, 1, 0), (3, 4, 2), (2, 3, 0)):
-        assert binding._lib.tq_init_ex(128, f[0], f[1], f[2], 1, ctypes.byref(h)) == \
+        assert binding._lib.tq_init_ex(128, f[0], f[1], f[2], 0, 1, ctypes.byref(h)) == \
             tq.TQ_ERR_UNSUPPORTED, f
-    assert binding._lib.tq_init_ex(96, 3, 4, 0, 1, ctypes.byref(h)) == tq.TQ_ERR_UNSUPPORTED
+    assert binding._lib.tq_init_ex(96, 3, 4, 0, 0, 1, ctypes.byref(h)) == tq.TQ_ERR_UNSUPPORTED
+    assert binding._lib.tq_init_ex(128, 3, 4, 0, 2, 1, ctypes.byref(h)) == tq.TQ_ERR_UNSUPPORTED
 
 
 def test_missing_library_fails_loudly(tmp_path):

@@ -16,16 +16,19 @@ DB = [(d, b) for d in (64, 128, 256) for b in (2, 3, 4)]
 _ctx_cache = {}
 
 
-def ctx_for(d, bits, seed=1, fmt=None):
+def ctx_for(d, bits, seed=1, fmt=None, kind="gauss"):
     """(library context, oracle tables) of TurboQuant at `bits`, or of the
-    format fmt = (B_K, B_V, qjl) when given."""
-    key = (d, bits, seed, fmt)
+    format fmt = (B_K, B_V, qjl) when given; kind "beta" selects the
+    exact-marginal codebooks."""
+    key = (d, bits, seed, fmt, kind)
     if key not in _ctx_cache:
-        if fmt is None:
+        if fmt is None and kind == "gauss":
             _ctx_cache[key] = (tq.tq_init(d, bits, seed), O.Tables(d, bits, seed))
         else:
-            _ctx_cache[key] = (tq.tq_init_ex(d, fmt[0], fmt[1], fmt[2], seed),
-                               O.Tables(d, fmt[1], seed, fmt=fmt))
+            f = (bits - 1, bits, 1) if fmt is None else fmt
+            code = tq.TQ_CODEBOOK_BETA if kind == "beta" else tq.TQ_CODEBOOK_GAUSS
+            _ctx_cache[key] = (tq.tq_init_ex(d, f[0], f[1], f[2], seed, codebook=code),
+                               O.Tables(d, f[1], seed, fmt=f, kind=kind))
     return _ctx_cache[key]
 
 
