@@ -72,10 +72,15 @@ struct AttTraits {
     static constexpr int STAGE_BYTES = TILE_BYTES;
     static constexpr size_t RING_BYTES = (size_t)WARPS * STAGES * STAGE_BYTES;
     static constexpr size_t QF_SMEM = QREG ? 0 : QF_BYTES;
-    // dynamic shared memory: [K table][V table][ring, then the merge buffer][query fragments]
+    // dynamic shared memory: [K table][V table] (unless static), [ring, then the
+    // merge buffer], [query fragments]
     static constexpr size_t BODY_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
-    static constexpr size_t DYN_SMEM = LUT_BYTES + BODY_BYTES + QF_SMEM;
-    static constexpr int SMEM_FIT = (int)((228u * 1024u) / (DYN_SMEM + 2048u));
+    // The decode tables are static shared arrays when they fit there (the
+    // table loads then take their base as an immediate), else the front of
+    // dynamic shared memory (4-bit keys with 4-bit values: 64 KB).
+    static constexpr bool STATIC_LUT = LUT_BYTES <= 40 * 1024;
+    static constexpr size_t DYN_SMEM = (STATIC_LUT ? 0 : LUT_BYTES) + BODY_BYTES + QF_SMEM;
+    static constexpr int SMEM_FIT = (int)((228u * 1024u) / (LUT_BYTES + BODY_BYTES + QF_SMEM + 2048u));
     static constexpr int CTAS_PER_SM = QREG ? (SMEM_FIT < 3 ? SMEM_FIT : 3) : 1;
 };
 
@@ -672,10 +677,14 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
         const uint4 bc = qf.fc(kk, lane);
-        uint32_t ak[4];
+        uint32_t ak[4], as[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-            ak[r] = lut_load(lutk, lut_off(td.s, Tr::KF * (4 * kk + r), Tr::KF, lane4));
+        for (int r = 0; r < 4; ++r) {
+            const int p = 4 * kk + r;
+            ak[r] = lut_load(lutk, lut_off(td.s, Tr::KF * p, Tr::KF, lane4));
+            if constexpr (QJ)
+                as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
+        }
         if (kk == 0) {
             mma_16816_first(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
             mma_16816_first(al, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
@@ -685,12 +694,6 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
         }
         if constexpr (QJ) {
             const uint4 bs = qf.fs(kk, lane);
-            uint32_t as[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int p = 4 * kk + r;
-                as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
-            }
             mma_16816(ah, as[0], as[1], as[2], as[3], bs.x, bs.y);
             mma_16816(al, as[0], as[1], as[2], as[3], bs.z, bs.w);
         }
@@ -781,9 +784,22 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     using Tr = AttTraits<D, KB, VB, QJ>;
     constexpr int KK = Tr::KK, WARPS = Tr::WARPS, NT = Tr::NT;
     extern __shared__ uint4 dyn_smem[];
-    uint32_t* lutk = reinterpret_cast<uint32_t*>(dyn_smem);   // decode tables first
-    uint32_t* lutv = lutk + Tr::NLK * 32;
-    uint8_t* body = reinterpret_cast<uint8_t*>(dyn_smem) + Tr::LUT_BYTES;
+    uint32_t* lutk;
+    uint32_t* lutv;
+    uint8_t* body;
+    if constexpr (Tr::STATIC_LUT) {
+        // two arrays, the value table first: with one combined array ptxas
+        // spends about 28 more instructions per tile on the table addresses
+        __shared__ __align__(16) uint32_t s_lutv[Tr::NLV * 32];
+        __shared__ __align__(16) uint32_t s_lutk[Tr::NLK * 32];
+        lutk = s_lutk;
+        lutv = s_lutv;
+        body = reinterpret_cast<uint8_t*>(dyn_smem);
+    } else {
+        lutk = reinterpret_cast<uint32_t*>(dyn_smem);
+        lutv = lutk + Tr::NLK * 32;
+        body = reinterpret_cast<uint8_t*>(dyn_smem) + Tr::LUT_BYTES;
+    }
 
     const int split = blockIdx.x, unit = blockIdx.y, b = blockIdx.z;
     const int groups = a.plan.groups;
@@ -847,9 +863,22 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     extern __shared__ uint4 dyn_smem[];
     // Lane-replicated decode tables: entry f of lane l at byte f*128 + 4l, so
     // the 32 lanes of a warp always hit 32 different banks.
-    uint32_t* lutk = reinterpret_cast<uint32_t*>(dyn_smem);
-    uint32_t* lutv = lutk + Tr::NLK * 32;
-    uint8_t* body = reinterpret_cast<uint8_t*>(dyn_smem) + Tr::LUT_BYTES;
+    uint32_t* lutk;
+    uint32_t* lutv;
+    uint8_t* body;
+    if constexpr (Tr::STATIC_LUT) {
+        // two arrays, the value table first: with one combined array ptxas
+        // spends about 28 more instructions per tile on the table addresses
+        __shared__ __align__(16) uint32_t s_lutv[Tr::NLV * 32];
+        __shared__ __align__(16) uint32_t s_lutk[Tr::NLK * 32];
+        lutk = s_lutk;
+        lutv = s_lutv;
+        body = reinterpret_cast<uint8_t*>(dyn_smem);
+    } else {
+        lutk = reinterpret_cast<uint32_t*>(dyn_smem);
+        lutv = lutk + Tr::NLK * 32;
+        body = reinterpret_cast<uint8_t*>(dyn_smem) + Tr::LUT_BYTES;
+    }
     float* mrg = reinterpret_cast<float*>(body);            // [WARPS][8][D+2] after a segment
     uint4* qsm = reinterpret_cast<uint4*>(body + Tr::BODY_BYTES);
 
