@@ -32,6 +32,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <utility>
+
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -40,6 +42,13 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+
+// Programmatic dependent launch: every attention launch lets the next kernel in
+// the stream start as soon as all of its own CTAs are running, and waits for
+// its predecessor's completion (and memory) before touching anything that
+// kernel may write. Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 
 // Format (KB, VB, QJ): key cells of KB bits, value cells of VB bits, and the
 // QJL sketch of the key residual (with rho) iff QJ = 1.
@@ -269,6 +278,8 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
 template <int D>
 __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArgs a)
 {
+    pdl_trigger();
+    pdl_wait();
     prologue_body<D>(tb, a);
 }
 
@@ -459,6 +470,8 @@ __global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArg
 {
     extern __shared__ uint4 app_smem[];
     const int units = a.Hkv * a.plan.groups;
+    pdl_trigger();
+    pdl_wait();
     if ((int)blockIdx.x >= units)
         append_tokens<D, KB, VB, QJ>(tb, a, blockIdx.y, blockIdx.x - units, reinterpret_cast<uint8_t*>(app_smem));
     else
@@ -467,15 +480,21 @@ __global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArg
 
 
 // ---------------------------------------------------------------- reduction
-// One CTA per (query head, batch): merges the partials of the CTAs whose
-// ranges cover the head's unit (the range of CTA c is [c W / G, (c+1) W / G)
-// of the W tiles, so tile x lies in CTA ((x + 1) G - 1) / W), then applies
-// Pi^T with an fp32 Walsh-Hadamard transform.
+// One CTA per (query head, batch): merges, in one online-softmax pass, the
+// partials of the CTAs whose ranges cover the head's unit (the range of CTA c
+// is [c W / G, (c+1) W / G) of the W tiles, so tile x lies in CTA
+// ((x + 1) G - 1) / W), then applies Pi^T with an fp32 Walsh-Hadamard
+// transform: thread i holds coordinate i = 32 w + lane; the butterflies over
+// the lane bits run on shuffles, those over the warp bits through shared
+// memory (double-buffered: one barrier per stage).
 template <int D>
 __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
 {
-    __shared__ float os[D];
-    const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+    constexpr int NW = D / 32;
+    __shared__ float xs[2][NW][33];
+    pdl_trigger();
+    pdl_wait();
+    const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x, w = i >> 5, lane = i & 31;
     const int ratio = a.Hq / a.Hkv, groups = a.plan.groups;
     const int hkv = hq / ratio, jh = hq % ratio, grp = jh >> 3, col = jh & 7;
     const int upb = a.Hkv * groups, ju = hkv * groups + grp;
@@ -490,31 +509,35 @@ __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
         const int cf = (int)(((U0 + 1) * G - 1) / W), cl = (int)((U1 * G - 1) / W);
         for (int c = cf; c <= cl; ++c) {
             if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;   // empty range
-            M = fmaxf(M, a.partial[((size_t)c + u) * 8 * RS + col * RS]);
-        }
-        if (M != -CUDART_INF_F) {
-            for (int c = cf; c <= cl; ++c) {
-                if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;
-                const float* ps = a.partial + ((size_t)c + u) * 8 * RS + col * RS;
-                const float ms = ps[0];
-                if (ms == -CUDART_INF_F) continue;
-                const float f = exp2f(ms - M);
-                L = fmaf(ps[1], f, L);
-                acc = fmaf(ps[2 + i], f, acc);
+            const float* ps = a.partial + ((size_t)c + u) * 8 * RS + col * RS;
+            const float ms = ps[0];
+            if (ms == -CUDART_INF_F) continue;
+            if (ms > M) {   // rescale what was merged so far (nothing while M = -inf)
+                const float f = M == -CUDART_INF_F ? 0.f : exp2f(M - ms);
+                L *= f;
+                acc *= f;
+                M = ms;
             }
+            const float f = exp2f(ms - M);
+            L = fmaf(ps[1], f, L);
+            acc = fmaf(ps[2 + i], f, acc);
         }
     }
-    os[i] = (L > 0.f) ? acc / L : 0.f;
-    __syncthreads();
+    float x = (L > 0.f) ? acc / L : 0.f;
 #pragma unroll
-    for (int s = 1; s < D; s <<= 1) {
-        const float mine = os[i], other = os[i ^ s];
+    for (int st = 1; st < 32; st <<= 1) {
+        const float other = __shfl_xor_sync(kFull, x, st);
+        x = (lane & st) ? (other - x) : (x + other);
+    }
+#pragma unroll
+    for (int st = 1, buf = 0; st < NW; st <<= 1, buf ^= 1) {
+        xs[buf][w][lane] = x;
         __syncthreads();
-        os[i] = (i & s) ? (other - mine) : (mine + other);
-        __syncthreads();
+        const float other = xs[buf][w ^ st][lane];
+        x = (w & st) ? (other - x) : (x + other);
     }
     // Pi^T = D H / sqrt(d), and the value table carries a factor sqrt(d)
-    a.out[((size_t)b * a.Hq + hq) * D + i] = os[i] * tb.signs[i] * (1.0f / (float)D);
+    a.out[((size_t)b * a.Hq + hq) * D + i] = x * tb.signs[i] * (1.0f / (float)D);
 }
 
 // ---------------------------------------------------------------- split kernel
@@ -809,6 +832,8 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     const size_t units = (size_t)a.Hkv * groups;
 
     fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
+    pdl_trigger();
+    pdl_wait();
     QueryFrags<KK, NT, Tr::QREG> qf;
     qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64,
             reinterpret_cast<uint4*>(body + Tr::BODY_BYTES), tid);
@@ -887,12 +912,8 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     const int c = blockIdx.x;
     const long long G = gridDim.x;
     const int groups = a.plan.groups, upb = a.Hkv * groups;
-    const long long W = a.prefix[a.B];
-    const long long x0 = (long long)c * W / G, x1 = (long long)(c + 1) * W / G;
-    if (x0 >= x1) return;   // an empty range (fewer tiles than CTAs): uniform, before any barrier
-
+    // before the wait: only the constant tables and this CTA's own barriers
     fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
-    const int lim = min(a.max_len, a.capacity);
     const uint32_t lane4 = 4u * lane;
     uint8_t* ring = body + (size_t)w * S * Tr::STAGE_BYTES;
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
@@ -902,6 +923,12 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
         fence_mbar_init();
     }
     __syncwarp();
+    pdl_trigger();
+    pdl_wait();   // the prologue's prefix and query fragments are complete from here on
+    const long long W = a.prefix[a.B];
+    const long long x0 = (long long)c * W / G, x1 = (long long)(c + 1) * W / G;
+    if (x0 >= x1) return;   // an empty range (fewer tiles than CTAs): uniform, before any barrier
+    const int lim = min(a.max_len, a.capacity);
     // Bulk copies this warp has issued / waited for (warp-uniform): copy n uses
     // ring slot n % S and completes phase (n / S) & 1 of that slot's barrier.
     uint32_t issued = 0, consumed = 0;
@@ -1056,6 +1083,24 @@ cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long& done_mask)
     return e;
 }
 
+// Launch with the programmatic-stream-serialization attribute (see pdl_wait).
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       A&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 template <int D, int KB, int VB, int QJ>
 cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool scores, cudaStream_t st)
 {
@@ -1070,26 +1115,24 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
         const size_t smem = 2 * (size_t)TB + 8 * (48 + (size_t)16 * D + (size_t)16 * D);
         auto kern = append_prologue<D, KB, VB, QJ>;
         if ((e = allow_smem(kern, smem, done_append)) != cudaSuccess) return e;
-        kern<<<dim3(units + a.Hkv, a.B), 2 * D, smem, st>>>(tb, a);
+        e = launch_pdl(kern, dim3(units + a.Hkv, a.B), dim3(2 * D), smem, st, tb, a);
     } else {
-        attend_prologue<D><<<dim3(units, a.B), 2 * D, 0, st>>>(tb, a);
+        e = launch_pdl(attend_prologue<D>, dim3(units, a.B), dim3(2 * D), 0, st, tb, a);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (scores) {
         auto kern = attend_scores<D, KB, VB, QJ>;
         if ((e = allow_smem(kern, Tr::DYN_SMEM, done_scores)) != cudaSuccess) return e;
         if (a.plan.tiles > 0)
-            kern<<<dim3(a.plan.nsplit, units, a.B), Tr::NT, Tr::DYN_SMEM, st>>>(tb, a);
-        return cudaGetLastError();
+            e = launch_pdl(kern, dim3(a.plan.nsplit, units, a.B), dim3(Tr::NT), Tr::DYN_SMEM, st, tb, a);
+        return e;
     }
     auto kern = attend_split<D, KB, VB, QJ>;
     if ((e = allow_smem(kern, Tr::DYN_SMEM, done_attend)) != cudaSuccess) return e;
-    if (a.plan.tiles > 0) kern<<<a.plan.ctas, Tr::NT, Tr::DYN_SMEM, st>>>(tb, a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    attend_reduce<D><<<dim3(a.Hq, a.B), D, 0, st>>>(tb, a);
-    return cudaGetLastError();
+    if (a.plan.tiles > 0 &&
+        (e = launch_pdl(kern, dim3(a.plan.ctas), dim3(Tr::NT), Tr::DYN_SMEM, st, tb, a)) != cudaSuccess)
+        return e;
+    return launch_pdl(attend_reduce<D>, dim3(a.Hq, a.B), dim3(D), 0, st, tb, a);
 }
 
 }  // namespace
