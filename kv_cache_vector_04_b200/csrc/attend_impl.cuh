@@ -171,8 +171,8 @@ __device__ __forceinline__ void tile_prefix(const DevTables& tb, const AttendArg
 template <int D>
 __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendArgs& a)
 {
-    constexpr int NT = 2 * D;
-    __shared__ float qt[D][8];          // rotated queries, [coordinate][head]
+    constexpr int NT = 2 * D, VPL = D / 32;
+    __shared__ float qt[D][9];          // rotated queries, [coordinate][head] (padded rows)
     __shared__ float pp[1][D][8];       // p = S q~
     __shared__ float es[8];             // per-head power-of-two scale of q~ for the split
     const int unit = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
@@ -181,39 +181,55 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
     const size_t units = (size_t)a.Hkv * groups;
     if (unit == 0 && b == 0 && tid < 32) tile_prefix(tb, a, tid);
 
-    for (int e = tid; e < 8 * D; e += NT) {
-        const int h = e / D, i = e % D, j = grp * 8 + h;
-        float x = 0.f;
-        if (j < ratio) {
-            const size_t off = ((size_t)b * a.Hq + hkv * ratio + j) * D + i;
-            x = a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[off])
-                         : __half2float(reinterpret_cast<const __half*>(a.q)[off]);
-            x *= tb.signs[i];
-        }
-        qt[i][h] = x;
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int st = 1; st < D; st <<= 1) {            // Walsh-Hadamard butterflies, 8 heads
-        for (int e = tid; e < 4 * D; e += NT) {
-            const int h = e & 7, bf = e >> 3;
-            const int i = (bf / st) * 2 * st + (bf % st);
-            const float x0 = qt[i][h], x1 = qt[i + st][h];
-            qt[i][h] = x0 + x1;
-            qt[i + st][h] = x0 - x1;
-        }
-        __syncthreads();
-    }
-    const float rs = rsqrtf((float)D);
-    for (int e = tid; e < 8 * D; e += NT) (&qt[0][0])[e] *= rs;
-    __syncthreads();
-    // per head a power of two es with max |q~| es in [64, 128): the hi and lo
-    // fp16 parts of q~ es below then stay clear of overflow and of subnormals
+    // One warp per head: lane l holds coordinates i = 32k + l (k < D/32), so the
+    // loads of q are coalesced and the transposed stores to qt hit distinct
+    // banks. Walsh-Hadamard butterflies over the low five index bits run on
+    // shuffles, over the high bits in-lane; then the scale 1/sqrt(d) and the
+    // head's power-of-two split scale es (max |q~| es in [64, 128): the hi and
+    // lo fp16 parts of q~ es below then stay clear of overflow and subnormals).
     {
         const int w = tid >> 5, lane = tid & 31;
+        const float rs = rsqrtf((float)D);
         for (int h = w; h < 8; h += NT / 32) {
+            const int j = grp * 8 + h;
+            float x[VPL];
+#pragma unroll
+            for (int k = 0; k < VPL; ++k) {
+                const int i = 32 * k + lane;
+                x[k] = 0.f;
+                if (j < ratio) {
+                    const size_t off = ((size_t)b * a.Hq + hkv * ratio + j) * D + i;
+                    x[k] = (a.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(a.q)[off])
+                                     : __half2float(reinterpret_cast<const __half*>(a.q)[off])) *
+                           tb.signs[i];
+                }
+            }
+#pragma unroll
+            for (int st = 1; st < 32; st <<= 1) {
+#pragma unroll
+                for (int k = 0; k < VPL; ++k) {
+                    const float o = __shfl_xor_sync(kFull, x[k], st);
+                    x[k] = (lane & st) ? (o - x[k]) : (x[k] + o);
+                }
+            }
+#pragma unroll
+            for (int st = 1; st < VPL; st <<= 1) {
+#pragma unroll
+                for (int k = 0; k < VPL; ++k) {
+                    if (!(k & st)) {
+                        const float x0 = x[k], x1 = x[k + st];
+                        x[k] = x0 + x1;
+                        x[k + st] = x0 - x1;
+                    }
+                }
+            }
             float mx = 0.f;
-            for (int c = lane; c < D; c += 32) mx = fmaxf(mx, fabsf(qt[c][h]));
+#pragma unroll
+            for (int k = 0; k < VPL; ++k) {
+                x[k] *= rs;
+                mx = fmaxf(mx, fabsf(x[k]));
+                qt[32 * k + lane][h] = x[k];
+            }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
             if (lane == 0) es[h] = (mx > 0.f && mx < 3.0e38f) ? exp2f((float)(6 - ilogbf(mx))) : 1.f;
@@ -430,12 +446,24 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
         double z[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0.0;
+        if (T == 1) {   // the decode step: one key, four independent partial sums
+            double z1 = 0.0, z2 = 0.0, z3 = 0.0;
+#pragma unroll 4
+            for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); c += 4) {
+                z[0] = fma((double)__ldg(tb.s_t + (size_t)c * M + j), rk[c], z[0]);
+                z1 = fma((double)__ldg(tb.s_t + (size_t)(c + 1) * M + j), rk[c + 1], z1);
+                z2 = fma((double)__ldg(tb.s_t + (size_t)(c + 2) * M + j), rk[c + 2], z2);
+                z3 = fma((double)__ldg(tb.s_t + (size_t)(c + 3) * M + j), rk[c + 3], z3);
+            }
+            z[0] = (z[0] + z1) + (z2 + z3);
+        } else {
 #pragma unroll 16
-        for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); ++c) {
-            const double sv = (double)__ldg(tb.s_t + (size_t)c * M + j);
+            for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); ++c) {
+                const double sv = (double)__ldg(tb.s_t + (size_t)c * M + j);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i < T) z[i] = fma(sv, rk[i * D + c], z[i]);
+                for (int i = 0; i < 16; ++i)
+                    if (i < T) z[i] = fma(sv, rk[i * D + c], z[i]);
+            }
         }
         if (hf == 1) {
 #pragma unroll
