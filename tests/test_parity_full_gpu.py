@@ -21,7 +21,7 @@ from tests import parity as P
 pytestmark = pytest.mark.gpu
 
 
-def _run_layer(w, samples, seq_fn=None):
+def _run_layer(w, samples, seq_fn=None, decode_step=False):
     """Quantize + attend one layer of workload `w` on the GPU, then check the
     sampled (b, kv head) streams against the oracle."""
     torch.cuda.set_device(0)
@@ -29,7 +29,7 @@ def _run_layer(w, samples, seq_fn=None):
     ctx = tq.tq_init(w.d, w.bits, 1)
     tab = O.Tables(w.d, w.bits, 1)
     k, v = inputs.kv_pair(w, w.N, layer=0, device=dev)
-    cache = tq.new_cache(ctx, w.B, w.Hkv, w.N)
+    cache = tq.new_cache(ctx, w.B, w.Hkv, w.N + (16 if decode_step else 0))
     tq.tq_quantize(ctx, k, v, torch.zeros(w.B, dtype=torch.int32, device=dev), cache)
     assert tq.tq_status(ctx) == 0
     host = cache.data.cpu().numpy()
@@ -50,9 +50,42 @@ def _run_layer(w, samples, seq_fn=None):
     stats.check()
     del k, v
     q = inputs.queries(w, device=dev)
-    seq = torch.full((w.B,), w.N, dtype=torch.int32) if seq_fn is None else seq_fn(w)
-    out = tq.tq_attend(ctx, q, cache, seq.to(dev), w.N).cpu().numpy().astype(np.float64)
-    assert tq.tq_status(ctx) == 0
+    if decode_step:
+        # the bench's step: tq_append_attend of one new token per sequence at
+        # position N, captured in a CUDA graph and replayed
+        nk, nv = inputs.kv_pair(w, 1, layer=10_000, device=dev)
+        start = torch.full((w.B,), w.N, dtype=torch.int32, device=dev)
+        seq = torch.full((w.B,), w.N + 1, dtype=torch.int32)
+        ws = tq.new_workspace(ctx, w.B, w.Hq, w.Hkv, w.N + 1)
+        outd = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+        seqd = seq.to(dev)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            tq.tq_append_attend(ctx, q, nk, nv, start, cache, seqd, w.N + 1, out=outd, workspace=ws)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            tq.tq_append_attend(ctx, q, nk, nv, start, cache, seqd, w.N + 1, out=outd, workspace=ws)
+        outd.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        out = outd.cpu().numpy().astype(np.float64)
+        del graph
+        assert tq.tq_status(ctx) == 0
+        host = cache.data.cpu().numpy()
+        for (b, h) in samples:
+            new = O.quantize(tab, nk[b, h].cpu().numpy(), nv[b, h].cpu().numpy())
+            sb = P.stream_bytes(host, lay["tile_bytes"], cache.capacity, w.Hkv, b, h, w.N + 1)
+            gpu = O.unpack_stream(w.d, tab, w.N + 1, sb)
+            P.compare_stream(tab, {kk: vv[w.N:] for kk, vv in gpu.items()}, new, 1, stats)
+            ora = oracle_streams[(b, h)]
+            oracle_streams[(b, h)] = {kk: np.concatenate([ora[kk], new[kk]]) for kk in ora}
+        stats.check()
+    else:
+        seq = torch.full((w.B,), w.N, dtype=torch.int32) if seq_fn is None else seq_fn(w)
+        out = tq.tq_attend(ctx, q, cache, seq.to(dev), w.N).cpu().numpy().astype(np.float64)
+        assert tq.tq_status(ctx) == 0
     qbits_all = P.q_bits(q.cpu())
     for (b, h) in samples:
         ora = oracle_streams[(b, h)]
@@ -71,6 +104,12 @@ def test_llama70b_shaped_layer_32k():
     # 16 sequences x 8 kv heads x 32768 tokens, K 3-bit + QJL, V 4-bit; 64 query heads
     w = inputs.WORKLOADS["llama3.3-70b_decode_32k"]
     _run_layer(w, samples=[(0, 0), (15, 7), (9, 3)])
+
+
+def test_llama70b_shaped_decode_step_in_a_cuda_graph():
+    # the benchmarked path: one tq_append_attend per layer, replayed from a graph
+    w = inputs.WORKLOADS["llama3.3-70b_decode_32k"]
+    _run_layer(w, samples=[(3, 1), (12, 6)], decode_step=True)
 
 
 def test_qwen32b_shaped_layer_128k():
