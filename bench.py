@@ -55,45 +55,60 @@ def parse_args(argv=None):
 # ---------------------------------------------------------------- plumbing
 
 class Dist:
+    """One process per GPU (torchrun env); the ranks run independent replicas of
+    the workload (weak scaling) and meet only to take the max of their step
+    times and the sum of their bytes. backend "nccl" on GPUs, "gloo" on CPU."""
+
     def __init__(self):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = None
 
     def init(self, backend="nccl"):
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(self.local_rank)
+        if backend == "nccl":
+            torch.cuda.set_device(self.local_rank)
+            self.device = torch.device("cuda", self.local_rank)
+        else:
+            self.device = torch.device("cpu")
         if self.world > 1:
             from datetime import timedelta
-            dist.init_process_group(backend, timeout=timedelta(seconds=600),
-                                    device_id=torch.device("cuda", self.local_rank))
+            kw = {"timeout": timedelta(seconds=600)}
+            if backend == "nccl":
+                kw["device_id"] = self.device
+            dist.init_process_group(backend, **kw)
             self.pg = dist
 
     def barrier(self):
         if self.pg:
             self.pg.barrier()
 
-    def max(self, x: float) -> float:
+    def _reduce(self, x: float, op) -> float:
         if not self.pg:
             return x
         import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=op)
         return float(t.item())
 
+    def max(self, x: float) -> float:
+        return self._reduce(x, self.pg.ReduceOp.MAX if self.pg else None)
+
     def sum(self, x: float) -> float:
-        if not self.pg:
-            return x
-        import torch
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        self.pg.all_reduce(t)
-        return float(t.item())
+        return self._reduce(x, self.pg.ReduceOp.SUM if self.pg else None)
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def whole_job_gbs(total_bytes: float, ms_max: float) -> float:
+    """Whole-job throughput: the bytes every rank processed in one step, over
+    the slowest rank's step time (ms)."""
+    return total_bytes / (ms_max / 1e3) / 1e9
 
 
 class ClockSampler:
@@ -356,7 +371,7 @@ def run_tq(args, dist: Dist):
     bytes_step = layers * w.B * w.Hkv * (N + 1) * per_tok
     bytes_attend = w.B * w.Hkv * (N + 1) * per_tok
     total_bytes = dist.sum(bytes_step)
-    value = total_bytes / (ms / 1e3) / 1e9
+    value = whole_job_gbs(total_bytes, ms)
     peak, peak_kind = measured_peaks()
     achieved = bytes_attend / (attend_ms / 1e3) / 1e9
 
