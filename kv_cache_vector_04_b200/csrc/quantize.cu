@@ -116,10 +116,32 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
     // ---------------- 1. normalise, rotate, encode (fp64) ----------------
     unsigned sat = 0u;
     const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    // The 8 vectors of this warp are processed one by one; the fp16 data of the
+    // next one is loaded while the current one is rotated (software pipeline).
+    auto load_vec = [&](int it, uint32_t (&raw)[VPL / 2]) {
+        const int n = w + 4 * (it & 3);
+#pragma unroll
+        for (int k = 0; k < VPL / 2; ++k) raw[k] = 0u;
+        if (n < lo_slot || n >= hi_slot) return;
+        const size_t row = (((size_t)b * a.Hkv + h) * (size_t)a.T + (size_t)(first + n - start)) * D;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>((it < 4 ? a.k : a.v) + row + lane * VPL);
+#pragma unroll
+        for (int k = 0; k < VPL / 2; ++k) raw[k] = __ldg(src + k);
+    };
+    uint32_t cur[VPL / 2];
+    load_vec(0, cur);
 #pragma unroll 1
     for (int it = 0; it < 8; ++it) {
         const int n = w + 4 * (it & 3);
         const bool is_key = it < 4;
+        uint32_t nxt[VPL / 2];
+        if (it < 7) load_vec(it + 1, nxt);
+        uint32_t raw[VPL / 2];
+#pragma unroll
+        for (int k = 0; k < VPL / 2; ++k) {
+            raw[k] = cur[k];
+            cur[k] = nxt[k];
+        }
         if (n < lo_slot || n >= hi_slot) {
             if (QJ && is_key) {
 #pragma unroll
@@ -131,24 +153,12 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
             }
             continue;
         }
-        const size_t row = (((size_t)b * a.Hkv + h) * (size_t)a.T + (size_t)(first + n - start)) * D;
-        const __half* src = (is_key ? a.k : a.v) + row + lane * VPL;
         double x[VPL];
-        if constexpr (VPL == 2) {
-            const __half2 p = *reinterpret_cast<const __half2*>(src);
-            x[0] = (double)__low2float(p);
-            x[1] = (double)__high2float(p);
-        } else {
 #pragma unroll
-            for (int k = 0; k < VPL; k += 4) {
-                const uint2 u = *reinterpret_cast<const uint2*>(src + k);
-                const __half2 p0 = *reinterpret_cast<const __half2*>(&u.x);
-                const __half2 p1 = *reinterpret_cast<const __half2*>(&u.y);
-                x[k] = (double)__low2float(p0);
-                x[k + 1] = (double)__high2float(p0);
-                x[k + 2] = (double)__low2float(p1);
-                x[k + 3] = (double)__high2float(p1);
-            }
+        for (int k = 0; k < VPL / 2; ++k) {
+            const __half2 p = *reinterpret_cast<const __half2*>(&raw[k]);
+            x[2 * k] = (double)__low2float(p);
+            x[2 * k + 1] = (double)__high2float(p);
         }
         double ss = 0.0;
 #pragma unroll
