@@ -14,16 +14,17 @@
 //  prologue  q~ = H (D o q) / sqrt(d) and p = S q~ per group of 8 query heads,
 //            written as fp16 m16n8k16 B fragments (hi/lo; log2(e) and the
 //            norms' scales folded in);
-//  split     one CTA per (batch, kv head, group of 8 query heads, context
-//            split); each warp streams 16-token tiles with 128-bit loads of its
-//            own lane string, decodes codes to fp16 tensor-core A fragments
+//  split     stream-K over the tiles of all (batch, kv head, group of 8 query
+//            heads) units, one CTA per SM; each warp streams 16-token tiles
+//            through a ring of whole-tile bulk copies, reads its own lane
+//            string of each, decodes codes to fp16 tensor-core A fragments
 //            through a lane-replicated shared-memory table (2 ALU ops + 1 LDS
 //            per fp16x2) and sign pairs with 2 ALU ops, and runs
 //              logits: [16 tok x d] x [d x 8 heads]  (codebook term)
 //                      [16 tok x m] x [m x 8 heads]  (QJL sign term)
 //              PV:     [d x 16 tok] x [16 tok x 8 heads]
 //            on mma.sync with fp32 accumulation, with an online softmax per
-//            head in registers; the 8 warps of a CTA merge in shared memory;
+//            head in registers; the warps of a CTA merge in shared memory;
 //  reduce    merges the splits per query head and applies Pi^T (fp32 WHT).
 // Operands come from registers because every A fragment is decoded on the
 // fly; the contraction is skinny (N = 8 heads), so the legacy register-fed
@@ -70,27 +71,31 @@ struct AttTraits {
     static constexpr int TILE_BYTES = CODE_BYTES + KNB + 32;
     static constexpr size_t LUT_BYTES = (size_t)(NLK + NLV) * 128;
     static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
-    // d <= 128: CTAs of 4 warps with the query fragments in registers;
-    // d = 256: CTAs of 8 warps, 1 per SM, query fragments in shared memory
-    static constexpr bool QREG = D <= 128;
-    static constexpr int WARPS = QREG ? 4 : 8, NT = 32 * WARPS;
+    // One CTA of 16 warps per SM, 128 registers a thread: the kernel is
+    // issue-bound, so warps to hide latency are worth more than registers; the
+    // query fragments are read from shared memory. (Measured against 3 CTAs of
+    // 4 warps with the fragments in registers at d <= 128, 8 warps at d = 256,
+    // and 20 or 24 warps at d = 64: 16 warps was the fastest at every d.)
+    static constexpr int WARPS = 16, NT = 32 * WARPS;
     static constexpr size_t MERGE_BYTES = (size_t)WARPS * 8 * (D + 2) * 4;
-    // staging ring: per warp STAGES images of whole tiles, each brought in by
-    // one bulk copy
-    static constexpr int STAGES = 3;
-    static constexpr int STAGE_BYTES = TILE_BYTES;
-    static constexpr size_t RING_BYTES = (size_t)WARPS * STAGES * STAGE_BYTES;
-    static constexpr size_t QF_SMEM = QREG ? 0 : QF_BYTES;
-    // dynamic shared memory: [K table][V table] (unless static), [ring, then the
-    // merge buffer], [query fragments]
-    static constexpr size_t BODY_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
+    static constexpr size_t QF_SMEM = QF_BYTES;
     // The decode tables are static shared arrays when they fit there (the
     // table loads then take their base as an immediate), else the front of
     // dynamic shared memory (4-bit keys with 4-bit values: 64 KB).
     static constexpr bool STATIC_LUT = LUT_BYTES <= 40 * 1024;
+    // staging ring: per warp STAGES images of whole tiles, each brought in by
+    // one bulk copy; 3 stages where they fit in shared memory, else 2
+    static constexpr size_t SMEM_CAP = 227u * 1024u - 1024u;
+    static constexpr int STAGES =
+        LUT_BYTES + (size_t)WARPS * 3 * TILE_BYTES + QF_SMEM <= SMEM_CAP ? 3 : 2;
+    static constexpr int STAGE_BYTES = TILE_BYTES;
+    static constexpr size_t RING_BYTES = (size_t)WARPS * STAGES * STAGE_BYTES;
+    // dynamic shared memory: [K table][V table] (unless static), [ring, then the
+    // merge buffer], [query fragments]
+    static constexpr size_t BODY_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
     static constexpr size_t DYN_SMEM = (STATIC_LUT ? 0 : LUT_BYTES) + BODY_BYTES + QF_SMEM;
-    static constexpr int SMEM_FIT = (int)((228u * 1024u) / (LUT_BYTES + BODY_BYTES + QF_SMEM + 2048u));
-    static constexpr int CTAS_PER_SM = QREG ? (SMEM_FIT < 3 ? SMEM_FIT : 3) : 1;
+    static_assert(LUT_BYTES + BODY_BYTES + QF_SMEM <= SMEM_CAP, "split CTA exceeds shared memory");
+    static constexpr int CTAS_PER_SM = 1;
 };
 
 // Offset, inside a lane-replicated table, of the entry selected by the F-bit
@@ -674,29 +679,10 @@ __device__ __forceinline__ void read_stage(const uint8_t* slot, int lane, TileDa
 }
 
 // Query B fragments of one k-step: x,y = hi (b0, b1), z,w = lo, for the
-// codebook term (c) and the QJL term (s). Held in registers (they do not
-// change from tile to tile) or, where registers are short, in shared memory.
-template <int KK, int NT, bool IN_REGS>
-struct QueryFrags;
-
+// codebook term (c) and the QJL term (s), copied once per unit into shared
+// memory and read from there by every tile (registers go to warps instead).
 template <int KK, int NT>
-struct QueryFrags<KK, NT, true> {
-    uint4 c[KK], s[KK];
-    __device__ __forceinline__ void load(const uint4* src, uint4*, int tid)
-    {
-        const int lane = tid & 31;
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) {
-            c[kk] = src[kk * 64 + lane];
-            s[kk] = src[kk * 64 + 32 + lane];
-        }
-    }
-    __device__ __forceinline__ uint4 fc(int kk, int) const { return c[kk]; }
-    __device__ __forceinline__ uint4 fs(int kk, int) const { return s[kk]; }
-};
-
-template <int KK, int NT>
-struct QueryFrags<KK, NT, false> {
+struct QueryFrags {
     const uint4* sm;
     __device__ __forceinline__ void load(const uint4* src, uint4* smem, int tid)
     {
@@ -862,7 +848,7 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
     pdl_trigger();
     pdl_wait();
-    QueryFrags<KK, NT, Tr::QREG> qf;
+    QueryFrags<KK, NT> qf;
     qf.load(reinterpret_cast<const uint4*>(a.qfrag) + ((size_t)b * units + unit) * KK * 64,
             reinterpret_cast<uint4*>(body + Tr::BODY_BYTES), tid);
     const int seq = min(max(a.seq_len[b], 0), min(a.max_len, a.capacity));
@@ -900,8 +886,8 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
 // query heads) units, laid end to end (sequence b's units start at
 // prefix[b]), are cut into gridDim.x equal contiguous ranges, one per CTA, so
 // that one wave of CTAs does equal work whatever the lengths. A CTA walks its
-// range unit by unit; for each piece (segment) its 8 warps stream the tiles
-// round-robin through a per-warp cp.async ring, merge in shared memory and
+// range unit by unit; for each piece (segment) its warps stream the tiles
+// round-robin through per-warp rings of bulk copies, merge in shared memory and
 // write one partial (m, l, acc per head) to slot CTA + unit, a slot no other
 // segment uses: along the tile order both the CTA index and the unit index
 // are non-decreasing and every new segment raises at least one of them.
@@ -961,7 +947,7 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     // ring slot n % S and completes phase (n / S) & 1 of that slot's barrier.
     uint32_t issued = 0, consumed = 0;
     bool stalled = false;   // a wait ran out: no further copies, tiles skipped
-    QueryFrags<KK, NT, Tr::QREG> qf;
+    QueryFrags<KK, NT> qf;
 
     // Each segment re-locates its unit from x, so that only x, x1 and the
     // partial slot stay live across the tile loop.
