@@ -110,6 +110,13 @@ typedef struct {
  *        at B_K*d/2 + 32*(p/16) + 16e + (p%16)  (1 = S r >= 0);
  *      V code of token 2t + 8(r>>1) + e, coordinate 16kk + g + 8(r&1):
  *        B_V bits at (B_K+qjl)*d/2 + 2*B_V*p + e*B_V.
+ *    Format (3, 4, 1) (TurboQuant at 4 bits) instead keeps each key pair and
+ *    two sign bits in one byte: the K code at 8p + 3e (bits 0..5 of byte p),
+ *    the sign at 32*(p/4) + 16e + a, a = 6, 7, 14, 15 for p%4 = 0, 1, 2, 3
+ *    (bits 6 and 7 of the bytes of word p/4); its V codes as above. With
+ *    4-bit value cells every V pair is one byte, and with (4, 4, 0) every K
+ *    pair too: the decoder turns such a byte into its table row with one
+ *    byte permute.
  *    (Lane l's bits are exactly the operands that lane l of a warp needs for
  *    the m16n8k16 tensor-core fragments of the attention kernel, so each lane
  *    streams its own bytes with 128-bit coalesced loads.)

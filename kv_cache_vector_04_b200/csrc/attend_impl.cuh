@@ -69,7 +69,20 @@ struct AttTraits {
     static constexpr int CODE_BYTES = 2 * W * D;             // code region of a tile
     static constexpr int KNB = 32 + 32 * QJ;                 // K norm bytes of a tile
     static constexpr int TILE_BYTES = CODE_BYTES + KNB + 32;
-    static constexpr size_t LUT_BYTES = (size_t)(NLK + NLV) * 128;
+    // Byte fields: an 8-bit field that starts on a byte of the lane string (a
+    // pair of 4-bit cells, or the 6-bit pair of 3-bit keys in the low bits of
+    // a byte whose top bits hold two QJL signs) is turned into its table
+    // offset, row * 256 + 4 * lane, by one byte permute. Such formats keep one
+    // table of 256 rows of 256 bytes: the key entry, then the value entry.
+    static constexpr bool PK = KB + QJ == 4;                 // keys: (3,4,1), (4,4,0)
+    static_assert(!PK || !QJ || TileLayout<D, KB, VB, QJ>::KS_BYTES, "key bytes carry the signs");
+    static constexpr bool PV = VB == 4;                      // values: (3,4,1), (4,4,0), (3,4,0)
+    static constexpr bool ROWS = PV;
+    static constexpr int LSH = ROWS ? 8 : 7;                 // log2 of a table entry's stride
+    static constexpr int VW0 = VBIT0 / 32;                   // first value word (byte fields)
+    static_assert(!PK || ROWS, "byte-field keys come with byte-field values");
+    static_assert(!PV || VBIT0 % 32 == 0, "byte-field values start on a word");
+    static constexpr size_t LUT_BYTES = ROWS ? (size_t)256 * 256 : (size_t)(NLK + NLV) * 128;
     static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
     // One CTA of 16 warps per SM, 128 registers a thread: the kernel is
     // issue-bound, so warps to hide latency are worth more than registers; the
@@ -98,23 +111,32 @@ struct AttTraits {
     static constexpr int CTAS_PER_SM = 1;
 };
 
-// Offset, inside a lane-replicated table, of the entry selected by the F-bit
-// field at bit `pos` of the lane string: field * 128 + 4 * lane, built with one
-// funnel (or plain) shift and one LOP3 (lane4 = 4 * lane occupies bits 2..6,
-// the field bits 7 and up). The table's own shared address is added by the
-// load as an immediate, so no alignment of the table is assumed: shared
-// memory does not start at address 0 of the window, and declared alignments
-// above 1 KB are not honoured there.
+// Offset, inside a lane-replicated table of stride 2^SH bytes, of the entry
+// selected by the F-bit field at bit `pos` of the lane string:
+// field * 2^SH + 4 * lane, built with one funnel (or plain) shift and one LOP3
+// (lane4 = 4 * lane occupies bits 2..6, the field bits SH and up). The
+// table's own shared address is added by the load as an immediate, so no
+// alignment of the table is assumed: shared memory does not start at address
+// 0 of the window, and declared alignments above 1 KB are not honoured there.
+template <int SH>
 __device__ __forceinline__ uint32_t lut_off(const uint32_t* s, int pos, int F, uint32_t lane4)
 {
     const int wi = pos >> 5, o = pos & 31;
-    const uint32_t mask = ((1u << F) - 1u) << 7;
+    const uint32_t mask = ((1u << F) - 1u) << SH;
     uint32_t v;
     if (o + F <= 32)
-        v = (o >= 7) ? (s[wi] >> (o - 7)) : (s[wi] << (7 - o));
+        v = (o >= SH) ? (s[wi] >> (o - SH)) : (s[wi] << (SH - o));
     else
-        v = __funnelshift_r(s[wi], s[wi + 1], o - 7);
+        v = __funnelshift_r(s[wi], s[wi + 1], o - SH);
     return (v & mask) | lane4;
+}
+
+// Offset of the row selected by byte r (0..3) of word w in a table of 256-byte
+// rows: w.byte[r] * 256 + 4 * lane, one byte permute (lane4 < 256 supplies
+// byte 0 and the zero bytes 2, 3).
+__device__ __forceinline__ uint32_t row_off(uint32_t w, int r, uint32_t lane4)
+{
+    return __byte_perm(w, lane4, 0x5504u | ((uint32_t)r << 4));
 }
 
 __device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t byte_off)
@@ -130,6 +152,14 @@ __device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q, uint32_t nrh
 {
     const uint32_t x = word << (15 - q);
     return (x & 0x80008000u) ^ nrho2;
+}
+
+// Byte-field keys with QJL: the sign pair of key pair r of a k-step sits in
+// that k-step's key word at bits a and a + 16, a = 6 + (r & 1) + 8 (r >> 1)
+// (the top two bits of each byte; for r = 3 no shift is needed).
+__device__ __forceinline__ uint32_t sign_pair_byte(uint32_t word, int r, uint32_t nrho2)
+{
+    return sign_pair(word, 6 + (r & 1) + 8 * (r >> 1), nrho2);
 }
 
 // ---------------------------------------------------------------- prologue
@@ -350,7 +380,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
     constexpr int BK = KB, BV = VB;
     constexpr int TB = Tr::TILE_BYTES;
     constexpr int CB = Tr::CB;
-    constexpr int SB0 = BK * D / 2, VB0 = Tr::VBIT0;          // first sign / value bit of a string
+    using Lay = TileLayout<D, KB, VB, QJ>;                     // field bits of a lane string
     constexpr int NB = Tr::CODE_BYTES;                        // first norm byte of a tile
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int T = a.T, start = a.start_pos[b];
@@ -414,7 +444,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
                 // K field: token g + 8 (r & 1), coordinate 16 kk + 8 (r >> 1) + 2 t + e
                 const int kk = c >> 4, t = (c & 7) >> 1, e = c & 1;
                 const int p = 4 * kk + 2 * ((c & 15) >> 3) + half;
-                put_field<CB>(tw, 4 * g + t, 2 * BK * p + e * BK, (uint32_t)idx, BK);
+                put_field<CB>(tw, 4 * g + t, Lay::kbit(p, e), (uint32_t)idx, BK);
             }
             if constexpr (QJ) {
                 rr = warp_sum(rr);
@@ -435,7 +465,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
                 // V field: token 2 t + 8 (r >> 1) + e, coordinate 16 kk + g' + 8 (r & 1)
                 const int kk = c >> 4, gc = c & 7, t = (tau & 7) >> 1, e = tau & 1;
                 const int p = 4 * kk + 2 * half + ((c & 15) >> 3);
-                put_field<CB>(tw, 4 * gc + t, VB0 + 2 * BV * p + e * BV, (uint32_t)idx, BV);
+                put_field<CB>(tw, 4 * gc + t, Lay::vbit(p, e), (uint32_t)idx, BV);
             }
             if (lane == 0)
                 *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(tw) + NB + Tr::KNB + 4 * g + 2 * half) =
@@ -483,8 +513,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
                 if (i >= T) break;
                 const int n = start + i, tau = n & 15;
                 const int p = 4 * kk + 2 * ((j & 15) >> 3) + (tau >> 3);
-                put_field<CB>(img + (n / 16 - t0) * (TB / 4), 4 * (tau & 7) + t,
-                              SB0 + 32 * (p >> 4) + 16 * e + (p & 15),
+                put_field<CB>(img + (n / 16 - t0) * (TB / 4), 4 * (tau & 7) + t, Lay::sbit(p, e),
                               z[i] + zp[i * M + j] >= 0.0 ? 1u : 0u, 1);
             }
         }
@@ -718,9 +747,14 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int p = 4 * kk + r;
-            ak[r] = lut_load(lutk, lut_off(td.s, Tr::KF * p, Tr::KF, lane4));
-            if constexpr (QJ)
-                as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
+            if constexpr (Tr::PK) {
+                ak[r] = lut_load(lutk, row_off(td.s[kk], r, lane4));
+                if constexpr (QJ) as[r] = sign_pair_byte(td.s[kk], r, (r & 1) ? nr_h : nr_g);
+            } else {
+                ak[r] = lut_load(lutk, lut_off<Tr::LSH>(td.s, Tr::KF * p, Tr::KF, lane4));
+                if constexpr (QJ)
+                    as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
+            }
         }
         if (kk == 0) {
             mma_16816_first(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
@@ -798,7 +832,9 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, KB, VB, QJ>& t
         uint32_t av[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
-            av[r] = lut_load(lutv, lut_off(td.s, Tr::VBIT0 + Tr::VF * (4 * kk + r), Tr::VF, lane4));
+            av[r] = Tr::PV ? lut_load(lutv, row_off(td.s[Tr::VW0 + kk], r, lane4))
+                           : lut_load(lutv, lut_off<Tr::LSH>(td.s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
+                                                             Tr::VF, lane4));
         mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0, b1);
     }
 }
@@ -808,8 +844,20 @@ template <int D, int KB, int VB, int QJ, int NT>
 __device__ __forceinline__ void fill_luts(const DevTables& tb, uint32_t* lutk, uint32_t* lutv, int tid)
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    for (int e = tid; e < Tr::NLK * 32; e += NT) lutk[e] = __ldg(tb.lut_k + (e >> 5));
-    for (int e = tid; e < Tr::NLV * 32; e += NT) lutv[e] = __ldg(tb.lut_v + (e >> 5));
+    if constexpr (Tr::ROWS) {
+        // row x: the key entry (key pair x & (NLK - 1): byte-field keys ignore
+        // the sign bits above it), then the value entry x; 64 words a row
+        for (int e = tid; e < 256 * 64; e += NT) {
+            const int x = e >> 6;
+            uint32_t v;
+            if ((e & 63) >= 32) v = __ldg(tb.lut_v + x);
+            else v = (Tr::PK || x < Tr::NLK) ? __ldg(tb.lut_k + (x & (Tr::NLK - 1))) : 0u;
+            lutk[e] = v;
+        }
+    } else {
+        for (int e = tid; e < Tr::NLK * 32; e += NT) lutk[e] = __ldg(tb.lut_k + (e >> 5));
+        for (int e = tid; e < Tr::NLV * 32; e += NT) lutv[e] = __ldg(tb.lut_v + (e >> 5));
+    }
 }
 
 // Estimated logits alone: one CTA per (batch, kv head, group of 8 query heads,
@@ -834,7 +882,7 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
         body = reinterpret_cast<uint8_t*>(dyn_smem);
     } else {
         lutk = reinterpret_cast<uint32_t*>(dyn_smem);
-        lutv = lutk + Tr::NLK * 32;
+        lutv = lutk + (Tr::ROWS ? 32 : Tr::NLK * 32);
         body = reinterpret_cast<uint8_t*>(dyn_smem) + Tr::LUT_BYTES;
     }
 
@@ -915,7 +963,7 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
         body = reinterpret_cast<uint8_t*>(dyn_smem);
     } else {
         lutk = reinterpret_cast<uint32_t*>(dyn_smem);
-        lutv = lutk + Tr::NLK * 32;
+        lutv = lutk + (Tr::ROWS ? 32 : Tr::NLK * 32);
         body = reinterpret_cast<uint8_t*>(dyn_smem) + Tr::LUT_BYTES;
     }
     float* mrg = reinterpret_cast<float*>(body);            // [WARPS][8][D+2] after a segment

@@ -10,6 +10,36 @@ namespace tq {
 
 constexpr unsigned kFull = 0xffffffffu;
 
+// Bit positions inside a lane string of the packed tile format (B_K, B_V, qjl)
+// at head dim D (include/tq.h): for pair slot p (k-step p / 4, fragment
+// register p % 4) and element e in {0, 1},
+//   key cell:    kbit(p, e), B_K bits;   QJL sign: sbit(p, e), 1 bit;
+//   value cell:  vbit(p, e), B_V bits.
+// Generic layout: key pairs packed at 2 B_K bits a pair, then the sign words
+// (pair p at bits p % 16 and 16 + p % 16 of sign word p / 16), then the value
+// pairs. With 3-bit keys and QJL ((3, 4, 1)) a key pair and its two signs fill
+// one byte each: key pair p in the low 6 bits of byte p, the sign pairs of
+// word w at bits a and a + 16 for a = 6, 7, 14, 15 (pairs 4w .. 4w + 3), so
+// the decoder finds a key pair's table row with one byte permute and a sign
+// pair with one shift. With 4-bit cells the generic layout is byte-aligned
+// already.
+template <int D, int KB, int VB, int QJ>
+struct TileLayout {
+    static constexpr bool KS_BYTES = QJ == 1 && KB == 3;
+    static constexpr int SB0 = KB * D / 2;                   // first sign bit (generic)
+    static constexpr int VB0 = (KB + QJ) * D / 2;            // first value bit
+    __host__ __device__ static constexpr int kbit(int p, int e)
+    {
+        return (KS_BYTES ? 8 : 2 * KB) * p + e * KB;
+    }
+    __host__ __device__ static constexpr int sbit(int p, int e)
+    {
+        return KS_BYTES ? 32 * (p >> 2) + 16 * e + 6 + (p & 1) + 8 * ((p >> 1) & 1)
+                        : SB0 + 32 * (p >> 4) + 16 * e + (p & 15);
+    }
+    __host__ __device__ static constexpr int vbit(int p, int e) { return VB0 + 2 * VB * p + e * VB; }
+};
+
 // Device copies of one context's tables (all pointers into one allocation).
 struct DevTables {
     const float* centroids_k;   // [2^BK] fp32

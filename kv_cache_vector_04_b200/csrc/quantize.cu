@@ -281,7 +281,23 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
             for (int q = 0; q < Tr::CW; ++q) {
                 const int wi = c * Tr::CW + q;
                 uint32_t val = 0u, msk = 0u;
-                if (wi < Tr::SBW) {                      // key cell fields
+                using Lay = TileLayout<D, BK, BV, QJ>;
+                if (Lay::KS_BYTES && wi < Tr::VBW) {      // key pairs 4 wi + j with their signs
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int p = 4 * wi + j, kk = wi;
+                        const int tok = gL + 8 * (j & 1);
+                        const int i0 = 16 * kk + 8 * (j >> 1) + 2 * tL;
+                        constexpr uint32_t cm = (1u << BK) - 1u;
+                        const uint32_t f = ((uint32_t)kc[tok][i0] & cm) |
+                                           (((uint32_t)kc[tok][i0 + 1] & cm) << BK);
+                        const uint32_t bits = (sg[tok][i0 >> 5] >> (i0 & 31)) & 3u;
+                        const int a0 = Lay::sbit(p, 0) - 32 * wi, a1 = Lay::sbit(p, 1) - 32 * wi;
+                        const int o = Lay::kbit(p, 0) - 32 * wi;
+                        val |= (f << o) | ((bits & 1u) << a0) | ((bits >> 1) << a1);
+                        if (is_new(tok)) msk |= (((1u << Tr::KF) - 1u) << o) | (1u << a0) | (1u << a1);
+                    }
+                } else if (wi < Tr::SBW) {               // key cell fields
                     const int bit0 = 32 * wi;
                     for (int p = bit0 / Tr::KF; p <= (bit0 + 31) / Tr::KF; ++p) {
                         const int kk = p >> 2, r = p & 3;

@@ -510,6 +510,10 @@ void oracle_quantize_values(int d, int N, const uint16_t* x, const int8_t* D,
 /*        at bit B_K*d/2 + 32*(p/16) + 16e + (p%16);                          */
 /*   V code of token 2t + 8(r>>1) + e, coordinate 16kk + g + 8(r&1),          */
 /*        B_V bits at bit (B_K+qjl)*d/2 + 2*B_V*p + e*B_V.                    */
+/* Except for (3, 4, 1), whose key pair and two signs share a byte: the K     */
+/* code at bit 8p + 3e (the low 6 bits of byte p), the sign at bit            */
+/* 32*(p/4) + 16e + a with a = 6, 7, 14, 15 for p%4 = 0, 1, 2, 3 (the top     */
+/* two bits of the bytes of word p/4); the V codes as above.                  */
 /* The TurboQuant format at b bits is (b-1, b, 1): tiles of 16*(b*d/4 + 6).   */
 /* ------------------------------------------------------------------------- */
 
@@ -550,9 +554,26 @@ static unsigned get_bits(const uint8_t* tile, int C, int lane, int64_t bit, int 
     return v;
 }
 
-/* Sign pair p of a lane: element 0 at bit p%16, element 1 at bit 16 + p%16 of
- * the lane's sign word p/16. */
-static int64_t sign_bit(int p, int e) { return 32LL * (p / 16) + 16 * e + (p % 16); }
+/* Whether format (kb, vb, qjl) keeps each key pair and two sign bits in one
+ * byte. */
+static int key_sign_bytes(int kb, int qjl) { return qjl == 1 && kb == 3; }
+
+/* Lane-string bit of key code (p, e). */
+static int64_t key_bit(int kb, int qjl, int p, int e)
+{
+    if (key_sign_bytes(kb, qjl)) return 8LL * p + 3 * e;
+    return 2LL * kb * p + (int64_t)e * kb;
+}
+
+/* Lane-string bit of sign (p, e). Generic layout: sign pair p of a lane has
+ * element 0 at bit p%16, element 1 at bit 16 + p%16 of the lane's sign word
+ * p/16, after the key codes (sign words start at bit kb*d/2). */
+static int64_t sign_bit(int d, int kb, int qjl, int p, int e)
+{
+    static const int top[4] = {6, 7, 14, 15};
+    if (key_sign_bytes(kb, qjl)) return 32LL * (p / 4) + 16 * e + top[p % 4];
+    return (int64_t)kb * d / 2 + 32LL * (p / 16) + 16 * e + (p % 16);
+}
 
 static void put_half(uint8_t* p, uint16_t h) { p[0] = (uint8_t)(h & 0xff); p[1] = (uint8_t)(h >> 8); }
 static uint16_t get_half(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
@@ -583,7 +604,7 @@ void oracle_pack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* ki
     int64_t TB = oracle_tile_bytes(d, kb, vb, qjl);
     int ntiles = (N + TQO_TILE - 1) / TQO_TILE;
     memset(out, 0, (size_t)(TB * ntiles));
-    int64_t sbase = (int64_t)kb * d / 2, vbase = (int64_t)(kb + qjl) * d / 2;
+    int64_t vbase = (int64_t)(kb + qjl) * d / 2;
     for (int tl = 0; tl < ntiles; ++tl) {
         uint8_t* tile = out + TB * tl;
         for (int lane = 0; lane < 32; ++lane) {
@@ -596,9 +617,9 @@ void oracle_pack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* ki
                     int nv = tl * TQO_TILE + 2 * t + 8 * (r >> 1) + e;
                     int iv = 16 * kk + g + 8 * (r & 1);
                     if (nk < N) {
-                        put_bits(tile, C, lane, 2LL * kb * p + e * kb, kb, kidx[(size_t)nk * d + ik]);
+                        put_bits(tile, C, lane, key_bit(kb, qjl, p, e), kb, kidx[(size_t)nk * d + ik]);
                         if (qjl)
-                            put_bits(tile, C, lane, sbase + sign_bit(p, e), 1,
+                            put_bits(tile, C, lane, sign_bit(d, kb, qjl, p, e), 1,
                                      ksign[(size_t)nk * m + ik]);
                     }
                     if (nv < N)
@@ -628,7 +649,7 @@ void oracle_unpack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* 
     int m = d, C = chunk_bytes(d, kb, vb, qjl);
     int64_t TB = oracle_tile_bytes(d, kb, vb, qjl);
     int ntiles = (N + TQO_TILE - 1) / TQO_TILE;
-    int64_t sbase = (int64_t)kb * d / 2, vbase = (int64_t)(kb + qjl) * d / 2;
+    int64_t vbase = (int64_t)(kb + qjl) * d / 2;
     for (int tl = 0; tl < ntiles; ++tl) {
         const uint8_t* tile = in + TB * tl;
         for (int lane = 0; lane < 32; ++lane) {
@@ -641,9 +662,10 @@ void oracle_unpack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* 
                     int nv = tl * TQO_TILE + 2 * t + 8 * (r >> 1) + e;
                     int iv = 16 * kk + g + 8 * (r & 1);
                     if (nk < N) {
-                        kidx[(size_t)nk * d + ik] = (uint8_t)get_bits(tile, C, lane, 2LL * kb * p + e * kb, kb);
+                        kidx[(size_t)nk * d + ik] =
+                            (uint8_t)get_bits(tile, C, lane, key_bit(kb, qjl, p, e), kb);
                         ksign[(size_t)nk * m + ik] =
-                            (uint8_t)(qjl ? get_bits(tile, C, lane, sbase + sign_bit(p, e), 1) : 0);
+                            (uint8_t)(qjl ? get_bits(tile, C, lane, sign_bit(d, kb, qjl, p, e), 1) : 0);
                     }
                     if (nv < N)
                         vidx[(size_t)nv * d + iv] =

@@ -237,6 +237,44 @@ def test_pack_fields_tile_the_tile(fmt):
     assert np.all(owner >= 0)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_pack_key_sign_bytes_of_3bit_keys(d):
+    # Format (3, 4, 1) keeps each key pair with two sign bits in one byte of a
+    # lane string: every key code lies in bits 0..5 of a byte, every sign in
+    # bit 6 or 7 of a byte of the same region, and the two signs of a sign
+    # pair sit 16 bits apart in one 32-bit word (a decoder's single shift).
+    fmt, N = (3, 4, 1), 16
+    zero = dict(kidx=np.zeros((N, d), np.uint8), ksign=np.zeros((N, d), np.uint8),
+                knorm=np.zeros(N, np.uint16), rnorm=np.zeros(N, np.uint16),
+                vidx=np.zeros((N, d), np.uint8), vnorm=np.zeros(N, np.uint16))
+    key_region = 2 * 4 * d                 # bytes of the key+sign words of a tile (of 2*W*d)
+    C = 16                                 # chunk bytes: a lane string is W*d/16 = d/2 bytes
+
+    def lane_bit(byte_in_tile, bit):
+        chunk, lane, off = byte_in_tile // (32 * C), (byte_in_tile // C) % 32, byte_in_tile % C
+        return lane, (chunk * C + off) * 8 + bit
+
+    for n in (0, 5, 8, 15):
+        for i in range(0, d, 3):
+            c = {k: v.copy() for k, v in zero.items()}
+            c["kidx"][n, i] = 7
+            bits = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+            assert bits.size == 3 and len({b // 8 for b in bits}) == 1
+            assert all(b % 8 <= 5 for b in bits) and bits[0] // 8 < key_region
+            c = {k: v.copy() for k, v in zero.items()}
+            c["ksign"][n, i] = 1
+            sb = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+            assert sb.size == 1 and sb[0] % 8 in (6, 7) and sb[0] // 8 < key_region
+            # its partner (the neighbouring coordinate of the pair) is 16 bits away
+            j = i ^ 1
+            c["ksign"][n, i] = 0
+            c["ksign"][n, j] = 1
+            sj = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))[0]
+            li, bi = lane_bit(sb[0] // 8, sb[0] % 8)
+            lj, bj = lane_bit(sj // 8, sj % 8)
+            assert li == lj and abs(bi - bj) == 16 and bi // 32 == bj // 32
+
+
 def test_pack_sizes_match_pages(golden):
     vals = {r[0]: float(r[1]) for r in golden("pages_numbers.txt")}
     d = 128
