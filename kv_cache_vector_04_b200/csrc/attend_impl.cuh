@@ -279,14 +279,19 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
         const float sc = es[g];
         for (int nt = w; nt < D / 8; nt += NT / 32) {
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+            // all of this n-tile's S fragments first: one L2 round trip, not D/16
+            uint2 bfs[D / 16];
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                bfs[kk] = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
+#pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const int c0 = 16 * kk + 2 * t;
                 const float x0 = qt[c0][g] * sc, x1 = qt[c0 + 1][g] * sc;
                 const float x2 = qt[c0 + 8][g] * sc, x3 = qt[c0 + 9][g] * sc;
                 const float h0 = __half2float(__float2half_rn(x0)), h1 = __half2float(__float2half_rn(x1));
                 const float h2 = __half2float(__float2half_rn(x2)), h3 = __half2float(__float2half_rn(x3));
-                const uint2 bf = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
+                const uint2 bf = bfs[kk];
                 mma_16816(acc, pack_half2(h0, h1), 0u, pack_half2(h2, h3), 0u, bf.x, bf.y);
                 mma_16816(acc, pack_half2(x0 - h0, x1 - h1), 0u, pack_half2(x2 - h2, x3 - h3), 0u,
                           bf.x, bf.y);
@@ -482,13 +487,21 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0.0;
         if (T == 1) {   // the decode step: one key, four independent partial sums
+            // the loads of S in batches of 32, all in flight at once
+            constexpr int NB = 32;
             double z1 = 0.0, z2 = 0.0, z3 = 0.0;
-#pragma unroll 4
-            for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); c += 4) {
-                z[0] = fma((double)__ldg(tb.s_t + (size_t)c * M + j), rk[c], z[0]);
-                z1 = fma((double)__ldg(tb.s_t + (size_t)(c + 1) * M + j), rk[c + 1], z1);
-                z2 = fma((double)__ldg(tb.s_t + (size_t)(c + 2) * M + j), rk[c + 2], z2);
-                z3 = fma((double)__ldg(tb.s_t + (size_t)(c + 3) * M + j), rk[c + 3], z3);
+#pragma unroll 1
+            for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += NB) {
+                float sv[NB];
+#pragma unroll
+                for (int u = 0; u < NB; ++u) sv[u] = __ldg(tb.s_t + (size_t)(c0 + u) * M + j);
+#pragma unroll
+                for (int u = 0; u < NB; u += 4) {
+                    z[0] = fma((double)sv[u], rk[c0 + u], z[0]);
+                    z1 = fma((double)sv[u + 1], rk[c0 + u + 1], z1);
+                    z2 = fma((double)sv[u + 2], rk[c0 + u + 2], z2);
+                    z3 = fma((double)sv[u + 3], rk[c0 + u + 3], z3);
+                }
             }
             z[0] = (z[0] + z1) + (z2 + z3);
         } else {
