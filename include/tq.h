@@ -144,8 +144,10 @@ int tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
 
 /* tq_init for any built format (B_K = kbits, B_V = vbits, QJL sketch on keys
  * iff qjl = 1); tq_init(d, b, ...) is tq_init_ex(d, b - 1, b, 1, ...). Built:
- * qjl = 1 with kbits = vbits - 1 and vbits in {2, 3, 4} (TurboQuant), and the
- * MSE-only key formats qjl = 0 with (kbits, vbits) in {(2,2), (3,3), (4,4),
+ * qjl = 1 with kbits = vbits - 1 and vbits in {2, 3, 4} (TurboQuant); qjl = 1
+ * with (kbits, vbits) = (7, 4): the k8v4 variant of the table below, read as
+ * TurboQuant keys at 8 bits (7-bit cells + the QJL sketch) with 4-bit values;
+ * and the MSE-only key formats qjl = 0 with (kbits, vbits) in {(2,2), (3,3), (4,4),
  * (3,4)}: the "nc" and k3v4-nc variants of the method table in the vLLM
  * section ("vLLM 工程師的實測") of turboquant-kvquant-vllm-benchmark, read as
  * "no QJL correction" ([MUNINN] §"MSE-Only vs QJL" contrasts the two). Without
@@ -157,7 +159,7 @@ int tq_init_ex(int d, int kbits, int vbits, int qjl, int codebook, uint64_t seed
  * approximates (turboquant-kvquant-vllm-benchmark, "TurboQuant 是什麼", step
  * 1: the rotation concentrates the coordinates as a Beta distribution). */
 
-/* One codebook alone, on the host (no device, no context): B in 1..4 bits,
+/* One codebook alone, on the host (no device, no context): B in 1..7 bits,
  * d >= 3; fp32 centroids[2^B] and boundaries[2^B - 1] (fp32 midpoints). */
 int tq_build_codebook(int B, int d, int codebook, float* centroids, float* bounds);
 

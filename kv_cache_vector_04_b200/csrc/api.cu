@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -22,12 +23,14 @@ struct tq_ctx {
 
 namespace {
 
-// The built formats (B_K, B_V, qjl): TurboQuant at 2, 3, 4 bits, and the
+// The built formats (B_K, B_V, qjl): TurboQuant at 2, 3, 4 bits; TurboQuant
+// keys at 8 bits with 4-bit values ("k8v4": 7-bit cells + QJL); and the
 // MSE-only key formats 2/2, 3/3, 4/4 and 3/4 bits.
 bool supported(int d, int kbits, int vbits, int qjl)
 {
     if (d != 64 && d != 128 && d != 256) return false;
-    if (qjl == 1) return vbits >= 2 && vbits <= 4 && kbits == vbits - 1;
+    if (qjl == 1)
+        return (vbits >= 2 && vbits <= 4 && kbits == vbits - 1) || (kbits == 7 && vbits == 4);
     if (qjl == 0)
         return (kbits == vbits && kbits >= 2 && kbits <= 4) || (kbits == 3 && vbits == 4);
     return false;
@@ -92,7 +95,8 @@ int upload_tables(tq_ctx* ctx)
     const int d = h.d, m = h.m, nk = 1 << h.kbits, nv = 1 << h.vbits;
     const float sd = std::sqrt(float(d));
 
-    std::vector<double> bounds_k(16, 0.0), centroids_kd(16, 0.0), bounds_v(16, 0.0);
+    std::vector<double> bounds_k(std::max(nk, 16), 0.0), centroids_kd(std::max(nk, 16), 0.0),
+        bounds_v(16, 0.0);
     for (int j = 0; j < nk; ++j) centroids_kd[j] = double(h.centroids_k[j]);
     for (int j = 0; j + 1 < nk; ++j) bounds_k[j] = double(h.bounds_k[j]);
     for (int j = 0; j + 1 < nv; ++j) bounds_v[j] = double(h.bounds_v[j]);
@@ -115,11 +119,23 @@ int upload_tables(tq_ctx* ctx)
     std::vector<float> st(size_t(d) * m);
     for (int j = 0; j < m; ++j)
         for (int i = 0; i < d; ++i) st[size_t(i) * m + j] = h.S[size_t(j) * d + i];
-    std::vector<uint32_t> lutk(size_t(nk) * nk), lutv(size_t(nv) * nv);
+    // Key decode table: per pair of cells, fp16x2 of both levels; for cells of
+    // more than 4 bits, per cell, the level split as fp16 {hi, lo = rest}
+    // (128 levels cannot all be fp16-exact under one scale).
+    const bool per_code = h.kbits > 4;
+    std::vector<uint32_t> lutk(per_code ? size_t(nk) : size_t(nk) * nk), lutv(size_t(nv) * nv);
     const double sdk = std::sqrt(double(d)) * double(h.alpha_k);
-    for (int f = 0; f < nk * nk; ++f)
-        lutk[f] = half2_bits(float(double(h.centroids_k[f & (nk - 1)]) * sdk),
-                             float(double(h.centroids_k[f >> h.kbits]) * sdk));
+    if (per_code) {
+        for (int f = 0; f < nk; ++f) {
+            const float x = float(double(h.centroids_k[f]) * sdk);
+            const float hi = __half2float(__float2half_rn(x));
+            lutk[f] = half2_bits(hi, x - hi);
+        }
+    } else {
+        for (int f = 0; f < nk * nk; ++f)
+            lutk[f] = half2_bits(float(double(h.centroids_k[f & (nk - 1)]) * sdk),
+                                 float(double(h.centroids_k[f >> h.kbits]) * sdk));
+    }
     for (int f = 0; f < nv * nv; ++f)
         lutv[f] = half2_bits(h.centroids_v[f & (nv - 1)] * sd, h.centroids_v[f >> h.vbits] * sd);
 
@@ -239,7 +255,8 @@ extern "C" {
 
 int tq_build_codebook(int B, int d, int codebook, float* centroids, float* bounds)
 {
-    if (B < 1 || B > 4 || d < 3 || d > 4096 || !centroids || !bounds) return TQ_ERR_INVALID_ARG;
+    if (B < 1 || B > tq::kMaxCellBits || d < 3 || d > 4096 || !centroids || !bounds)
+        return TQ_ERR_INVALID_ARG;
     if (codebook == TQ_CODEBOOK_GAUSS)
         return tq::build_codebook(B, d, centroids, bounds) ? TQ_OK : TQ_ERR_CUDA;
     if (codebook == TQ_CODEBOOK_BETA)

@@ -69,6 +69,10 @@ struct AttTraits {
     static constexpr int CODE_BYTES = 2 * W * D;             // code region of a tile
     static constexpr int KNB = 32 + 32 * QJ;                 // K norm bytes of a tile
     static constexpr int TILE_BYTES = CODE_BYTES + KNB + 32;
+    static constexpr int NTAB = (1 << KB) > 16 ? (1 << KB) : 16;   // key table slots of the append
+    // Keys of more than 4 bits (7-bit cells, the 8-bit TurboQuant keys of
+    // k8v4) are decoded code by code: a pair table would have 2^14 rows.
+    static constexpr bool CK = KB > 4;
     // Byte fields: an 8-bit field that starts on a byte of the lane string (a
     // pair of 4-bit cells, or the 6-bit pair of 3-bit keys in the low bits of
     // a byte whose top bits hold two QJL signs) is turned into its table
@@ -81,15 +85,19 @@ struct AttTraits {
     static constexpr int LSH = ROWS ? 8 : 7;                 // log2 of a table entry's stride
     static constexpr int VW0 = VBIT0 / 32;                   // first value word (byte fields)
     static_assert(!PK || ROWS, "byte-field keys come with byte-field values");
+    static_assert(!CK || (ROWS && KB <= 7), "per-code keys use the row table (up to 128 codes)");
     static_assert(!PV || VBIT0 % 32 == 0, "byte-field values start on a word");
     static constexpr size_t LUT_BYTES = ROWS ? (size_t)256 * 256 : (size_t)(NLK + NLV) * 128;
     static constexpr size_t QF_BYTES = (size_t)KK * 32 * 32; // hi/lo B fragments per k-step
+    static constexpr size_t SMEM_CAP = 227u * 1024u - 1024u;
     // One CTA of 16 warps per SM, 128 registers a thread: the kernel is
     // issue-bound, so warps to hide latency are worth more than registers; the
     // query fragments are read from shared memory. (Measured against 3 CTAs of
     // 4 warps with the fragments in registers at d <= 128, 8 warps at d = 256,
     // and 20 or 24 warps at d = 64: 16 warps was the fastest at every d.)
-    static constexpr int WARPS = 16, NT = 32 * WARPS;
+    // 8 warps where 16 rings of 2 tiles do not fit (k8v4 at d = 256).
+    static constexpr int WARPS = LUT_BYTES + (size_t)16 * 2 * TILE_BYTES + QF_BYTES <= SMEM_CAP ? 16 : 8;
+    static constexpr int NT = 32 * WARPS;
     static constexpr size_t MERGE_BYTES = (size_t)WARPS * 8 * (D + 2) * 4;
     static constexpr size_t QF_SMEM = QF_BYTES;
     // The decode tables are static shared arrays when they fit there (the
@@ -98,7 +106,6 @@ struct AttTraits {
     static constexpr bool STATIC_LUT = LUT_BYTES <= 40 * 1024;
     // staging ring: per warp STAGES images of whole tiles, each brought in by
     // one bulk copy; 3 stages where they fit in shared memory, else 2
-    static constexpr size_t SMEM_CAP = 227u * 1024u - 1024u;
     static constexpr int STAGES =
         LUT_BYTES + (size_t)WARPS * 3 * TILE_BYTES + QF_SMEM <= SMEM_CAP ? 3 : 2;
     static constexpr int STAGE_BYTES = TILE_BYTES;
@@ -395,16 +402,17 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
         return;
     }
     uint32_t* img = reinterpret_cast<uint32_t*>(smem);                      // [2][TB]
-    double* tabs = reinterpret_cast<double*>(smem + 2 * TB);                // ck[16] tk[16] tv[16]
-    double* rk = tabs + 48;                                                  // [16][D] key residuals
+    constexpr int NK = Tr::NTAB;                                              // key table slots
+    double* tabs = reinterpret_cast<double*>(smem + 2 * TB);                // ck[NK] tk[NK] tv[16]
+    double* rk = tabs + 2 * NK + 16;                                         // [16][D] key residuals
     double* zp = rk + 16 * D;                                                // [16][M] half-sums of z
     const int t0 = start / 16, ntile = (start + T - 1) / 16 - t0 + 1;
     uint8_t* stream = a.cache_w + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity / 16) * TB;
     for (int e = tid; e < ntile * TB / 16; e += NT)
         reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(stream + (size_t)t0 * TB)[e];
     if (tid < (1 << BK)) tabs[tid] = tb.centroids_kd[tid];
-    if (tid < (1 << BK) - 1) tabs[16 + tid] = tb.bounds_k[tid];
-    if (tid < (1 << BV) - 1) tabs[32 + tid] = tb.bounds_v[tid];
+    if (tid < (1 << BK) - 1) tabs[NK + tid] = tb.bounds_k[tid];
+    if (tid < (1 << BV) - 1) tabs[2 * NK + tid] = tb.bounds_v[tid];
     __syncthreads();
 
     unsigned sat = 0u;
@@ -440,7 +448,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
             for (int k = 0; k < VPL; ++k) {
                 const int c = lane * VPL + k;
                 const double y = x[k] * scale;
-                const int idx = encode_cell<BK>(y, tabs + 16);
+                const int idx = encode_cell<BK>(y, tabs + NK);
                 if constexpr (QJ) {
                     const double r = y - tabs[idx];
                     rk[i * D + c] = r;
@@ -466,7 +474,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
 #pragma unroll
             for (int k = 0; k < VPL; ++k) {
                 const int c = lane * VPL + k;
-                const int idx = encode_cell<BV>(x[k] * scale, tabs + 32);
+                const int idx = encode_cell<BV>(x[k] * scale, tabs + 2 * NK);
                 // V field: token 2 t + 8 (r >> 1) + e, coordinate 16 kk + g' + 8 (r & 1)
                 const int kk = c >> 4, gc = c & 7, t = (tau & 7) >> 1, e = tau & 1;
                 const int p = 4 * kk + 2 * half + ((c & 15) >> 3);
@@ -756,13 +764,23 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
         const uint4 bc = qf.fc(kk, lane);
-        uint32_t ak[4], as[4];
+        uint32_t ak[4], as[4], akl[4];   // akl: lo parts of per-code key levels
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int p = 4 * kk + r;
             if constexpr (Tr::PK) {
                 ak[r] = lut_load(lutk, row_off(td.s[kk], r, lane4));
                 if constexpr (QJ) as[r] = sign_pair_byte(td.s[kk], r, (r & 1) ? nr_h : nr_g);
+            } else if constexpr (Tr::CK) {
+                // one table row per code, {hi, lo} of its level: the pair's hi
+                // parts form the A fragment, its lo parts a second one
+                using Lay = TileLayout<D, KB, VB, QJ>;
+                const uint32_t e0 = lut_load(lutk, lut_off<8>(td.s, Lay::kbit(p, 0), KB, lane4));
+                const uint32_t e1 = lut_load(lutk, lut_off<8>(td.s, Lay::kbit(p, 1), KB, lane4));
+                ak[r] = __byte_perm(e0, e1, 0x5410u);
+                akl[r] = __byte_perm(e0, e1, 0x7632u);
+                if constexpr (QJ)
+                    as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
             } else {
                 ak[r] = lut_load(lutk, lut_off<Tr::LSH>(td.s, Tr::KF * p, Tr::KF, lane4));
                 if constexpr (QJ)
@@ -776,6 +794,7 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
             mma_16816(ah, ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
             mma_16816(al, ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
         }
+        if constexpr (Tr::CK) mma_16816(al, akl[0], akl[1], akl[2], akl[3], bc.x, bc.y);
         if constexpr (QJ) {
             const uint4 bs = qf.fs(kk, lane);
             mma_16816(ah, as[0], as[1], as[2], as[3], bs.x, bs.y);
@@ -859,11 +878,13 @@ __device__ __forceinline__ void fill_luts(const DevTables& tb, uint32_t* lutk, u
     using Tr = AttTraits<D, KB, VB, QJ>;
     if constexpr (Tr::ROWS) {
         // row x: the key entry (key pair x & (NLK - 1): byte-field keys ignore
-        // the sign bits above it), then the value entry x; 64 words a row
+        // the sign bits above it; per-code keys: level x as fp16 hi and lo),
+        // then the value entry x; 64 words a row
         for (int e = tid; e < 256 * 64; e += NT) {
             const int x = e >> 6;
             uint32_t v;
             if ((e & 63) >= 32) v = __ldg(tb.lut_v + x);
+            else if (Tr::CK) v = x < (1 << KB) ? __ldg(tb.lut_k + x) : 0u;   // level x: {hi, lo}
             else v = (Tr::PK || x < Tr::NLK) ? __ldg(tb.lut_k + (x & (Tr::NLK - 1))) : 0u;
             lutk[e] = v;
         }
@@ -1187,7 +1208,7 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
     if (a.k_new != nullptr && a.T > 0) {
         static unsigned long long done_append = 0;
         constexpr int TB = Tr::TILE_BYTES;
-        const size_t smem = 2 * (size_t)TB + 8 * (48 + (size_t)16 * D + (size_t)16 * D);
+        const size_t smem = 2 * (size_t)TB + 8 * (2 * (size_t)Tr::NTAB + 16 + (size_t)16 * D + (size_t)16 * D);
         auto kern = append_prologue<D, KB, VB, QJ>;
         if ((e = allow_smem(kern, smem, done_append)) != cudaSuccess) return e;
         e = launch_pdl(kern, dim3(units + a.Hkv, a.B), dim3(2 * D), smem, st, tb, a);

@@ -70,7 +70,8 @@ int attend_ctas_per_sm(const Format& f);
 
 // Every built format, for the launch tables: X(D, KB, VB, QJL).
 #define TQ_FORMATS_D(X, D) \
-    X(D, 1, 2, 1) X(D, 2, 3, 1) X(D, 3, 4, 1) X(D, 2, 2, 0) X(D, 3, 3, 0) X(D, 4, 4, 0) X(D, 3, 4, 0)
+    X(D, 1, 2, 1) X(D, 2, 3, 1) X(D, 3, 4, 1) X(D, 7, 4, 1) X(D, 2, 2, 0) X(D, 3, 3, 0) X(D, 4, 4, 0) \
+    X(D, 3, 4, 0)
 #define TQ_FORMATS(X) TQ_FORMATS_D(X, 64) TQ_FORMATS_D(X, 128) TQ_FORMATS_D(X, 256)
 
 }  // namespace tq

@@ -64,7 +64,7 @@ struct QuantSmem {
     uint32_t sg[16][D / 32];          // QJL sign bits, row j at bit j%32 of word j/32
     uint8_t kc[16][D];                // key cell indices
     uint8_t vc[16][D];                // value cell indices
-    double ck[16], tk[16], tv[16];    // key centroids, key / value boundaries (fp64 copies)
+    double ck[128], tk[128], tv[16];  // key centroids, key / value boundaries (fp64 copies; keys up to 7 bits)
     float rho[16];                    // |r| of each key
     uint16_t nk[16], nr[16], nv[16];  // fp16 norms
 };

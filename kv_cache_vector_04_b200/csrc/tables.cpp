@@ -81,7 +81,7 @@ bool gaussian_lloyd_max(int B, double* level)
 {
     const int n = 1 << B;
     for (int j = 0; j < n; ++j) level[j] = 3.0 * (2.0 * j + 1.0 - n) / (2.0 * n);
-    double edge[17];
+    double edge[kMaxLevels + 1];
     bool converged = false;
     double last_step = INFINITY;
     for (int iter = 0; iter < 4000000 && !converged; ++iter) {
@@ -174,7 +174,7 @@ bool beta_lloyd_max(int B, int d, double* level)
     bool converged = false;
     double last_step = INFINITY;
     for (int iter = 0; iter < 100000 && !converged; ++iter) {
-        double moved = 0.0, next[16];
+        double moved = 0.0, next[kMaxLevels];
         for (int j = 0; j < n; ++j) {
             const double lo = (j == 0) ? -1.0 : 0.5 * (level[j - 1] + level[j]);
             const double hi = (j == n - 1) ? 1.0 : 0.5 * (level[j] + level[j + 1]);
@@ -195,7 +195,7 @@ bool beta_lloyd_max(int B, int d, double* level)
 
 bool build_codebook_beta(int B, int d, float* centroids, float* bounds)
 {
-    double level[16];
+    double level[kMaxLevels];
     const bool ok = beta_lloyd_max(B, d, level);
     const int n = 1 << B;
     for (int j = 0; j < n; ++j) centroids[j] = float(level[j]);
@@ -206,7 +206,7 @@ bool build_codebook_beta(int B, int d, float* centroids, float* bounds)
 
 bool build_codebook(int B, int d, float* centroids, float* bounds)
 {
-    double unit[16];
+    double unit[kMaxLevels];
     const bool ok = gaussian_lloyd_max(B, unit);
     const int n = 1 << B;
     const double scale = 1.0 / std::sqrt(double(d));
@@ -283,7 +283,8 @@ bool build_host_tables(int d, int kbits, int vbits, int qjl, int codebook, uint6
     ok = cb(t.vbits, d, t.centroids_v.data(), t.bounds_v.data()) && ok;
     build_rotation_signs(d, seed, t.signs.data());
     build_qjl_matrix(t.m, d, seed, t.S.data());
-    t.alpha_k = choose_decode_scale(t.centroids_k.data(), 1 << t.kbits, d);
+    // cells of more than 4 bits are decoded as fp16 hi + lo parts: no scale needed
+    t.alpha_k = t.kbits > 4 ? 1.f : choose_decode_scale(t.centroids_k.data(), 1 << t.kbits, d);
     return ok;
 }
 

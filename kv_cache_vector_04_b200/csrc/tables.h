@@ -5,6 +5,11 @@
 
 namespace tq {
 
+// Most codebook levels of a format: 7-bit key cells (the 8-bit TurboQuant keys
+// of k8v4, (7, 4, 1)).
+constexpr int kMaxCellBits = 7;
+constexpr int kMaxLevels = 1 << kMaxCellBits;
+
 struct HostTables {
     int d = 0, bits = 0, m = 0, kbits = 0, vbits = 0, qjl = 1;
     int codebook = 0;                          // 0: N(0, 1/d) model, 1: exact Beta marginal

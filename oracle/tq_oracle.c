@@ -46,6 +46,7 @@
 #include <string.h>
 
 #define TQO_TILE 16
+#define TQO_MAXL 128   /* most codebook levels: 7-bit cells */
 
 /* ------------------------------------------------------------------------- */
 /* Scalar conversions.                                                        */
@@ -188,7 +189,7 @@ static double Phi(double x) { return 0.5 * erfc(-x / M_SQRT2); }
 int oracle_lloyd_max_unit(int B, double* c, int* iters_out)
 {
     int L = 1 << B;
-    double nc[16];
+    double nc[TQO_MAXL];
     for (int j = 0; j < L; ++j) c[j] = -2.0 + 4.0 * (j + 0.5) / L;
     int it, ok = -1;
     double prev = INFINITY;
@@ -242,7 +243,7 @@ double oracle_quantizer_mse_unit(int B, const double* c)
  * rounded once to fp32; boundaries are the fp32 midpoints of neighbours. */
 int oracle_codebook(int B, int d, float* centroids, float* bounds)
 {
-    double c[16];
+    double c[TQO_MAXL];
     int rc = oracle_lloyd_max_unit(B, c, NULL);
     int L = 1 << B;
     for (int j = 0; j < L; ++j) centroids[j] = (float)(c[j] / sqrt((double)d));
@@ -300,13 +301,13 @@ int oracle_lloyd_max_beta(int d, int B, double* c)
 {
     int L = 1 << B;
     if (d >= 16) {
-        double g[16];
+        double g[TQO_MAXL];
         oracle_lloyd_max_unit(B, g, NULL);
         for (int j = 0; j < L; ++j) c[j] = g[j] / sqrt((double)d);
     } else {
         for (int j = 0; j < L; ++j) c[j] = -1.0 + (2.0 * j + 1.0) / L;
     }
-    double nc[16], prev = INFINITY;
+    double nc[TQO_MAXL], prev = INFINITY;
     int ok = -1;
     for (int it = 0; it < 100000; ++it) {
         double delta = 0.0;
@@ -351,7 +352,7 @@ double oracle_quantizer_mse_beta(int d, int B, const double* c)
  * boundaries the fp32 midpoints (the same rounding as oracle_codebook). */
 int oracle_codebook_beta(int B, int d, float* centroids, float* bounds)
 {
-    double c[16];
+    double c[TQO_MAXL];
     int rc = oracle_lloyd_max_beta(d, B, c);
     int L = 1 << B;
     for (int j = 0; j < L; ++j) centroids[j] = (float)c[j];
@@ -768,7 +769,7 @@ void oracle_attend_batch(int d, int B, int Hq, int Hkv, int cap, const int32_t* 
  * vectors and coordinates of (y_i - c[idx_i])^2 [MUNINN §Lloyd-Max Codebook]. */
 double oracle_distortion_mc(int d, int B, int nvec, uint64_t seed)
 {
-    float c[16], t[15];
+    float c[TQO_MAXL], t[TQO_MAXL];
     oracle_codebook(B, d, c, t);
     int L = 1 << B;
     double total = 0.0;
@@ -800,7 +801,7 @@ void oracle_ip_trials(int d, int bits, int ntrials, uint64_t seed0, const double
                       const double* k, double* est_mse, double* est_qjl)
 {
     int m = d;
-    float cM[16], tM[15], cK[16], tK[15];
+    float cM[TQO_MAXL], tM[TQO_MAXL], cK[TQO_MAXL], tK[TQO_MAXL];
     oracle_codebook(bits, d, cM, tM);
     if (bits > 1) oracle_codebook(bits - 1, d, cK, tK);
     double kn = 0.0;

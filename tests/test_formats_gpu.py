@@ -132,3 +132,71 @@ def test_beta_codebook_tables_quantize_and_attend(d, fmt):
     ref = O.attend_batch(tab, P.q_bits(q), True, P.stack_codes(codes, 112), np.array(seq, np.int32), 2)
     assert P.attn_error(got.cpu().numpy().astype(np.float64), ref).max() <= P.ATTN_TOL
     assert tq.tq_status(ctx) == 0
+
+
+# ---------------------------------------------------------------- k8v4: 8-bit TurboQuant keys
+
+# "TQ k8v4" of the same vLLM table, read as TurboQuant keys at 8 bits (7-bit
+# Lloyd-Max cells plus the 1-bit QJL sketch) with 4-bit values: (7, 4, 1). The
+# decoder takes the 7-bit key levels code by code, each as fp16 hi + lo parts.
+K8V4 = (7, 4, 1)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_k8v4_layout_and_quantize(d):
+    # check_quantize unpacks the device's bytes with the oracle's packer layout
+    # and compares every code with the oracle's: the layout and the decisions
+    ctx, tab = ctx_for(d, 4, fmt=K8V4)
+    lay = tq.tq_cache_layout(ctx)
+    assert (lay["kbits"], lay["vbits"], lay["qjl"]) == K8V4
+    assert lay["tile_bytes"] == O.tile_bytes(d, K8V4)
+    assert lay["k_bytes_per_token"] == d + 4 and lay["v_bytes_per_token"] == d // 2 + 2
+    stats = P.QuantStats()
+    for T, dist in ((77, "lognormal_norm"), (40, "outlier_channels"), (33, "spiky_tokens")):
+        k, v = kv(2, 2, T, d, seed=d + T, dist=dist)
+        cache = P.quantize_on_gpu(ctx, k, v, capacity=T + 19)
+        check_quantize(ctx, tab, k, v, cache, stats=stats)
+    stats.check()
+    assert tq.tq_status(ctx) == 0
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("dist", ["lognormal_norm", "outlier_channels", "spiky_tokens"])
+def test_k8v4_attend_on_oracle_packed_cache(d, dist):
+    ctx, tab = ctx_for(d, 4, fmt=K8V4)
+    B, Hkv, Hq, N, cap = 2, 2, 8, 203, 208
+    k, v = kv(B, Hkv, N, d, seed=70 + d, dist=dist)
+    codes = P.oracle_codes(tab, k, v)
+    cache = tq.Cache(P.pack_cache(tab, codes, cap, d, 4), B, Hkv, cap)
+    seq = [203, 90]
+    for qs in (1.0, 3.0):
+        q = (qtensor(B, Hq, d, seed=8).float() * qs).to(torch.bfloat16)
+        got = tq.tq_attend(ctx, q.cuda(), cache, torch.tensor(seq, dtype=torch.int32).cuda(), N)
+        torch.cuda.synchronize()
+        ref = O.attend_batch(tab, P.q_bits(q), True, P.stack_codes(codes, cap), np.array(seq, np.int32),
+                             Hkv)
+        err = P.attn_error(got.cpu().numpy().astype(np.float64), ref)
+        assert err.max() <= P.ATTN_TOL, (qs, err.max())
+    assert tq.tq_status(ctx) == 0
+
+
+def test_k8v4_scores_match_oracle_logits():
+    d = 128
+    ctx, tab = ctx_for(d, 4, fmt=K8V4)
+    B, Hkv, Hq, N, cap = 1, 2, 4, 77, 80
+    k, v = kv(B, Hkv, N, d, seed=12, dist="outlier_channels")
+    codes = P.oracle_codes(tab, k, v)
+    cache = tq.Cache(P.pack_cache(tab, codes, cap, d, 4), B, Hkv, cap)
+    q = qtensor(B, Hq, d, seed=3)
+    got = tq.tq_scores(ctx, q.cuda(), cache, torch.tensor([N], dtype=torch.int32).cuda(), N)
+    torch.cuda.synchronize()
+    _, lg = O.attend_batch(tab, P.q_bits(q), True, P.stack_codes(codes, cap),
+                           np.array([N], np.int32), Hkv, want_logits=True)
+    g = got.cpu().numpy().astype(np.float64)
+    ref = lg[:, :, :N]
+    assert np.abs(g - ref).max() <= P.ATTN_TOL * (np.abs(ref).max() + 1.0)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_k8v4_append_one_token_then_attend(d):
+    run_append(d, 4, 1, [32, 37, 47], seed=d + 7, fmt=K8V4)

@@ -83,9 +83,13 @@ def test_monte_carlo_distortion_matches():
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("B", [1, 2, 3, 4])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 7])
 def test_library_codebooks_equal_oracle(d, B):
-    for kind, code in (("gauss", tq.TQ_CODEBOOK_GAUSS), ("beta", tq.TQ_CODEBOOK_BETA)):
+    # 7 bits (the key cells of k8v4): the Gaussian model only; the oracle's
+    # exact-marginal iteration integrates every cell by quadrature, minutes at 7 bits
+    kinds = (("gauss", tq.TQ_CODEBOOK_GAUSS),) if B > 4 else \
+        (("gauss", tq.TQ_CODEBOOK_GAUSS), ("beta", tq.TQ_CODEBOOK_BETA))
+    for kind, code in kinds:
         c_lib, t_lib = tq.tq_build_codebook(B, d, code)
         c_ora, t_ora = O.codebook(B, d, kind)
         assert np.array_equal(c_lib, c_ora), (kind, c_lib, c_ora)

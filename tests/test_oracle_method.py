@@ -175,7 +175,7 @@ def test_pack_round_trip(d, b):
                 assert np.unpackbits(blk).mean() > 0.4
 
 
-FORMATS = [(1, 2, 1), (2, 3, 1), (3, 4, 1), (2, 2, 0), (3, 3, 0), (4, 4, 0), (3, 4, 0)]
+FORMATS = [(1, 2, 1), (2, 3, 1), (3, 4, 1), (7, 4, 1), (2, 2, 0), (3, 3, 0), (4, 4, 0), (3, 4, 0)]
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
@@ -304,7 +304,7 @@ def _random_codes(tab, N, seed, kscale=1.0):
 
 
 @pytest.mark.parametrize("d,bits,fmt", [(64, 2, None), (128, 3, None), (256, 4, None),
-                                        (128, 3, (3, 3, 0)), (64, 4, (3, 4, 0))])
+                                        (128, 3, (3, 3, 0)), (64, 4, (3, 4, 0)), (128, 4, (7, 4, 1))])
 def test_attention_equals_sdpa_over_reconstructed(d, bits, fmt):
     # with fmt (B_K, B_V, 0) the keys are the MSE-only reconstructions
     tab = O.Tables(d, bits, seed=5, fmt=fmt)

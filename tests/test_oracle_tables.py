@@ -141,7 +141,7 @@ def test_codebook_matches_textbook_table(golden):
         assert abs(O.quantizer_mse_unit(B, c) - mse_ref) < 1e-3 * mse_ref + 2e-5
 
 
-@pytest.mark.parametrize("B", [1, 2, 3, 4])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 7])
 def test_codebook_centroid_condition_by_quadrature(B):
     # Independent numerical integration: each centroid is the mean of N(0,1)
     # over its cell, and MSE = 1 - sum_j c_j^2 P_j at the optimum.
@@ -157,12 +157,12 @@ def test_codebook_centroid_condition_by_quadrature(B):
         s += c[j] ** 2 * mass
     mse_q = scipy.integrate.quad(
         lambda x: (x - c[np.searchsorted(t[1:-1], x)]) ** 2 * scipy.stats.norm.pdf(x),
-        -12, 12, points=list(t[1:-1]), limit=400, epsabs=1e-13)[0]
+        -12, 12, points=list(t[1:-1]), limit=4000, epsabs=1e-13)[0]
     assert abs(O.quantizer_mse_unit(B, c) - mse_q) < 1e-9
     assert abs(O.quantizer_mse_unit(B, c) - (1.0 - s)) < 1e-9
 
 
-@pytest.mark.parametrize("B", [1, 2, 3, 4])
+@pytest.mark.parametrize("B", [1, 2, 3, 4, 7])
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_codebook_scaling_and_boundaries(B, d):
     c, t = O.codebook(B, d)
@@ -175,6 +175,19 @@ def test_codebook_scaling_and_boundaries(B, d):
     mid = ((c[:-1].astype(np.float64) + c[1:].astype(np.float64)) / 2).astype(np.float32)
     assert np.array_equal(t, mid)
     assert np.all(np.diff(c) > 0) and np.all(np.diff(t) > 0)
+
+
+def test_codebook_high_rate_limit():
+    # Panter-Dite: the optimal B-bit quantizer of N(0, 1) has MSE -> (pi sqrt(3) / 2) 4^-B
+    # as B grows, approached from below. The 7-bit key cells of k8v4 sit within 2 % of it.
+    limit = math.pi * math.sqrt(3.0) / 2.0
+    scaled = []
+    for B in (4, 5, 6, 7):
+        c, _, _ = O.lloyd_max_unit(B)
+        scaled.append(O.quantizer_mse_unit(B, c) * 4.0 ** B)
+    assert all(x < limit for x in scaled)
+    assert all(b > a for a, b in zip(scaled, scaled[1:]))
+    assert scaled[-1] > 0.98 * limit
 
 
 def test_distortion_matches_pages(golden):
