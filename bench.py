@@ -49,7 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-graph", action="store_true",
                     help="time the eager launch loop only (no CUDA graph of the step)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--report", choices=["all", "single", "qwen3b", "qwen32b", "sweep"], default=None,
+    ap.add_argument("--report", choices=["all", "single", "qwen3b", "qwen32b", "sweep", "formats"],
+                    default=None,
                     help="measure the other workloads instead of the bench line: one JSON line each")
     return ap.parse_args(argv)
 
@@ -240,9 +241,9 @@ def workload_by_name(name: str):
     from kv_cache_vector_04_b200 import inputs
     if name in inputs.WORKLOADS:
         return inputs.WORKLOADS[name]
-    sweep = {x.name: x for x in inputs.sweep_workloads()}
-    if name in sweep:
-        return sweep[name]
+    extra = {x.name: x for x in inputs.sweep_workloads() + inputs.format_workloads()}
+    if name in extra:
+        return extra[name]
     raise SystemExit("unknown workload %r" % name)
 
 
@@ -254,7 +255,7 @@ def run_tq(args, dist: Dist):
     w = workload_by_name(args.workload)
     layers = args.layers or w.layers
     dev = torch.device("cuda", dist.local_rank)
-    ctx = tq.tq_init(w.d, w.bits, 1)
+    ctx = tq.tq_init(w.d, w.bits, 1) if w.fmt is None else tq.tq_init_ex(w.d, *w.fmt, 1)
     lay = tq.tq_cache_layout(ctx)
     per_tok = lay["tile_bytes"] // 16                     # K + V bytes per head-token
     N = w.N
@@ -461,6 +462,7 @@ def run_tq(args, dist: Dist):
         "data": "synthetic",
         "config": {"workload": w.name, "layers": layers, "batch": w.B, "q_heads": w.Hq,
                    "kv_heads": w.Hkv, "head_dim": w.d, "bits": w.bits, "context": N + 1,
+                   "format": list(tq.tq_cache_layout(ctx)[k] for k in ("kbits", "vbits", "qjl")),
                    "packed_cache_gb": round(layers * w.B * w.Hkv * cap * per_tok / 1e9, 2),
                    "step": "per layer: tq_append_attend (append 1 token, then attend)",
                    "step_launch": "one CUDA graph per step" if ms_graph is not None else "eager",
@@ -611,6 +613,11 @@ def run_report(args, dist: Dist):
     if which in ("all", "sweep"):
         from kv_cache_vector_04_b200 import inputs
         for w in inputs.sweep_workloads():
+            print(json.dumps(dict(report=w.name, **run(workload=w.name, layers=1, steps=10,
+                                                         warmup=3))), flush=True)
+    if which in ("all", "formats"):
+        from kv_cache_vector_04_b200 import inputs
+        for w in inputs.format_workloads():
             print(json.dumps(dict(report=w.name, **run(workload=w.name, layers=1, steps=10,
                                                          warmup=3))), flush=True)
 

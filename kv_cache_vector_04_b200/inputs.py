@@ -34,6 +34,7 @@ class Workload:
     seed: int
     decode_steps: int = 1
     notes: str = ""
+    fmt: tuple | None = None   # (B_K, B_V, qjl); None: TurboQuant at `bits`, (bits-1, bits, 1)
 
 
 WORKLOADS = {
@@ -63,6 +64,19 @@ def sweep_workloads():
                                     B=8, Hq=32, Hkv=8, N=N, kv_dist="lognormal_norm",
                                     q_dtype=torch.bfloat16, seed=1005))
     return out
+
+
+# Every built cache format: TurboQuant at 2, 3, 4 bits, k8v4, and the MSE-only keys.
+FORMATS = {"tq2": (1, 2, 1), "tq3": (2, 3, 1), "tq4": (3, 4, 1), "k8v4": (7, 4, 1),
+           "nc2": (2, 2, 0), "nc3": (3, 3, 0), "nc4": (4, 4, 0), "k3v4nc": (3, 4, 0)}
+
+
+def format_workloads():
+    """One decode layer per built format: d = 128, 8 kv heads, 32 query heads,
+    batch 8, 32K context."""
+    return [Workload("format_%s_d128_n32768" % name, d=128, bits=f[1], layers=1, B=8, Hq=32, Hkv=8,
+                     N=32768, kv_dist="lognormal_norm", q_dtype=torch.bfloat16, seed=1007, fmt=f)
+            for name, f in FORMATS.items()]
 
 
 def _gen(seed: int, device) -> torch.Generator:
