@@ -139,7 +139,8 @@ typedef struct {
  * Draw k of stream s is output k+1 of SplitMix64 started at
  * seed ^ (0x5851F42D4C957F2D * (s+1)).
  * *out receives a new context (owned by the caller; free with tq_destroy).
- * Allocates a small device block (< 600 KB) and synchronizes. */
+ * Allocates a small device block (under 1 MB: about 0.9 MB for 4-bit key pairs at
+ * d = 256, about 120 KB for TurboQuant at 3 bits and d = 128) and synchronizes. */
 int tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
 
 /* tq_init for any built format (B_K = kbits, B_V = vbits, QJL sketch on keys
