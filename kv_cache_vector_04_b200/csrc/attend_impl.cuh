@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArg
 
 
 // ---------------------------------------------------------------- reduction
-// One CTA per (query head, batch): merges, in one online-softmax pass, the
+// One CTA per (query head, batch): merges, in two passes (max, then sums), the
 // partials of the CTAs whose ranges cover the head's unit (the range of CTA c
 // is [c W / G, (c+1) W / G) of the W tiles, so tile x lies in CTA
 // ((x + 1) G - 1) / W), then applies Pi^T with an fp32 Walsh-Hadamard
@@ -590,20 +590,40 @@ __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
     if (T > 0) {
         const long long U0 = pb + ju * T, U1 = U0 + T;
         const int cf = (int)(((U0 + 1) * G - 1) / W), cl = (int)((U1 * G - 1) / W);
+        const float* base = a.partial + u * 8 * RS + col * RS;   // + c * 8 * RS: slot c + u
+        // CTA c's range starts at tile floor(c W / G); walked as quotient and
+        // remainder, so the loops divide nothing (a unit of a short batch can
+        // span most of the grid). A CTA with an empty range wrote no partial.
+        const long long wq = W / G, wr = W - wq * G;
+        const long long q0 = (long long)cf * W / G, r0 = (long long)cf * W - q0 * G;
+        // Two passes with independent loads (not one chain of dependent ones):
+        // the largest partial max, then the sums rescaled to it (a partial with
+        // max -inf adds 0).
+        long long q = q0, r = r0;
+#pragma unroll 4
         for (int c = cf; c <= cl; ++c) {
-            if ((long long)c * W / G == (long long)(c + 1) * W / G) continue;   // empty range
-            const float* ps = a.partial + ((size_t)c + u) * 8 * RS + col * RS;
-            const float ms = ps[0];
-            if (ms == -CUDART_INF_F) continue;
-            if (ms > M) {   // rescale what was merged so far (nothing while M = -inf)
-                const float f = M == -CUDART_INF_F ? 0.f : exp2f(M - ms);
-                L *= f;
-                acc *= f;
-                M = ms;
+            long long qn = q + wq, rn = r + wr;
+            if (rn >= G) { ++qn; rn -= G; }
+            if (qn != q) M = fmaxf(M, base[(size_t)c * 8 * RS]);
+            q = qn;
+            r = rn;
+        }
+        if (M != -CUDART_INF_F) {
+            q = q0;
+            r = r0;
+#pragma unroll 4
+            for (int c = cf; c <= cl; ++c) {
+                long long qn = q + wq, rn = r + wr;
+                if (rn >= G) { ++qn; rn -= G; }
+                if (qn != q) {
+                    const float* ps = base + (size_t)c * 8 * RS;
+                    const float f = exp2f(ps[0] - M);
+                    L = fmaf(ps[1], f, L);
+                    acc = fmaf(ps[2 + i], f, acc);
+                }
+                q = qn;
+                r = rn;
             }
-            const float f = exp2f(ms - M);
-            L = fmaf(ps[1], f, L);
-            acc = fmaf(ps[2 + i], f, acc);
         }
     }
     float x = (L > 0.f) ? acc / L : 0.f;
