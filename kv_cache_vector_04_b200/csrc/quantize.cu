@@ -297,6 +297,17 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
                         val |= (f << o) | ((bits & 1u) << a0) | ((bits >> 1) << a1);
                         if (is_new(tok)) msk |= (((1u << Tr::KF) - 1u) << o) | (1u << a0) | (1u << a1);
                     }
+                } else if (Tr::KF == 8 && wi < Tr::SBW) { // 4-bit key pairs 4 wi + j, one byte each
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int kk = wi;
+                        const int tok = gL + 8 * (j & 1);
+                        const int i0 = 16 * kk + 8 * (j >> 1) + 2 * tL;
+                        const uint32_t f = ((uint32_t)kc[tok][i0] & 15u) |
+                                           (((uint32_t)kc[tok][i0 + 1] & 15u) << 4);
+                        val |= f << (8 * j);
+                        if (is_new(tok)) msk |= 0xFFu << (8 * j);
+                    }
                 } else if (wi < Tr::SBW) {               // key cell fields
                     const int bit0 = 32 * wi;
                     for (int p = bit0 / Tr::KF; p <= (bit0 + 31) / Tr::KF; ++p) {
@@ -324,6 +335,18 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
                         const uint32_t bits = (sg[tok][row >> 5] >> (row & 31)) & 3u;
                         val |= ((bits & 1u) << q2) | ((bits >> 1) << (16 + q2));
                         if (is_new(tok)) msk |= (1u << q2) | (1u << (16 + q2));
+                    }
+                } else if (Tr::VF == 8) {                 // 4-bit value pairs, one byte each
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int kk = wi - Tr::VBW;       // pair 4 kk + j
+                        const int tok0 = 2 * tL + 8 * (j >> 1);
+                        const int coord = 16 * kk + gL + 8 * (j & 1);
+                        const uint32_t f = ((uint32_t)vc[tok0][coord] & 15u) |
+                                           (((uint32_t)vc[tok0 + 1][coord] & 15u) << 4);
+                        const uint32_t fm = (is_new(tok0) ? 0x0Fu : 0u) | (is_new(tok0 + 1) ? 0xF0u : 0u);
+                        val |= f << (8 * j);
+                        msk |= fm << (8 * j);
                     }
                 } else {                                  // value cell fields
                     const int bit0 = 32 * (wi - Tr::VBW);
