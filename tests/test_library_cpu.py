@@ -84,3 +84,21 @@ def test_host_tables_equal_oracle_tables(d, bits, seed):
     assert np.array_equal(t["bounds_v"], o.tV)
     assert np.array_equal(t["signs"], o.D)
     assert np.array_equal(t["S"].astype(np.float64), o.S)
+
+
+def test_k8v4_is_a_built_format_and_its_neighbours_are_not():
+    # (7, 4, 1) passes the format check (on a machine without a GPU the call then
+    # fails at the device, with another code); its near misses are refused first
+    h = ctypes.c_void_p()
+    rc = binding._lib.tq_init_ex(128, 7, 4, 1, 0, 1, ctypes.byref(h))
+    assert rc != tq.TQ_ERR_UNSUPPORTED
+    if rc == tq.TQ_OK:
+        binding._lib.tq_destroy(h)
+    for f in ((6, 4, 1), (7, 3, 1), (7, 4, 0), (8, 4, 1), (7, 2, 1)):
+        assert binding._lib.tq_init_ex(128, f[0], f[1], f[2], 0, 1, ctypes.byref(h)) == \
+            tq.TQ_ERR_UNSUPPORTED, f
+    for d in (64, 256):
+        rc = binding._lib.tq_init_ex(d, 7, 4, 1, 0, 1, ctypes.byref(h))
+        assert rc != tq.TQ_ERR_UNSUPPORTED
+        if rc == tq.TQ_OK:
+            binding._lib.tq_destroy(h)
