@@ -111,10 +111,21 @@ struct AttTraits {
     static constexpr int STAGE_BYTES = TILE_BYTES;
     static constexpr size_t RING_BYTES = (size_t)WARPS * STAGES * STAGE_BYTES;
     // dynamic shared memory: [K table][V table] (unless static), [ring, then the
-    // merge buffer], [query fragments]
+    // merge buffer], [query fragments]; with an aligned row table (below):
+    // [ring / merge buffer][query fragments] ... [row table at LUT_ADDR]
     static constexpr size_t BODY_BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
-    static constexpr size_t DYN_SMEM = (STATIC_LUT ? 0 : LUT_BYTES) + BODY_BYTES + QF_SMEM;
+    // The 64 KB row table sits at shared address LUT_ADDR (64 KB-aligned) when
+    // the ring, the merge buffer and the query fragments fit below it: the byte
+    // permute of row_off (or the OR of lut_off) then yields the entry's full
+    // shared address, and no lookup needs an add. (Measured: the adds were
+    // about 65 of 464 instructions per tile.) The dynamic region then reaches
+    // LUT_ADDR + 64 KB whatever the offset at which it starts.
+    static constexpr uint32_t LUT_ADDR = 0x20000u;
+    static constexpr bool ALIGNED = ROWS && !CK && WARPS == 16 && BODY_BYTES + QF_SMEM + 4096 <= LUT_ADDR;
+    static constexpr size_t DYN_SMEM =
+        ALIGNED ? (size_t)LUT_ADDR + 65536 : (STATIC_LUT ? 0 : LUT_BYTES) + BODY_BYTES + QF_SMEM;
     static_assert(LUT_BYTES + BODY_BYTES + QF_SMEM <= SMEM_CAP, "split CTA exceeds shared memory");
+    static_assert(DYN_SMEM <= SMEM_CAP, "split CTA exceeds shared memory");
     static constexpr int CTAS_PER_SM = 1;
 };
 
@@ -139,16 +150,25 @@ __device__ __forceinline__ uint32_t lut_off(const uint32_t* s, int pos, int F, u
 }
 
 // Offset of the row selected by byte r (0..3) of word w in a table of 256-byte
-// rows: w.byte[r] * 256 + 4 * lane, one byte permute (lane4 < 256 supplies
-// byte 0 and the zero bytes 2, 3).
+// rows: w.byte[r] * 256 + lane4, one byte permute: lane4 supplies bytes 0, 2
+// and 3 (4 * lane, plus the table's shared address when that is a multiple of
+// 64 KB, which makes the result the entry's full address).
 __device__ __forceinline__ uint32_t row_off(uint32_t w, int r, uint32_t lane4)
 {
-    return __byte_perm(w, lane4, 0x5504u | ((uint32_t)r << 4));
+    return __byte_perm(w, lane4, 0x7604u | ((uint32_t)r << 4));
 }
 
-__device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t byte_off)
+// A table entry: at `table` + x, or (ABS) at shared address x.
+template <bool ABS = false>
+__device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t x)
 {
-    return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(table) + byte_off);
+    if constexpr (ABS) {
+        uint32_t v;
+        asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(x));
+        return v;
+    } else {
+        return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const char*>(table) + x);
+    }
 }
 
 // fp16x2 (+-rho, +-rho) from sign pair p: element 0 at bit p%16, element 1 at
@@ -789,20 +809,20 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
         for (int r = 0; r < 4; ++r) {
             const int p = 4 * kk + r;
             if constexpr (Tr::PK) {
-                ak[r] = lut_load(lutk, row_off(td.s[kk], r, lane4));
+                ak[r] = lut_load<Tr::ALIGNED>(lutk, row_off(td.s[kk], r, lane4));
                 if constexpr (QJ) as[r] = sign_pair_byte(td.s[kk], r, (r & 1) ? nr_h : nr_g);
             } else if constexpr (Tr::CK) {
                 // one table row per code, {hi, lo} of its level: the pair's hi
                 // parts form the A fragment, its lo parts a second one
                 using Lay = TileLayout<D, KB, VB, QJ>;
-                const uint32_t e0 = lut_load(lutk, lut_off<8>(td.s, Lay::kbit(p, 0), KB, lane4));
-                const uint32_t e1 = lut_load(lutk, lut_off<8>(td.s, Lay::kbit(p, 1), KB, lane4));
+                const uint32_t e0 = lut_load<Tr::ALIGNED>(lutk, lut_off<8>(td.s, Lay::kbit(p, 0), KB, lane4));
+                const uint32_t e1 = lut_load<Tr::ALIGNED>(lutk, lut_off<8>(td.s, Lay::kbit(p, 1), KB, lane4));
                 ak[r] = __byte_perm(e0, e1, 0x5410u);
                 akl[r] = __byte_perm(e0, e1, 0x7632u);
                 if constexpr (QJ)
                     as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
             } else {
-                ak[r] = lut_load(lutk, lut_off<Tr::LSH>(td.s, Tr::KF * p, Tr::KF, lane4));
+                ak[r] = lut_load<Tr::ALIGNED>(lutk, lut_off<Tr::LSH>(td.s, Tr::KF * p, Tr::KF, lane4));
                 if constexpr (QJ)
                     as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
             }
@@ -884,9 +904,9 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, KB, VB, QJ>& t
         uint32_t av[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
-            av[r] = Tr::PV ? lut_load(lutv, row_off(td.s[Tr::VW0 + kk], r, lane4))
-                           : lut_load(lutv, lut_off<Tr::LSH>(td.s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
-                                                             Tr::VF, lane4));
+            av[r] = Tr::PV ? lut_load<Tr::ALIGNED>(lutv, row_off(td.s[Tr::VW0 + kk], r, lane4))
+                           : lut_load<Tr::ALIGNED>(lutv, lut_off<Tr::LSH>(td.s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
+                                                                          Tr::VF, lane4));
         mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0, b1);
     }
 }
@@ -934,6 +954,12 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
         lutk = s_lutk;
         lutv = s_lutv;
         body = reinterpret_cast<uint8_t*>(dyn_smem);
+    } else if constexpr (Tr::ALIGNED) {
+        // the row table at shared address LUT_ADDR, the ring and fragments below it
+        const uint32_t dyn_s = (uint32_t)__cvta_generic_to_shared(dyn_smem);
+        lutk = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(dyn_smem) + (Tr::LUT_ADDR - dyn_s));
+        lutv = lutk + 32;
+        body = reinterpret_cast<uint8_t*>(dyn_smem);
     } else {
         lutk = reinterpret_cast<uint32_t*>(dyn_smem);
         lutv = lutk + (Tr::ROWS ? 32 : Tr::NLK * 32);
@@ -960,7 +986,8 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     const int t_end = min(t_begin + a.plan.tps, a.plan.tiles);
     const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
                                          (size_t)a.tile_bytes;
-    const uint32_t lane4 = 4u * lane;
+    // table offsets of this lane (full shared addresses with an aligned table)
+    const uint32_t lane4 = (Tr::ALIGNED ? Tr::LUT_ADDR : 0u) + 4u * lane;
     const int ratio = a.Hq / a.Hkv;
     const int j0 = grp * 8 + 2 * t;
     TileData<D, KB, VB, QJ> td;
@@ -1015,6 +1042,12 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
         lutk = s_lutk;
         lutv = s_lutv;
         body = reinterpret_cast<uint8_t*>(dyn_smem);
+    } else if constexpr (Tr::ALIGNED) {
+        // the row table at shared address LUT_ADDR, the ring and fragments below it
+        const uint32_t dyn_s = (uint32_t)__cvta_generic_to_shared(dyn_smem);
+        lutk = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(dyn_smem) + (Tr::LUT_ADDR - dyn_s));
+        lutv = lutk + 32;
+        body = reinterpret_cast<uint8_t*>(dyn_smem);
     } else {
         lutk = reinterpret_cast<uint32_t*>(dyn_smem);
         lutv = lutk + (Tr::ROWS ? 32 : Tr::NLK * 32);
@@ -1030,7 +1063,10 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     const int groups = a.plan.groups, upb = a.Hkv * groups;
     // before the wait: only the constant tables and this CTA's own barriers
     fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
-    const uint32_t lane4 = 4u * lane;
+    // table offsets of this lane (full shared addresses with an aligned table,
+    // whose value entries follow the key entries of a row at + 128)
+    const uint32_t lane4 = (Tr::ALIGNED ? Tr::LUT_ADDR : 0u) + 4u * lane;
+    const uint32_t lane4v = lane4 + (Tr::ALIGNED ? 128u : 0u);
     uint8_t* ring = body + (size_t)w * S * Tr::STAGE_BYTES;
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
     const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(bars + w * S);
@@ -1131,7 +1167,7 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
             const bool v0 = tl * 16 + g < seq, v1 = tl * 16 + g + 8 < seq;
             if (!v0) L[0] = L[1] = -CUDART_INF_F;
             if (!v1) L[2] = L[3] = -CUDART_INF_F;
-            tile_accumulate<D, KB, VB, QJ>(td, L, v0, v1, lutv, lane4, st);
+            tile_accumulate<D, KB, VB, QJ>(td, L, v0, v1, lutv, lane4v, st);
         }
 
         float l0 = st.l0, l1 = st.l1;
