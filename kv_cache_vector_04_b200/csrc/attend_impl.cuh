@@ -1221,6 +1221,374 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
     }
 }
 
+// ---------------------------------------------------------------- split kernel, tile pairs
+// The same computation as attend_split, with each warp taking two consecutive
+// tiles per iteration: the query fragments of a k-step are read from shared
+// memory once for both tiles (half the shared-memory traffic they cost), the
+// two tiles' decode and MMA chains interleave, and one bulk copy brings in both
+// tiles. The row table sits at shared address LUT_ADDR = 64 KB, with the query
+// fragments and the rings of the first WA warps below it and the other rings
+// (and, after a segment, the merge buffer) above it.
+template <int D, int KB, int VB, int QJ>
+struct PairTraits {
+    using Tr = AttTraits<D, KB, VB, QJ>;
+    static constexpr uint32_t LUT_ADDR = 0x10000u;
+    static constexpr int WARPS = 16, NT = 32 * WARPS;
+    static constexpr int PSLOT = 2 * Tr::TILE_BYTES;      // one pair of tiles
+    static constexpr int RPW = 2 * PSLOT;                 // ring of one warp: two pair slots
+    static constexpr size_t QF = Tr::QF_SMEM;
+    static constexpr int WA_FIT = (int)((LUT_ADDR - 4096 - QF) / RPW);
+    static constexpr int WA = WA_FIT > WARPS ? WARPS : WA_FIT;   // rings below the table
+    static constexpr size_t MERGE = (size_t)WARPS * 8 * (D + 2) * 4;
+    static constexpr size_t ABOVE = (size_t)(WARPS - WA) * RPW > MERGE ? (size_t)(WARPS - WA) * RPW : MERGE;
+    static constexpr size_t DYN_SMEM = LUT_ADDR + 65536 + ABOVE;
+    static constexpr bool SUPPORTED =
+        Tr::ROWS && !Tr::CK && D <= 128 && WA >= 1 && DYN_SMEM <= Tr::SMEM_CAP && Tr::LUT_BYTES == 65536;
+    // lane-string words holding the key operands (codes and, byte-field keys, signs) and the values
+    static constexpr int KW0 = 0, KWN = Tr::PK ? Tr::KK : Tr::VW0;
+    static constexpr int VW0 = Tr::VW0, VWN = Tr::NWORDS - Tr::VW0;
+};
+
+// Words [W0, W0 + NW) of this lane's string in a tile image (chunk-major, CB-byte chunks).
+template <int CB, int W0, int NW, int CAP>
+__device__ __forceinline__ void stage_words(const uint8_t* slot, int lane, uint32_t (&s)[CAP])
+{
+    constexpr int CW = CB / 4;
+#pragma unroll
+    for (int c = W0 / CW; c * CW < W0 + NW; ++c) {
+        const uint8_t* src = slot + (c * 32 + lane) * CB;
+        uint32_t v[CW];
+        if constexpr (CB == 16) {
+            const uint4 x = *reinterpret_cast<const uint4*>(src);
+            v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+        } else if constexpr (CB == 8) {
+            const uint2 x = *reinterpret_cast<const uint2*>(src);
+            v[0] = x.x; v[1] = x.y;
+        } else {
+            v[0] = *reinterpret_cast<const uint32_t*>(src);
+        }
+#pragma unroll
+        for (int i = 0; i < CW; ++i)
+            if (c * CW + i >= W0 && c * CW + i < W0 + NW) s[c * CW + i] = v[i];
+    }
+}
+
+// Logits of two tiles (log2 units) for tokens g, g+8 and heads 2t, 2t+1; the
+// query fragments of each k-step serve both tiles.
+template <int D, int KB, int VB, int QJ, typename QF>
+__device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[2], const QF& qf, int lane,
+                                            const uint32_t* lutk, uint32_t lane4, float (&L)[2][4])
+{
+    using Tr = AttTraits<D, KB, VB, QJ>;
+    uint32_t nr_g[2], nr_h[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        nr_g[u] = QJ ? (__byte_perm(td[u].kn.x, 0u, 0x3232) | 0x80008000u) : 0u;
+        nr_h[u] = QJ ? (__byte_perm(td[u].kn.y, 0u, 0x3232) | 0x80008000u) : 0u;
+    }
+    float ah[2][4], al[2][4];
+#pragma unroll
+    for (int kk = 0; kk < Tr::KK; ++kk) {
+        const uint4 bc = qf.fc(kk, lane);
+        uint4 bs;
+        if constexpr (QJ) bs = qf.fs(kk, lane);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            uint32_t ak[4], as[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int p = 4 * kk + r;
+                if constexpr (Tr::PK) {
+                    ak[r] = lut_load<true>(lutk, row_off(td[u].s[kk], r, lane4));
+                    if constexpr (QJ) as[r] = sign_pair_byte(td[u].s[kk], r, (r & 1) ? nr_h[u] : nr_g[u]);
+                } else {
+                    ak[r] = lut_load<true>(lutk, lut_off<Tr::LSH>(td[u].s, Tr::KF * p, Tr::KF, lane4));
+                    if constexpr (QJ)
+                        as[r] = sign_pair(td[u].s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h[u] : nr_g[u]);
+                }
+            }
+            if (kk == 0) {
+                mma_16816_first(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
+                mma_16816_first(al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+            } else {
+                mma_16816(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
+                mma_16816(al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+            }
+            if constexpr (QJ) {
+                mma_16816(ah[u], as[0], as[1], as[2], as[3], bs.x, bs.y);
+                mma_16816(al[u], as[0], as[1], as[2], as[3], bs.z, bs.w);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        float kn_g, kn_h;
+        if constexpr (QJ) {
+            kn_g = __low2float(*reinterpret_cast<const __half2*>(&td[u].kn.x)) * (1.0f / 128.0f);
+            kn_h = __low2float(*reinterpret_cast<const __half2*>(&td[u].kn.y)) * (1.0f / 128.0f);
+        } else {
+            const float2 kk2 = __half22float2(*reinterpret_cast<const __half2*>(&td[u].kn.x));
+            kn_g = kk2.x * (1.0f / 128.0f);
+            kn_h = kk2.y * (1.0f / 128.0f);
+        }
+        L[u][0] = kn_g * (ah[u][0] + al[u][0]);
+        L[u][1] = kn_g * (ah[u][1] + al[u][1]);
+        L[u][2] = kn_h * (ah[u][2] + al[u][2]);
+        L[u][3] = kn_h * (ah[u][3] + al[u][3]);
+    }
+}
+
+// Online-softmax update and P V for two tiles (one running-maximum check for both).
+template <int D, int KB, int VB, int QJ>
+__device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&td)[2], float (&L)[2][4],
+                                                const bool (&v)[2][2], uint32_t lane4v, SplitState<D>& st)
+{
+    using Tr = AttTraits<D, KB, VB, QJ>;
+    const bool above = (L[0][0] > st.m0) || (L[0][2] > st.m0) || (L[0][1] > st.m1) || (L[0][3] > st.m1) ||
+                       (L[1][0] > st.m0) || (L[1][2] > st.m0) || (L[1][1] > st.m1) || (L[1][3] > st.m1);
+    if (__any_sync(kFull, above)) {
+        float mx0 = fmaxf(fmaxf(L[0][0], L[0][2]), fmaxf(L[1][0], L[1][2]));
+        float mx1 = fmaxf(fmaxf(L[0][1], L[0][3]), fmaxf(L[1][1], L[1][3]));
+#pragma unroll
+        for (int sh = 4; sh <= 16; sh <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
+        }
+        const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+        const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
+        st.l0 *= al0;
+        st.l1 *= al1;
+#pragma unroll
+        for (int kk = 0; kk < Tr::KK; ++kk) {
+            st.acc[kk][0] *= al0;
+            st.acc[kk][1] *= al1;
+            st.acc[kk][2] *= al0;
+            st.acc[kk][3] *= al1;
+        }
+        st.m0 = mn0;
+        st.m1 = mn1;
+    }
+    uint32_t b0[2], b1[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const float p0 = fast_exp2(L[u][0] - st.m0), p1 = fast_exp2(L[u][1] - st.m1);
+        const float p2 = fast_exp2(L[u][2] - st.m0), p3 = fast_exp2(L[u][3] - st.m1);
+        st.l0 += p0 + p2;
+        st.l1 += p1 + p3;
+        // slots past seq_len may hold anything (even NaN norms): select, never multiply
+        const float2 vnf = __half22float2(*reinterpret_cast<const __half2*>(&td[u].vn));
+        const float vn_g = v[u][0] ? vnf.x : 0.f;
+        const float vn_h = v[u][1] ? vnf.y : 0.f;
+        b0[u] = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
+        b1[u] = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
+    }
+#pragma unroll
+    for (int kk = 0; kk < Tr::KK; ++kk) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            uint32_t av[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                av[r] = Tr::PV ? lut_load<true>(nullptr, row_off(td[u].s[Tr::VW0 + kk], r, lane4v))
+                               : lut_load<true>(nullptr, lut_off<Tr::LSH>(td[u].s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
+                                                                          Tr::VF, lane4v));
+            mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0[u], b1[u]);
+        }
+    }
+}
+
+template <int D, int KB, int VB, int QJ>
+__global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split2(DevTables tb, AttendArgs a)
+{
+    using Tr = AttTraits<D, KB, VB, QJ>;
+    using P2 = PairTraits<D, KB, VB, QJ>;
+    constexpr int KK = Tr::KK, WARPS = P2::WARPS, NT = P2::NT, TB = Tr::TILE_BYTES, CB = Tr::CB;
+    constexpr int RS = D + 2;
+    __shared__ __align__(8) uint64_t bars[WARPS * 2];   // one mbarrier per pair slot
+    extern __shared__ uint4 dyn_smem[];
+    uint8_t* dyn = reinterpret_cast<uint8_t*>(dyn_smem);
+    const uint32_t dyn_s = (uint32_t)__cvta_generic_to_shared(dyn_smem);
+    uint32_t* lutk = reinterpret_cast<uint32_t*>(dyn + (P2::LUT_ADDR - dyn_s));
+    uint32_t* lutv = lutk + 32;
+    uint8_t* above = dyn + (P2::LUT_ADDR + 65536 - dyn_s);
+    uint4* qsm = reinterpret_cast<uint4*>(dyn);
+    float* mrg = reinterpret_cast<float*>(above);         // [WARPS][8][D+2] after a segment
+
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int c = blockIdx.x;
+    const long long G = gridDim.x;
+    const int groups = a.plan.groups, upb = a.Hkv * groups;
+    fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
+    // full shared addresses of this lane's table entries (value entries at + 128 in a row)
+    const uint32_t lane4 = P2::LUT_ADDR + 4u * lane, lane4v = lane4 + 128u;
+    uint8_t* ring = w < P2::WA ? dyn + P2::QF + (size_t)w * P2::RPW : above + (size_t)(w - P2::WA) * P2::RPW;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(bars + w * 2);
+    if (lane == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_s + 8, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    pdl_trigger();
+    pdl_wait();   // the prologue's prefix and query fragments are complete from here on
+    const long long W = a.prefix[a.B];
+    const long long x0 = (long long)c * W / G, x1 = (long long)(c + 1) * W / G;
+    if (x0 >= x1) return;   // an empty range (fewer tiles than CTAs): uniform, before any barrier
+    const int lim = min(a.max_len, a.capacity);
+    // Pair copies this warp has issued / waited for (warp-uniform): copy n uses
+    // slot n % 2 and completes phase (n / 2) & 1 of that slot's barrier.
+    uint32_t issued = 0, consumed = 0;
+    bool stalled = false;
+    QueryFrags<KK, NT> qf;
+
+    long long x = x0;
+#pragma unroll 1
+    while (x < x1) {
+        int b = 0;
+        {
+            int hi = a.B - 1;
+            while (b < hi) {
+                const int mid = (b + hi + 1) >> 1;
+                if (a.prefix[mid] <= x) b = mid; else hi = mid - 1;
+            }
+        }
+        const long long pb = a.prefix[b];
+        const long long T = (a.prefix[b + 1] - pb) / upb;
+        const int j = (int)((x - pb) / T);
+        const long long U0 = pb + (long long)j * T;
+        const int sb = (int)(x - U0);
+        const int se = (int)min(T, x1 - U0);
+        const int seq = min(max(a.seq_len[b], 0), lim);
+        const int hkv = j / groups;
+        const size_t u = (size_t)b * upb + j;
+        qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
+        __syncthreads();   // tables (first segment) and query fragments visible
+
+        const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
+                                             (size_t)a.tile_bytes;
+        SplitState<D> st;
+        st.m0 = st.m1 = -CUDART_INF_F;
+        st.l0 = st.l1 = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
+
+        // pair p of the segment: tiles sb + 2p and sb + 2p + 1 (the last pair may hold one)
+        const int ntile = se - sb, npair = (ntile + 1) >> 1;
+        fence_proxy_async();
+        if (!stalled && w < npair) {
+            if (lane == 0) {
+                const int n = min(2, ntile - 2 * w);
+                const uint32_t sl = issued & 1u;
+                bulk_load(ring_s + sl * P2::PSLOT, sbase + (size_t)(sb + 2 * w) * TB, (uint32_t)(n * TB),
+                          bar_s + 8 * sl);
+            }
+            ++issued;
+        }
+        TileData<D, KB, VB, QJ> td[2];
+#pragma unroll 1
+        for (int p = w; p < npair && !stalled; p += WARPS) {
+            const int pn = p + WARPS;
+            if (pn < npair) {
+                fence_proxy_async();
+                if (lane == 0) {
+                    const int n = min(2, ntile - 2 * pn);
+                    const uint32_t sl = issued & 1u;
+                    bulk_load(ring_s + sl * P2::PSLOT, sbase + (size_t)(sb + 2 * pn) * TB, (uint32_t)(n * TB),
+                              bar_s + 8 * sl);
+                }
+                ++issued;
+            }
+            const uint32_t slot = consumed & 1u;
+            if (!mbar_wait(bar_s + 8 * slot, (consumed >> 1) & 1u)) {
+                stalled = true;
+                if (lane == 0) atomicOr(tb.status, TQ_STATUS_WAIT_TIMEOUT);
+                break;
+            }
+            ++consumed;
+            const uint8_t* sp = ring + slot * P2::PSLOT;
+            const int tl0 = sb + 2 * p;
+            const bool two = 2 * p + 1 < ntile;
+            // key words and norms of both tiles (a missing second tile reads stale
+            // bytes of the slot: every table index stays in range and it is masked)
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu) {
+                const uint8_t* tp = sp + uu * TB;
+                stage_words<CB, P2::KW0, P2::KWN, Tr::NWORDS>(tp, lane, td[uu].s);
+                if constexpr (QJ)
+                    td[uu].kn = *reinterpret_cast<const uint2*>(tp + Tr::CODE_BYTES + 8 * g);
+                else
+                    td[uu].kn.x = *reinterpret_cast<const uint32_t*>(tp + Tr::CODE_BYTES + 4 * g);
+                td[uu].vn = *reinterpret_cast<const uint32_t*>(tp + Tr::CODE_BYTES + Tr::KNB + 4 * g);
+            }
+            float L[2][4];
+            pair_logits<D, KB, VB, QJ>(td, qf, lane, lutk, lane4, L);
+            bool v[2][2];
+            v[0][0] = tl0 * 16 + g < seq;
+            v[0][1] = tl0 * 16 + g + 8 < seq;
+            v[1][0] = two && (tl0 + 1) * 16 + g < seq;
+            v[1][1] = two && (tl0 + 1) * 16 + g + 8 < seq;
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu) {
+                if (!v[uu][0]) L[uu][0] = L[uu][1] = -CUDART_INF_F;
+                if (!v[uu][1]) L[uu][2] = L[uu][3] = -CUDART_INF_F;
+                stage_words<CB, P2::VW0, P2::VWN, Tr::NWORDS>(sp + uu * TB, lane, td[uu].s);
+            }
+            pair_accumulate<D, KB, VB, QJ>(td, L, v, lane4v, st);
+        }
+
+        float l0 = st.l0, l1 = st.l1;
+#pragma unroll
+        for (int sh = 4; sh <= 16; sh <<= 1) {
+            l0 += __shfl_xor_sync(kFull, l0, sh);
+            l1 += __shfl_xor_sync(kFull, l1, sh);
+        }
+        fence_proxy_async();
+        __syncthreads();   // every warp is done with its ring: reuse the upper rings for the merge
+        float* mw = mrg + (size_t)w * 8 * RS;
+        if (g == 0) {
+            mw[(2 * t) * RS] = st.m0;
+            mw[(2 * t) * RS + 1] = l0;
+            mw[(2 * t + 1) * RS] = st.m1;
+            mw[(2 * t + 1) * RS + 1] = l1;
+        }
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) {
+            mw[(2 * t) * RS + 2 + 16 * kk + g] = st.acc[kk][0];
+            mw[(2 * t + 1) * RS + 2 + 16 * kk + g] = st.acc[kk][1];
+            mw[(2 * t) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][2];
+            mw[(2 * t + 1) * RS + 2 + 16 * kk + g + 8] = st.acc[kk][3];
+        }
+        __syncthreads();
+        float* dst = a.partial + ((size_t)c + u) * 8 * RS;
+        for (int e = tid; e < 8 * RS; e += NT) {
+            const int head = e / RS, col = e % RS;
+            float M = -CUDART_INF_F;
+#pragma unroll
+            for (int ww = 0; ww < WARPS; ++ww) M = fmaxf(M, mrg[(ww * 8 + head) * RS]);
+            float sum = 0.f;
+            if (col == 0) {
+                sum = M;
+            } else {
+#pragma unroll
+                for (int ww = 0; ww < WARPS; ++ww) {
+                    const float mwv = mrg[(ww * 8 + head) * RS];
+                    if (mwv != -CUDART_INF_F) sum += mrg[(ww * 8 + head) * RS + col] * exp2f(mwv - M);
+                }
+            }
+            dst[e] = sum;
+        }
+        __syncthreads();   // merge buffer and query fragments free for the next segment
+        x = U0 + se;
+    }
+    // after a wait ran out: wait (bounded) for this warp's copies still in flight
+    while (consumed < issued) {
+        if (!mbar_wait(bar_s + 8 * (consumed & 1u), (consumed >> 1) & 1u)) break;
+        ++consumed;
+    }
+}
+
 // cudaFuncSetAttribute once per (kernel, device).
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes, unsigned long long& done_mask)
@@ -1279,11 +1647,20 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
             e = launch_pdl(kern, dim3(a.plan.nsplit, units, a.B), dim3(Tr::NT), Tr::DYN_SMEM, st, tb, a);
         return e;
     }
-    auto kern = attend_split<D, KB, VB, QJ>;
-    if ((e = allow_smem(kern, Tr::DYN_SMEM, done_attend)) != cudaSuccess) return e;
-    if (a.plan.tiles > 0 &&
-        (e = launch_pdl(kern, dim3(a.plan.ctas), dim3(Tr::NT), Tr::DYN_SMEM, st, tb, a)) != cudaSuccess)
-        return e;
+    if constexpr (PairTraits<D, KB, VB, QJ>::SUPPORTED) {
+        using P2 = PairTraits<D, KB, VB, QJ>;
+        auto kern = attend_split2<D, KB, VB, QJ>;
+        if ((e = allow_smem(kern, P2::DYN_SMEM, done_attend)) != cudaSuccess) return e;
+        if (a.plan.tiles > 0 &&
+            (e = launch_pdl(kern, dim3(a.plan.ctas), dim3(P2::NT), P2::DYN_SMEM, st, tb, a)) != cudaSuccess)
+            return e;
+    } else {
+        auto kern = attend_split<D, KB, VB, QJ>;
+        if ((e = allow_smem(kern, Tr::DYN_SMEM, done_attend)) != cudaSuccess) return e;
+        if (a.plan.tiles > 0 &&
+            (e = launch_pdl(kern, dim3(a.plan.ctas), dim3(Tr::NT), Tr::DYN_SMEM, st, tb, a)) != cudaSuccess)
+            return e;
+    }
     return launch_pdl(attend_reduce<D>, dim3(a.Hq, a.B), dim3(D), 0, st, tb, a);
 }
 
