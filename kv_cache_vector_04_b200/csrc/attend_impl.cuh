@@ -1226,9 +1226,10 @@ __global__ void __launch_bounds__(AttTraits<D, KB, VB, QJ>::NT, AttTraits<D, KB,
 // tiles per iteration: the query fragments of a k-step are read from shared
 // memory once for both tiles (half the shared-memory traffic they cost), the
 // two tiles' decode and MMA chains interleave, and one bulk copy brings in both
-// tiles. The row table sits at shared address LUT_ADDR = 64 KB, with the query
-// fragments and the rings of the first WA warps below it and the other rings
-// (and, after a segment, the merge buffer) above it.
+// tiles. The decode tables sit in a 64 KB region at shared address LUT_ADDR =
+// 64 KB, with the query fragments and the rings of the first WA warps below it
+// and the other rings (and, after a segment, the merge buffer) above it; every
+// table lookup address is then one byte permute or one OR.
 template <int D, int KB, int VB, int QJ>
 struct PairTraits {
     using Tr = AttTraits<D, KB, VB, QJ>;
@@ -1242,8 +1243,13 @@ struct PairTraits {
     static constexpr size_t MERGE = (size_t)WARPS * 8 * (D + 2) * 4;
     static constexpr size_t ABOVE = (size_t)(WARPS - WA) * RPW > MERGE ? (size_t)(WARPS - WA) * RPW : MERGE;
     static constexpr size_t DYN_SMEM = LUT_ADDR + 65536 + ABOVE;
-    static constexpr bool SUPPORTED =
-        Tr::ROWS && !Tr::CK && D <= 128 && WA >= 1 && DYN_SMEM <= Tr::SMEM_CAP && Tr::LUT_BYTES == 65536;
+    static constexpr bool SUPPORTED = !Tr::CK && D <= 128 && WA >= 1 && DYN_SMEM <= Tr::SMEM_CAP;
+    // the value table: in the key table's rows (+ 128 bytes) for the 256-row
+    // table; else its own table at LUT_ADDR + 32 KB (aligned above its size, so
+    // an OR with a field offset still yields a full address)
+    static constexpr uint32_t V_OFF = Tr::ROWS ? 128u : 0x8000u;
+    static_assert(Tr::ROWS || ((size_t)Tr::NLK * 128 <= 0x8000 && (size_t)Tr::NLV * 128 <= 0x8000),
+                  "small tables fit their 32 KB halves");
     // lane-string words holding the key operands (codes and, byte-field keys, signs) and the values
     static constexpr int KW0 = 0, KWN = Tr::PK ? Tr::KK : Tr::VW0;
     static constexpr int VW0 = Tr::VW0, VWN = Tr::NWORDS - Tr::VW0;
@@ -1409,7 +1415,7 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
     uint8_t* dyn = reinterpret_cast<uint8_t*>(dyn_smem);
     const uint32_t dyn_s = (uint32_t)__cvta_generic_to_shared(dyn_smem);
     uint32_t* lutk = reinterpret_cast<uint32_t*>(dyn + (P2::LUT_ADDR - dyn_s));
-    uint32_t* lutv = lutk + 32;
+    uint32_t* lutv = lutk + P2::V_OFF / 4;
     uint8_t* above = dyn + (P2::LUT_ADDR + 65536 - dyn_s);
     uint4* qsm = reinterpret_cast<uint4*>(dyn);
     float* mrg = reinterpret_cast<float*>(above);         // [WARPS][8][D+2] after a segment
@@ -1420,8 +1426,8 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
     const long long G = gridDim.x;
     const int groups = a.plan.groups, upb = a.Hkv * groups;
     fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
-    // full shared addresses of this lane's table entries (value entries at + 128 in a row)
-    const uint32_t lane4 = P2::LUT_ADDR + 4u * lane, lane4v = lane4 + 128u;
+    // full shared addresses of this lane's table entries
+    const uint32_t lane4 = P2::LUT_ADDR + 4u * lane, lane4v = lane4 + P2::V_OFF;
     uint8_t* ring = w < P2::WA ? dyn + P2::QF + (size_t)w * P2::RPW : above + (size_t)(w - P2::WA) * P2::RPW;
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
     const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(bars + w * 2);
