@@ -49,6 +49,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-graph", action="store_true",
                     help="time the eager launch loop only (no CUDA graph of the step)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other long-context workloads reported beside the bench line")
     ap.add_argument("--report", choices=["all", "single", "qwen3b", "qwen32b", "sweep", "formats"],
                     default=None,
                     help="measure the other workloads instead of the bench line: one JSON line each")
@@ -167,25 +169,24 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attend_split_llama70b_32k.json")
+
+
 def profiled_traffic(workload: str):
-    """DRAM bytes per attend_split launch from the committed ncu summary, if it
-    was taken on this workload and on the kernel source as it is now (else None)."""
+    """DRAM bytes (read + write) per split-kernel launch, from the data file
+    written beside the ncu summary of this workload's capture, if it was taken
+    on the attention source as it is now (else None)."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "attend_split_llama70b_32k.md")
     src = os.path.join(ROOT, "kv_cache_vector_04_b200", "csrc", "attend_impl.cuh")
-    if workload != DEFAULT_WORKLOAD or not os.path.exists(prof):
+    if workload != DEFAULT_WORKLOAD or not os.path.exists(TRAFFIC_FILE):
         return None
-    fields = {}
-    for line in open(prof, encoding="utf-8"):
-        if ":" in line and line.split(":", 1)[0].strip() in ("kernel_source_sha1",
-                                                             "dram_bytes_per_launch"):
-            key, val = line.split(":", 1)
-            fields[key.strip()] = val.split()[0]
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f)
     with open(src, "rb") as f:
         sha = hashlib.sha1(f.read()).hexdigest()
-    if fields.get("kernel_source_sha1") != sha or "dram_bytes_per_launch" not in fields:
+    if rec.get("kernel_source_sha1") != sha or rec.get("workload") != workload:
         return None
-    return int(fields["dram_bytes_per_launch"])
+    return int(rec["dram_bytes_per_launch"])
 
 
 def measured_peaks():
@@ -199,40 +200,85 @@ def measured_peaks():
 
 # ---------------------------------------------------------------- CPU oracle sample
 
-def cpu_oracle_sample(w, seconds: float, streams: int = 4, N: int | None = None):
-    """Time the fp64 oracle's decode attention on `streams` (batch, kv-head)
-    streams of the workload (all their query heads, full context), repeated
-    until about `seconds` of work. Returns (GB/s, description, threads)."""
-    import numpy as np
-    import torch
-    from kv_cache_vector_04_b200 import inputs
-    from oracle import oracle as O
+class OracleSample:
+    """The fp64 oracle's decode attention over `streams` (batch, kv-head)
+    streams of the workload (all their query heads, N tokens each): the codes
+    are computed once, then timed repeatedly."""
 
-    N = w.N if N is None else N
-    tab = O.Tables(w.d, w.bits, 1)
-    g = w.Hq // w.Hkv
-    k, v = inputs.kv_pair(w, N, layer=0, device="cpu", B=1, Hkv=streams)
-    codes = [[O.quantize(tab, k[0, h].numpy(), v[0, h].numpy()) for h in range(streams)]]
-    cap = N
-    st = {}
-    for key in ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm"):
-        st[key] = np.stack([c[key] for c in codes[0]])[None]
-    q = inputs.queries(w, B=1, Hq=streams * g)
-    qb = q.contiguous().view(torch.int16).numpy().view(np.uint16)
-    seq = np.array([N], np.int32)
-    reps, t_total = 0, 0.0
-    while t_total < seconds or reps == 0:
-        t0 = time.perf_counter()
-        O.attend_batch(tab, qb, w.q_dtype == torch.bfloat16, st, seq, streams)
-        t_total += time.perf_counter() - t0
-        reps += 1
-    bytes_per_rep = streams * N * (w.bits * w.d // 4 + 6)
-    gbs = bytes_per_rep * reps / t_total / 1e9
+    def __init__(self, w, streams: int = 4, N: int | None = None):
+        import numpy as np
+        import torch
+        from kv_cache_vector_04_b200 import inputs
+        from oracle import oracle as O
+        self.O, self.np = O, np
+        self.N = w.N if N is None else N
+        self.streams = streams
+        self.tab = O.Tables(w.d, w.bits, 1, fmt=w.fmt) if w.fmt is not None else O.Tables(w.d, w.bits, 1)
+        g = w.Hq // w.Hkv
+        k, v = inputs.kv_pair(w, self.N, layer=0, device="cpu", B=1, Hkv=streams)
+        codes = [O.quantize(self.tab, k[0, h].numpy(), v[0, h].numpy()) for h in range(streams)]
+        self.st = {key: np.stack([c[key] for c in codes])[None]
+                   for key in ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm")}
+        q = inputs.queries(w, B=1, Hq=streams * g)
+        self.qb = q.contiguous().view(torch.int16).numpy().view(np.uint16)
+        self.q_bf16 = w.q_dtype == torch.bfloat16
+        self.seq = np.array([self.N], np.int32)
+        self.bytes_per_rep = streams * self.N * bytes_per_head_token(w)
+        self.g = g
+
+    def run(self, seconds: float):
+        """Repeat the attention until about `seconds` of work; (GB/s, seconds per rep)."""
+        reps, t_total = 0, 0.0
+        while t_total < seconds or reps == 0:
+            t0 = time.perf_counter()
+            self.O.attend_batch(self.tab, self.qb, self.q_bf16, self.st, self.seq, self.streams)
+            t_total += time.perf_counter() - t0
+            reps += 1
+        self.last = (reps, t_total)
+        return self.bytes_per_rep * reps / t_total / 1e9, t_total / reps
+
+    def describe(self) -> str:
+        reps, t_total = self.last
+        return ("fp64 C oracle decode attention over %d (batch, kv-head) streams x %d query heads x "
+                "%d tokens of layer 0, %d repetitions in %.1f s (append of one token excluded: "
+                "<0.01%% of the step)" % (self.streams, self.g, self.N, reps, t_total))
+
+
+def cpu_oracle_sample(w, seconds: float, streams: int = 4, N: int | None = None):
+    """Time the oracle on a bounded sample: (GB/s, description, threads, seconds per rep)."""
+    smp = OracleSample(w, streams, N)
+    gbs, per = smp.run(seconds)
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    desc = ("fp64 C oracle decode attention over %d (batch, kv-head) streams x %d query heads x "
-            "%d tokens of layer 0, %d repetitions in %.1f s (append of one token excluded: "
-            "<0.01%% of the step)" % (streams, g, N, reps, t_total))
-    return gbs, desc, threads, t_total / reps
+    return gbs, smp.describe(), threads, per
+
+
+# ---------------------------------------------------------------- workload description
+
+def fmt_of(w):
+    """(B_K, B_V, qjl) of a workload: its named format, else TurboQuant at w.bits."""
+    return tuple(w.fmt) if w.fmt is not None else (w.bits - 1, w.bits, 1)
+
+
+def bytes_per_head_token(w) -> int:
+    """Packed K + V bytes of one (token, kv head): codes, signs and fp16 norms
+    (the tile layout of include/tq.h, per token)."""
+    kb, vb, qjl = fmt_of(w)
+    return ((kb + qjl) * w.d // 8 + 2 + 2 * qjl) + (vb * w.d // 8 + 2)
+
+
+def workload_config(w, layers: int, world: int) -> dict:
+    """The `config` of a bench line: the workload as both arms run it (the
+    context includes the decode step's appended token)."""
+    N = w.N
+    per_tok = bytes_per_head_token(w)
+    layer_bytes = w.B * w.Hkv * (N + 1) * per_tok
+    return {"workload": w.name, "layers": layers, "batch": w.B, "q_heads": w.Hq,
+            "kv_heads": w.Hkv, "head_dim": w.d, "bits": w.bits, "context": N + 1,
+            "format": list(fmt_of(w)),
+            "packed_cache_gb": round(layers * w.B * w.Hkv * (N + 16) * per_tok / 1e9, 2),
+            "step": "per layer: tq_append_attend (append 1 token, then attend)",
+            "l2": l2_note(layers * layer_bytes, layer_bytes),
+            "parallelism": "replicas x%d (weak)" % world}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -258,6 +304,7 @@ def run_tq(args, dist: Dist):
     ctx = tq.tq_init(w.d, w.bits, 1) if w.fmt is None else tq.tq_init_ex(w.d, *w.fmt, 1)
     lay = tq.tq_cache_layout(ctx)
     per_tok = lay["tile_bytes"] // 16                     # K + V bytes per head-token
+    assert per_tok == bytes_per_head_token(w), (per_tok, bytes_per_head_token(w))
     N = w.N
     cap = N + 16
     zeros = torch.zeros(w.B, dtype=torch.int32, device=dev)
@@ -460,14 +507,8 @@ def run_tq(args, dist: Dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 tensor-core operands, f32 accumulate (codes u2-u4)",
         "data": "synthetic",
-        "config": {"workload": w.name, "layers": layers, "batch": w.B, "q_heads": w.Hq,
-                   "kv_heads": w.Hkv, "head_dim": w.d, "bits": w.bits, "context": N + 1,
-                   "format": list(tq.tq_cache_layout(ctx)[k] for k in ("kbits", "vbits", "qjl")),
-                   "packed_cache_gb": round(layers * w.B * w.Hkv * cap * per_tok / 1e9, 2),
-                   "step": "per layer: tq_append_attend (append 1 token, then attend)",
-                   "step_launch": "one CUDA graph per step" if ms_graph is not None else "eager",
-                   "l2": l2_note(layers * bytes_attend, bytes_attend),
-                   "parallelism": "replicas x%d (weak)" % dist.world},
+        "config": dict(workload_config(w, layers, dist.world),
+                       step_launch="one CUDA graph per step" if ms_graph is not None else "eager"),
         "pct_of_hbm_peak": round(100.0 * value / dist.world / peak, 1),
         "ms_per_step_eager": round(ms_eager, 4),
         "ms_per_step_graph": round(ms_graph, 4) if ms_graph is not None else None,
@@ -477,9 +518,9 @@ def run_tq(args, dist: Dist):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 3), "peak_kind": peak_kind,
                      "traffic": profiled_traffic(w.name),
-                     "traffic_note": "dram read+write bytes of one attend_split launch (ncu, "
-                                     "profiles/attend_split_llama70b_32k.md); null when the "
-                                     "kernel source changed since",
+                     "traffic_note": "dram read+write bytes of one split-kernel launch of this "
+                                     "workload from an ncu capture; null when the attention "
+                                     "source changed since",
                      "algorithmic_bytes_per_launch": bytes_attend,
                      "frac_of_same_run_copy_kernel": round(achieved / copy_gbs, 3)},
         "copy_kernel_gbs": round(copy_gbs, 1),
@@ -489,7 +530,7 @@ def run_tq(args, dist: Dist):
         "e2e": e2e,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        gbs, desc, threads, _ = cpu_oracle_sample(w, args.cpu_seconds)
+        gbs, desc, threads, _ = cpu_oracle_sample(w, args.cpu_seconds, N=N + 1)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
                                 "kind": "oracle", "sample": desc}
     for L in range(layers):
@@ -499,25 +540,27 @@ def run_tq(args, dist: Dist):
 
 def run_reference(args, dist: Dist):
     """The fp64 CPU oracle as the reference arm: each step is a bounded sample
-    (2 streams of the workload) of oracle decode attention."""
-    import torch
+    (about half a second: 4 (batch, kv head) streams of the workload over the
+    same context as the GPU arm, N + 1 tokens) of oracle decode attention."""
     from kv_cache_vector_04_b200 import inputs
     w = inputs.WORKLOADS[args.workload]
     if dist.rank != 0:
         return None
+    smp = OracleSample(w, streams=4, N=w.N + 1)
     times = []
-    desc = threads = None
     for i in range(args.warmup + args.steps):
-        gbs, desc, threads, t = cpu_oracle_sample(w, 0.0, streams=2)
+        gbs, _ = smp.run(0.5)
         if i >= args.warmup:
             times.append(gbs)
     value = statistics.mean(times)
+    desc = smp.describe() + "; %d timed steps of ~0.5 s, mean GB/s" % args.steps
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    layers = getattr(args, "layers", None) or w.layers
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
             "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv,
-                       "head_dim": w.d, "bits": w.bits, "context": w.N},
+            "config": dict(workload_config(w, layers, dist.world), step_launch="one CUDA graph per step"),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -622,6 +665,34 @@ def run_report(args, dist: Dist):
                                                          warmup=3))), flush=True)
 
 
+def secondary_workloads(args, dist: Dist) -> dict:
+    """The other long-context workloads, measured after the bench line's own
+    timed region and reported beside it: one layer of the Qwen2.5-32B-shaped
+    128K decode (32 timed steps) and the nine sweep points at 65536 tokens.
+    Each entry carries its own clock sample."""
+    from kv_cache_vector_04_b200 import inputs
+    base = dict(vars(args))
+    base.update(no_cpu_baseline=True, no_e2e=True, no_graph=False)
+
+    def run(**kw):
+        line = run_tq(argparse.Namespace(**dict(base, **kw)), dist)
+        return {"format": line["config"]["format"], "context": line["config"]["context"],
+                "ms_per_layer": line["ms_per_layer"], "packed_gbs": line["value"],
+                "attend_gbs": line["roofline"]["achieved"], "attend_frac": line["roofline"]["frac"],
+                "quantize_mtok_s": (line.get("quantize") or {}).get("value"),
+                "clocks": {"sm_mhz": line["clocks"].get("sm_mhz"),
+                           "reasons": line["clocks"].get("reasons")}}
+
+    out = {"note": "one layer each, step as one CUDA graph; attend_* from per-call events "
+                   "(prologue with the append + split + reduce); frac of the measured HBM peak"}
+    out["qwen2.5-32b_prefill_decode_128k"] = run(workload="qwen2.5-32b_prefill_decode_128k",
+                                                 layers=1, steps=32, warmup=3)
+    for w in inputs.sweep_workloads():
+        if w.N == 65536:
+            out[w.name] = run(workload=w.name, layers=1, steps=10, warmup=3)
+    return out
+
+
 def main(argv=None):
     args = parse_args(argv)
     dist = Dist()
@@ -641,6 +712,11 @@ def main(argv=None):
     dist.init()
     try:
         line = run_tq(args, dist)
+        if (dist.world == 1 and args.workload == DEFAULT_WORKLOAD and args.layers is None
+                and not args.no_secondary):
+            import torch
+            torch.cuda.empty_cache()
+            line["secondary"] = secondary_workloads(args, dist)
         if dist.rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -247,18 +247,20 @@ int tq_scores(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_c
               size_t workspace_bytes, void* stream);
 
 /* tq_attend without a workspace argument, for callers that cannot allocate
- * device memory: code running during CUDA-graph stream capture, runtimes whose
- * device memory belongs to an allocator they do not control, and serving
- * loops that forbid allocation after start-up. (The pages describe no such
- * call; it is an addition of this library.) The scratch is a static device
- * array of TQ_NOALLOC_SCRATCH_BYTES that exists on every GPU that loads the
- * library until the process exits; calls needing more (tq_attend_workspace)
- * return TQ_ERR_WORKSPACE without launching anything. The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current: make that first call before any stream capture. All calls
- * share the one array: calls that overlap on a GPU race and must be
- * serialized by the caller. No memory is allocated or freed. Other arguments,
- * results and launches are those of tq_attend. */
+ * device memory: runtimes whose device memory belongs to an allocator they do
+ * not control, and serving loops that forbid allocation after start-up. (The
+ * pages describe no such call; it is an addition of this library.) The
+ * scratch is a static device array of TQ_NOALLOC_SCRATCH_BYTES that exists on
+ * every GPU that loads the library until the process exits; calls needing
+ * more (tq_attend_workspace) return TQ_ERR_WORKSPACE without launching
+ * anything. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and keeps it for the life
+ * of the process: make that first call before any stream capture, and do not
+ * use the library across a cudaDeviceReset (which also invalidates every
+ * context's device tables). All calls share the one array: calls that
+ * overlap on a GPU race and must be serialized by the caller. No memory is
+ * allocated or freed. Other arguments, results and launches are those of
+ * tq_attend. */
 #define TQ_NOALLOC_SCRATCH_BYTES (16u << 20)
 int tq_attend_noalloc(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,
                       const int32_t* seq_len, int max_len, float* out, void* stream);

@@ -92,7 +92,19 @@ def _load(path: str = LIB_PATH):
     return lib
 
 
-_lib = _load()
+class _LazyLib:
+    """The CUDA library, loaded on first use (a missing library then raises
+    ImportError at that first call): importing the package for its workload
+    shapes alone maps no GPU code."""
+    _handle = None
+
+    def __getattr__(self, name):
+        if _LazyLib._handle is None:
+            _LazyLib._handle = _load()
+        return getattr(_LazyLib._handle, name)
+
+
+_lib = _LazyLib()
 
 
 def _strerror(code: int) -> str:
@@ -312,8 +324,9 @@ def tq_scores(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor
 def tq_attend_noalloc(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor,
                       max_len: int, out: torch.Tensor | None = None, stream=None):
     """tq_attend with the library's static device scratch instead of a
-    workspace: for callers that cannot allocate device memory (see tq.h).
-    Overlapping calls on one GPU race on that scratch."""
+    workspace: for callers that cannot allocate device memory (their device
+    memory belongs to another allocator, or allocation is forbidden after
+    start-up; see tq.h). Overlapping calls on one GPU race on that scratch."""
     if q.dim() != 3 or q.shape[2] != ctx.d:
         raise ValueError("q must be [B, Hq, d] with d = %d" % ctx.d)
     if out is None:

@@ -2,14 +2,12 @@
 // array, for callers that cannot allocate device memory.
 //
 // tq_attend needs a workspace (the query fragments and the split-K partial
-// results). Most callers pass one they allocated. Some cannot: code that runs
-// while a stream is being captured into a CUDA graph (an allocation there
-// breaks or invalidates the capture), runtimes whose memory is owned by a
-// caching allocator they do not control, and real-time serving loops that
-// forbid allocation after start-up. This entry point takes its scratch from a
-// file-scope __device__ array of TQ_NOALLOC_SCRATCH_BYTES instead. The array
-// exists on every GPU that loads this library, for as long as the process
-// runs.
+// results). Most callers pass one they allocated. Some cannot: runtimes whose
+// memory is owned by a caching allocator they do not control, and real-time
+// serving loops that forbid allocation after start-up. This entry point takes
+// its scratch from a file-scope __device__ array of TQ_NOALLOC_SCRATCH_BYTES
+// instead. The array exists on every GPU that loads this library, for as long
+// as the process runs.
 //
 // Rules that follow from sharing one array:
 //  - Calls that overlap on a GPU (other streams, other threads, other
@@ -19,7 +17,10 @@
 //  - The host cannot pass the array's name to a kernel (in host code it is
 //    only a stand-in): its device address is looked up with
 //    cudaGetSymbolAddress once per device, on the first call made with that
-//    device current. Make that first call before any stream capture.
+//    device current, and kept for the life of the process. Make that first
+//    call before any stream capture. A cudaDeviceReset (which also
+//    invalidates every context's tables) can move the array: do not use the
+//    library across one.
 #include <cuda_runtime.h>
 
 #include <atomic>

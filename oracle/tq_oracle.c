@@ -23,10 +23,10 @@
  *  [DIGIPUB] "Google把32B模型壓到5GB顯存，實測后我發現3個坑" (m.digipub.cc):
  *            opening section (Walsh–Hadamard rotation, then scalar quantization).
  *
- * Where the pages leave a step open the oracle takes the plain reading that is
- * listed in the design doc (codebook for N(0,1/d); K uses (b-1)-bit codes + QJL with
- * m = d rows, V uses b-bit codes; fp16 norms; SplitMix64 tables; strict '>'
- * for the encoder; z >= 0 gives sign bit 1; the packed tile layout).
+ * Where the pages leave a step open the oracle takes the plainest reading:
+ * codebook for N(0,1/d); K uses (b-1)-bit codes + QJL with m = d rows, V uses
+ * b-bit codes; fp16 norms; SplitMix64 tables; strict '>' for the encoder;
+ * z >= 0 gives sign bit 1; the packed tile layout of include/tq.h.
  *
  * Pins (tests/test_oracle_*.py check each function against something other
  * than itself): the generator against published SplitMix64 outputs and

@@ -17,34 +17,52 @@ def _src_sha():
 
 
 def test_profiled_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
-    # the committed summary carries the hash of the source it was taken on
-    fields = {}
-    with open(os.path.join(ROOT, "profiles", "attend_split_llama70b_32k.md"), encoding="utf-8") as f:
-        for line in f:
-            if ":" in line and line.split(":", 1)[0].strip() in ("kernel_source_sha1",
-                                                                 "dram_bytes_per_launch"):
-                k, v = line.split(":", 1)
-                fields[k.strip()] = v.split()[0]
+    # the committed record carries the hash of the source it was taken on
+    import json
     got = bench.profiled_traffic(bench.DEFAULT_WORKLOAD)
-    if fields.get("kernel_source_sha1") == _src_sha():
-        assert got == int(fields["dram_bytes_per_launch"])
+    if os.path.exists(bench.TRAFFIC_FILE):
+        rec = json.load(open(bench.TRAFFIC_FILE))
+        if rec.get("kernel_source_sha1") == _src_sha() and rec.get("workload") == bench.DEFAULT_WORKLOAD:
+            assert got == int(rec["dram_bytes_per_launch"])
+        else:
+            assert got is None
     else:
         assert got is None
     # another workload never borrows the figure
     assert bench.profiled_traffic("qwen2.5-3b_decode_8k") is None
-    # a summary taken on other source is ignored
+    # a record taken on other source is ignored
     fake_root = tmp_path
     (fake_root / "profiles").mkdir()
     (fake_root / "kv_cache_vector_04_b200" / "csrc").mkdir(parents=True)
     (fake_root / "kv_cache_vector_04_b200" / "csrc" / "attend_impl.cuh").write_bytes(b"other source")
-    (fake_root / "profiles" / "attend_split_llama70b_32k.md").write_text(
-        "kernel_source_sha1: %s\ndram_bytes_per_launch: 123\n" % _src_sha())
+    rec_path = fake_root / "profiles" / "attend_split_llama70b_32k.json"
+    rec_path.write_text(json.dumps({"workload": bench.DEFAULT_WORKLOAD, "kernel_source_sha1": _src_sha(),
+                                    "dram_bytes_per_launch": 123}))
     monkeypatch.setattr(bench, "ROOT", str(fake_root))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(rec_path))
     assert bench.profiled_traffic(bench.DEFAULT_WORKLOAD) is None
     sha_other = hashlib.sha1(b"other source").hexdigest()
-    (fake_root / "profiles" / "attend_split_llama70b_32k.md").write_text(
-        "kernel_source_sha1: %s\ndram_bytes_per_launch: 123\n" % sha_other)
+    rec_path.write_text(json.dumps({"workload": bench.DEFAULT_WORKLOAD, "kernel_source_sha1": sha_other,
+                                    "dram_bytes_per_launch": 123}))
     assert bench.profiled_traffic(bench.DEFAULT_WORKLOAD) == 123
+
+
+def test_bytes_per_head_token_match_the_oracle_tiles():
+    # the bench's byte count per (token, kv head) is the packed tile layout's
+    from kv_cache_vector_04_b200 import inputs
+    from oracle import oracle as O
+    for w in list(inputs.WORKLOADS.values()) + inputs.sweep_workloads() + inputs.format_workloads():
+        fmt = bench.fmt_of(w)
+        assert bench.bytes_per_head_token(w) * 16 == O.tile_bytes(w.d, fmt), w.name
+
+
+def test_reference_arm_reports_the_gpu_arms_config():
+    # both arms describe the same workload (context N + 1: the decode step's token included)
+    from kv_cache_vector_04_b200 import inputs
+    w = inputs.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    cfg = bench.workload_config(w, w.layers, 1)
+    assert cfg["context"] == w.N + 1 and cfg["format"] == [3, 4, 1] and cfg["layers"] == 80
+    assert cfg["packed_cache_gb"] == round(80 * 16 * 8 * (w.N + 16) * 134 / 1e9, 2)
 
 
 def test_l2_note():

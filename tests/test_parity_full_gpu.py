@@ -124,10 +124,69 @@ def test_qwen3b_shaped_layer_8k():
     _run_layer(w, samples=[(0, 0), (0, 1)])
 
 
-@pytest.mark.parametrize("name", ["sweep_d64_b2_n65536", "sweep_d256_b4_n65536",
-                                  "sweep_d128_b3_n16384", "sweep_d256_b2_n4096"])
+@pytest.mark.parametrize("name", [w.name for w in inputs.sweep_workloads()])
 def test_sweep_points(name):
+    # every point of the d x bits x context sweep at its full size (batch 8,
+    # 8 kv heads, 32 query heads), with unequal lengths across the batch; one
+    # sampled stream per point
     w = {x.name: x for x in inputs.sweep_workloads()}[name]
-    # unequal lengths across the batch
     _run_layer(w, samples=[(7, 5)],
                seq_fn=lambda w: torch.tensor([w.N - 37 * i for i in range(w.B)], dtype=torch.int32))
+
+
+def test_qwen32b_shaped_prefill_then_32_decode_steps():
+    # The long-context workload as specified: bulk tq_quantize of all 131072
+    # prefill tokens of one layer, then 32 decode steps, each one
+    # tq_append_attend (append the step's token at position N + s, attend over
+    # N + s + 1 tokens). On one sampled (batch, kv head) stream, every appended
+    # token's codes and every step's output (its 5 query heads) are compared
+    # with the oracle's, the oracle attending over its own codes of the prefix
+    # and of the appended tokens.
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = inputs.WORKLOADS["qwen2.5-32b_prefill_decode_128k"]
+    assert w.decode_steps == 32
+    steps, (b, h) = w.decode_steps, (0, 6)
+    ctx = tq.tq_init(w.d, w.bits, 1)
+    tab = O.Tables(w.d, w.bits, 1)
+    k, v = inputs.kv_pair(w, w.N, layer=0, device=dev)
+    cap = w.N + steps
+    cache = tq.new_cache(ctx, w.B, w.Hkv, cap)
+    tq.tq_quantize(ctx, k, v, torch.zeros(w.B, dtype=torch.int32, device=dev), cache)
+    assert tq.tq_status(ctx) == 0
+    lay = tq.tq_cache_layout(ctx)
+    per_stream = (cap // 16) * lay["tile_bytes"]
+    stats = P.QuantStats()
+    ora = O.quantize(tab, k[b, h].cpu().numpy(), v[b, h].cpu().numpy())
+    host = cache.data.cpu().numpy()
+    P.compare_stream(tab, O.unpack_stream(w.d, w.bits, w.N,
+                                          P.stream_bytes(host, lay["tile_bytes"], cap, w.Hkv, b, h, w.N)),
+                     ora, w.N, stats)
+    # the sampled stream holds the oracle's packing of its own codes from here on
+    s0 = (b * w.Hkv + h) * per_stream
+    packed = torch.from_numpy(O.pack_stream(w.d, w.bits, ora)).to(dev)
+    cache.data[s0: s0 + packed.numel()].copy_(packed)
+    del k, v
+    g = w.Hq // w.Hkv
+    ws = tq.new_workspace(ctx, w.B, w.Hq, w.Hkv, cap)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    for s in range(steps):
+        n = w.N + s
+        q = inputs.queries(w, layer=s, device=dev)
+        nk, nv = inputs.kv_pair(w, 1, layer=10_000 + s, device=dev)
+        start = torch.full((w.B,), n, dtype=torch.int32, device=dev)
+        seq = torch.full((w.B,), n + 1, dtype=torch.int32, device=dev)
+        tq.tq_append_attend(ctx, q, nk, nv, start, cache, seq, n + 1, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        assert tq.tq_status(ctx) == 0
+        new = O.quantize(tab, nk[b, h].cpu().numpy(), nv[b, h].cpu().numpy())
+        tb0 = s0 + (n // 16) * lay["tile_bytes"]   # the tile holding token n
+        gpu = O.unpack_stream(w.d, tab, 16, cache.data[tb0: tb0 + lay["tile_bytes"]].cpu().numpy())
+        P.compare_stream(tab, {kk: vv[n % 16: n % 16 + 1] for kk, vv in gpu.items()}, new, 1, stats)
+        ora = {kk: np.concatenate([ora[kk], new[kk]]) for kk in ora}
+        codes = {key: ora[key][None, None] for key in ("kidx", "ksign", "knorm", "rnorm", "vidx", "vnorm")}
+        qb = np.ascontiguousarray(P.q_bits(q.cpu())[b:b + 1, h * g:(h + 1) * g])
+        ref = O.attend_batch(tab, qb, True, codes, np.array([n + 1], np.int32), 1)
+        err = P.attn_error(out[b:b + 1, h * g:(h + 1) * g].cpu().numpy().astype(np.float64), ref)
+        assert err.max() <= P.ATTN_TOL, (s, err.max())
+    stats.check()
