@@ -583,18 +583,24 @@ __global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArg
 
 
 // ---------------------------------------------------------------- reduction
-// One CTA per (query head, batch): merges, in two passes (max, then sums), the
-// partials of the CTAs whose ranges cover the head's unit (the range of CTA c
-// is [c W / G, (c+1) W / G) of the W tiles, so tile x lies in CTA
-// ((x + 1) G - 1) / W), then applies Pi^T with an fp32 Walsh-Hadamard
-// transform: thread i holds coordinate i = 32 w + lane; the butterflies over
-// the lane bits run on shuffles, those over the warp bits through shared
-// memory (double-buffered: one barrier per stage).
+// One CTA per (query head, batch): merges the partials of the CTAs whose ranges
+// cover the head's unit (the range of CTA c is [c W / G, (c+1) W / G) of the W
+// tiles, so tile x lies in CTA ((x + 1) G - 1) / W; a CTA with an empty range
+// wrote no partial), then applies Pi^T with an fp32 Walsh-Hadamard transform.
+// The partials are taken D at a time, one per thread: each thread loads one
+// partial's max and sum, the block reduces them, and every thread then adds
+// the chunk's rescaled accumulators of its coordinate with independent loads
+// (a unit of a short batch spans many CTAs: no load waits on another).
+// WHT: thread i holds coordinate i = 32 w + lane; the butterflies over the
+// lane bits run on shuffles, those over the warp bits through shared memory
+// (double-buffered: one barrier per stage).
 template <int D>
 __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
 {
     constexpr int NW = D / 32;
     __shared__ float xs[2][NW][33];
+    __shared__ float fsh[D];          // the chunk's partial weights exp2(m_c - M)
+    __shared__ float red[2][NW];
     pdl_trigger();
     pdl_wait();
     const int hq = blockIdx.x, b = blockIdx.y, i = threadIdx.x, w = i >> 5, lane = i & 31;
@@ -607,43 +613,52 @@ __global__ void __launch_bounds__(D) attend_reduce(DevTables tb, AttendArgs a)
     const long long T = (a.prefix[b + 1] - pb) / upb;
     const long long G = a.plan.ctas;
     float M = -CUDART_INF_F, L = 0.f, acc = 0.f;
-    if (T > 0) {
+    if (T > 0) {   // uniform over the block
         const long long U0 = pb + ju * T, U1 = U0 + T;
         const int cf = (int)(((U0 + 1) * G - 1) / W), cl = (int)((U1 * G - 1) / W);
         const float* base = a.partial + u * 8 * RS + col * RS;   // + c * 8 * RS: slot c + u
-        // CTA c's range starts at tile floor(c W / G); walked as quotient and
-        // remainder, so the loops divide nothing (a unit of a short batch can
-        // span most of the grid). A CTA with an empty range wrote no partial.
-        const long long wq = W / G, wr = W - wq * G;
-        const long long q0 = (long long)cf * W / G, r0 = (long long)cf * W - q0 * G;
-        // Two passes with independent loads (not one chain of dependent ones):
-        // the largest partial max, then the sums rescaled to it (a partial with
-        // max -inf adds 0).
-        long long q = q0, r = r0;
-#pragma unroll 4
-        for (int c = cf; c <= cl; ++c) {
-            long long qn = q + wq, rn = r + wr;
-            if (rn >= G) { ++qn; rn -= G; }
-            if (qn != q) M = fmaxf(M, base[(size_t)c * 8 * RS]);
-            q = qn;
-            r = rn;
-        }
-        if (M != -CUDART_INF_F) {
-            q = q0;
-            r = r0;
-#pragma unroll 4
-            for (int c = cf; c <= cl; ++c) {
-                long long qn = q + wq, rn = r + wr;
-                if (rn >= G) { ++qn; rn -= G; }
-                if (qn != q) {
-                    const float* ps = base + (size_t)c * 8 * RS;
-                    const float f = exp2f(ps[0] - M);
-                    L = fmaf(ps[1], f, L);
-                    acc = fmaf(ps[2 + i], f, acc);
-                }
-                q = qn;
-                r = rn;
+#pragma unroll 1
+        for (int c0 = cf; c0 <= cl; c0 += D) {
+            const int c = c0 + i;
+            float mc = -CUDART_INF_F, lc = 0.f;
+            if (c <= cl && (long long)(c + 1) * W / G > (long long)c * W / G) {
+                const float* ps = base + (size_t)c * 8 * RS;
+                mc = ps[0];
+                lc = ps[1];
             }
+            float mx = mc;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+            if (lane == 0) red[0][w] = mx;
+            __syncthreads();
+            float Mn = M;
+#pragma unroll
+            for (int k = 0; k < NW; ++k) Mn = fmaxf(Mn, red[0][k]);
+            // partials with max -inf (no valid token) weigh 0; so does the
+            // running state while it holds nothing
+            const float fo = (M == -CUDART_INF_F) ? 0.f : exp2f(M - Mn);
+            const float fc = (mc == -CUDART_INF_F) ? 0.f : exp2f(mc - Mn);
+            fsh[i] = fc;
+            float ls = lc * fc;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) ls += __shfl_xor_sync(kFull, ls, o);
+            if (lane == 0) red[1][w] = ls;
+            __syncthreads();
+            float lsum = 0.f;
+#pragma unroll
+            for (int k = 0; k < NW; ++k) lsum += red[1][k];
+            L = L * fo + lsum;
+            acc *= fo;
+            M = Mn;
+            const int nc = min(D, cl - c0 + 1);
+            const float* pc = base + (size_t)c0 * 8 * RS + 2 + i;
+#pragma unroll 8
+            for (int k = 0; k < nc; ++k) {
+                const float f = fsh[k];
+                const float v = pc[(size_t)k * 8 * RS];   // in the buffer even where unwritten
+                acc = fmaf(f != 0.f ? v : 0.f, f, acc);
+            }
+            __syncthreads();   // fsh and red are rewritten by the next chunk
         }
     }
     float x = (L > 0.f) ? acc / L : 0.f;

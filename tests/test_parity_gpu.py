@@ -239,6 +239,24 @@ def test_attend_many_heads_per_group_and_empty_sequence():
     assert P.attn_error(got, ref).max() <= P.ATTN_TOL
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_attend_one_unit_over_the_whole_grid(d):
+    # One sequence, one kv head, one group of query heads, 188 tiles: the unit
+    # is split over every CTA of the grid, so the reduce merges one partial per
+    # CTA: more partials than its D threads take at once at d = 64 and 128.
+    ctx, tab = ctx_for(d, 3)
+    B, Hkv, Hq, N = 1, 1, 6, 3001
+    cap = 3008
+    k, v = kv(B, Hkv, N, d, seed=900 + d)
+    codes = P.oracle_codes(tab, k, v)
+    cache = tq.Cache(P.pack_cache(tab, codes, cap, d, 3), B, Hkv, cap)
+    q = qtensor(B, Hq, d, seed=d)
+    got = run_attend(ctx, tab, cache, q, [N], N, Hkv)
+    ref = O.attend_batch(tab, P.q_bits(q), True, P.stack_codes(codes, cap), np.array([N], np.int32), Hkv)
+    assert P.attn_error(got, ref).max() <= P.ATTN_TOL
+    assert tq.tq_status(ctx) == 0
+
+
 @pytest.mark.parametrize("d,bits,max_len", [(64, 4, 600), (128, 3, 600), (128, 2, 4096)])
 def test_attend_many_ragged_sequences(d, bits, max_len):
     # Many sequences of mixed lengths (empty, one token, tile edges, a few
