@@ -171,22 +171,67 @@ __device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t x)
     }
 }
 
-// fp16x2 (+-rho, +-rho) from sign pair p: element 0 at bit p%16, element 1 at
-// bit 16 + p%16 of sign word p/16 (bit 1 = +); nrho2 holds -rho in both halves.
-// The residual norm rho rides on the sign operand, so the QJL products land in
-// the same accumulators as the codebook products.
-__device__ __forceinline__ uint32_t sign_pair(uint32_t word, int q, uint32_t nrho2)
+// ---------------------------------------------------------------- QJL term, int8 path
+// The QJL product sum_i (2 s_i - 1) x_i of a key's sign bits s_i with the
+// head's projected query x = S q~ (scaled as the logits need) runs as an
+// integer MMA (m16n8k32, twice the k of an fp16 MMA at the same issue cost):
+// x is held as 16-bit fixed point n_i = rint(x_i / u), u = max_i |x_i| / 32767
+// per head, split into a signed high byte and an unsigned low byte
+// (n = 256 hi + lo); the A operand carries the signs as bytes 0 / sigma. With
+// acc = sum_i sigma s_i n_i (exact in int32) and T = sum_i n_i,
+//     sum_i (2 s_i - 1) x_i = u (2 acc / sigma - T) + (rounding of x, <= u/2 a term).
+// Sign layouts (SL): 0 none (no QJL), 1 sign words (two bits a key pair at bits
+// q and q + 16 of the pair's sign word), 2 byte fields (the two top bits of each
+// key byte: token g at bit 6, token g + 8 at bit 7).
+template <int KB, int QJ>
+struct SignLayout {
+    static constexpr int SL = QJ == 0 ? 0 : (TileLayout<64, KB, 1, QJ>::KS_BYTES ? 2 : 1);
+};
+
+// The coordinate held by byte i (0..3) of the B register `half` (0: b0, 1: b1)
+// of lane group t in int8 k-step J: the k-positions of an A register of byte-
+// field signs are the coordinates of its key word; those of sign word m are
+// read with the shifts 4h + {0, 1, 2, 3} (h = J & 1), each picking one bit of
+// every byte.
+template <int SL>
+__host__ __device__ __forceinline__ int qjl_dim(int J, int t, int half, int i)
 {
-    const uint32_t x = word << (15 - q);
-    return (x & 0x80008000u) ^ nrho2;
+    if constexpr (SL == 2)
+        return 16 * (2 * J + half) + 8 * (i & 1) + 2 * t + (i >> 1);
+    else
+        return 16 * (4 * (J >> 1) + (J & 1) + 2 * (i & 1)) + 8 * half + 2 * t + (i >> 1);
 }
 
-// Byte-field keys with QJL: the sign pair of key pair r of a k-step sits in
-// that k-step's key word at bits a and a + 16, a = 6 + (r & 1) + 8 (r >> 1)
-// (the top two bits of each byte; for r = 3 no shift is needed).
-__device__ __forceinline__ uint32_t sign_pair_byte(uint32_t word, int r, uint32_t nrho2)
+// sigma of the A bytes of tokens g (sg) and g + 8 (sh)
+template <int SL>
+struct QjlSigma {
+    static constexpr float sg = SL == 2 ? 64.f : 1.f, sh = SL == 2 ? 128.f : 1.f;
+};
+
+// A registers of int8 k-step J: a0, a2 token g, a1, a3 token g + 8 (bytes 0 / sigma).
+template <int SL, int SBW>
+__device__ __forceinline__ void qjl_a(const uint32_t* s, int J, uint32_t (&a)[4])
 {
-    return sign_pair(word, 6 + (r & 1) + 8 * (r >> 1), nrho2);
+    if constexpr (SL == 2) {
+        const uint32_t w0 = s[2 * J], w1 = s[2 * J + 1];
+        a[0] = w0 & 0x40404040u;
+        a[1] = w0 & 0x80808080u;
+        a[2] = w1 & 0x40404040u;
+        a[3] = w1 & 0x80808080u;
+    } else {
+        const uint32_t w = s[SBW + (J >> 1)] >> (4 * (J & 1));
+        a[0] = w & 0x01010101u;
+        a[1] = (w >> 1) & 0x01010101u;
+        a[2] = (w >> 2) & 0x01010101u;
+        a[3] = (w >> 3) & 0x01010101u;
+    }
+}
+
+// Fixed-point code of x with inv = 32767 / max |x| (0 when there is no scale).
+__device__ __forceinline__ int qjl_fix(float x, float inv)
+{
+    const int n = __float2int_rn(x * inv);
+    return max(-32767, min(32767, n));
 }
 
 // ---------------------------------------------------------------- prologue
@@ -230,13 +275,15 @@ __device__ __forceinline__ void tile_prefix(const DevTables& tb, const AttendArg
 // each as a hi part and a lo part (x - hi), so that the two tensor-core
 // products carry ~22 significant bits. alpha is the scale that makes the key
 // codebook almost exact in fp16 (chosen on the host).
-template <int D>
+template <int D, int SL>
 __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendArgs& a)
 {
     constexpr int NT = 2 * D, VPL = D / 32;
     __shared__ float qt[D][9];          // rotated queries, [coordinate][head] (padded rows)
     __shared__ float pp[1][D][8];       // p = S q~
     __shared__ float es[8];             // per-head power-of-two scale of q~ for the split
+    __shared__ float qinv[8], qu[8];    // QJL fixed point: 32767 / max |x|, and u = its inverse
+    __shared__ int qsum[8];             // QJL fixed point: T = sum of the codes
     const int unit = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     const int groups = a.plan.groups, ratio = a.Hq / a.Hkv;
     const int hkv = unit / groups, grp = unit % groups;
@@ -298,6 +345,7 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
         }
     }
     __syncthreads();
+    if constexpr (SL != 0) {
     // p^T = q~^T S^T on the tensor cores: A = q~ es (rows = the 8 heads, rows
     // 8..15 zero) as hi + lo fp16 parts, B = the fp16-exact S^T fragments,
     // fp32 accumulation; warp w takes n-tiles (8 rows of S each) w, w + NW, ...
@@ -328,42 +376,86 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
             pp[0][8 * nt + 2 * t + 1][g] = acc[1] / sc;
         }
     }
+    }
     __syncthreads();
+    const float scale_s = kLog2e * 128.0f * 1.2533141373155003f / ((float)D * sqrtf((float)D));
+    if constexpr (SL != 0) {
+        // the QJL fixed point of each head: x = p scale_s, max |x|, T = sum of the codes
+        const int w = tid >> 5, lane = tid & 31;
+        for (int h = w; h < 8; h += NT / 32) {
+            float mx = 0.f;
+            for (int i = lane; i < D; i += 32) mx = fmaxf(mx, fabsf(pp[0][i][h] * scale_s));
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+            const bool ok = mx > 0.f && mx < 3.0e38f;
+            const float inv = ok ? 32767.0f / mx : 0.f;
+            int T = 0;
+            for (int i = lane; i < D; i += 32) T += qjl_fix(pp[0][i][h] * scale_s, inv);
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) T += __shfl_xor_sync(kFull, T, o);
+            if (lane == 0) {
+                qinv[h] = inv;
+                qu[h] = ok ? mx / 32767.0f : 0.f;
+                qsum[h] = T;
+            }
+        }
+        __syncthreads();
+    }
     {
-        // one fragment entry (k-step, thread-in-group, head column) per thread
+        // one codebook fragment entry (k-step, thread-in-group, head column) per thread
         const int e = tid, col = e & 7, t = (e >> 3) & 3, kk = e >> 5;
         const int c0 = 16 * kk + 2 * t;
         const int idx[4] = {c0, c0 + 1, c0 + 8, c0 + 9};
         const float scale_c = kLog2e * 128.0f / ((float)D * tb.alpha_k);
-        const float scale_s = kLog2e * 128.0f * 1.2533141373155003f / ((float)D * sqrtf((float)D));
-        uint32_t hi[4], lo[4];
+        float hv[4], lv[4];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            float hv[4], lv[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float x = q ? pp[0][idx[u]][col] * scale_s : qt[idx[u]][col] * scale_c;
-                hv[u] = __half2float(__float2half_rn(x));
-                lv[u] = x - hv[u];
-            }
-            hi[2 * q] = pack_half2(hv[0], hv[1]);
-            hi[2 * q + 1] = pack_half2(hv[2], hv[3]);
-            lo[2 * q] = pack_half2(lv[0], lv[1]);
-            lo[2 * q + 1] = pack_half2(lv[2], lv[3]);
+        for (int u = 0; u < 4; ++u) {
+            const float x = qt[idx[u]][col] * scale_c;
+            hv[u] = __half2float(__float2half_rn(x));
+            lv[u] = x - hv[u];
         }
-        uint4* dst = reinterpret_cast<uint4*>(a.qfrag) +
-                     (((size_t)b * units + unit) * (D / 16) + kk) * 64 + col * 4 + t;
-        dst[0] = make_uint4(hi[0], hi[1], lo[0], lo[1]);    // codebook term: b0,b1 hi; b0,b1 lo
-        dst[32] = make_uint4(hi[2], hi[3], lo[2], lo[3]);   // QJL term
+        uint4* frag = reinterpret_cast<uint4*>(a.qfrag) + ((size_t)b * units + unit) * (D / 16) * 64;
+        // codebook term: b0, b1 hi; b0, b1 lo
+        frag[kk * 64 + col * 4 + t] =
+            make_uint4(pack_half2(hv[0], hv[1]), pack_half2(hv[2], hv[3]), pack_half2(lv[0], lv[1]),
+                       pack_half2(lv[2], lv[3]));
+        if constexpr (SL != 0) {
+            if (e < D) {
+                // int8 k-step J, lane (col, t): b0, b1 high bytes; b0, b1 low bytes
+                const int J = e >> 5, ln = e & 31, hc = ln >> 2, tt = ln & 3;
+                const float inv = qinv[hc];
+                uint32_t bh[2] = {0u, 0u}, bl[2] = {0u, 0u};
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = qjl_fix(pp[0][qjl_dim<SL>(J, tt, half, i)][hc] * scale_s, inv);
+                        bh[half] |= ((uint32_t)(n >> 8) & 0xFFu) << (8 * i);
+                        bl[half] |= ((uint32_t)n & 0xFFu) << (8 * i);
+                    }
+                }
+                frag[J * 64 + 32 + ln] = make_uint4(bh[0], bh[1], bl[0], bl[1]);
+            } else if (e < D + 32) {
+                // lane ln's constants: {2u/sigma} of (g, 2t), (g, 2t+1), (g+8, 2t),
+                // (g+8, 2t+1), then {-u T} of heads 2t, 2t+1
+                const int ln = e - D, tt = ln & 3, h0 = 2 * tt, h1 = 2 * tt + 1;
+                const float u0 = qu[h0], u1 = qu[h1];
+                frag[(D / 32) * 64 + 32 + ln] =
+                    make_uint4(__float_as_uint(2.f * u0 / QjlSigma<SL>::sg), __float_as_uint(2.f * u1 / QjlSigma<SL>::sg),
+                               __float_as_uint(2.f * u0 / QjlSigma<SL>::sh), __float_as_uint(2.f * u1 / QjlSigma<SL>::sh));
+                frag[(D / 32 + 1) * 64 + 32 + ln] =
+                    make_uint4(__float_as_uint(-u0 * (float)qsum[h0]), __float_as_uint(-u1 * (float)qsum[h1]), 0u, 0u);
+            }
+        }
     }
 }
 
-template <int D>
+template <int D, int SL>
 __global__ void __launch_bounds__(2 * D) attend_prologue(DevTables tb, AttendArgs a)
 {
     pdl_trigger();
     pdl_wait();
-    prologue_body<D>(tb, a);
+    prologue_body<D, SL>(tb, a);
 }
 
 // ---------------------------------------------------------------- fused append
@@ -578,7 +670,7 @@ __global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArg
     if ((int)blockIdx.x >= units)
         append_tokens<D, KB, VB, QJ>(tb, a, blockIdx.y, blockIdx.x - units, reinterpret_cast<uint8_t*>(app_smem));
     else
-        prologue_body<D>(tb, a);
+        prologue_body<D, SignLayout<KB, QJ>::SL>(tb, a);
 }
 
 
@@ -783,9 +875,11 @@ __device__ __forceinline__ void read_stage(const uint8_t* slot, int lane, TileDa
     td.vn = *reinterpret_cast<const uint32_t*>(slot + nb + Tr::KNB + 4 * g);
 }
 
-// Query B fragments of one k-step: x,y = hi (b0, b1), z,w = lo, for the
-// codebook term (c) and the QJL term (s), copied once per unit into shared
-// memory and read from there by every tile (registers go to warps instead).
+// Query B fragments, copied once per unit into shared memory and read from
+// there by every tile (registers go to warps instead): per fp16 k-step kk the
+// codebook term's x,y = hi (b0, b1), z,w = lo; per int8 k-step J < KK/2 the QJL
+// term's x,y = high bytes (b0, b1), z,w = low bytes; then the lane's QJL
+// constants {2u/sigma} and {-u T} (see qjl_a).
 template <int KK, int NT>
 struct QueryFrags {
     const uint4* sm;
@@ -795,8 +889,50 @@ struct QueryFrags {
         sm = smem;
     }
     __device__ __forceinline__ uint4 fc(int kk, int lane) const { return sm[kk * 64 + lane]; }
-    __device__ __forceinline__ uint4 fs(int kk, int lane) const { return sm[kk * 64 + 32 + lane]; }
+    __device__ __forceinline__ uint4 fs(int J, int lane) const { return sm[J * 64 + 32 + lane]; }
+    __device__ __forceinline__ float4 qa(int lane) const
+    {
+        const uint4 v = sm[(KK / 2) * 64 + 32 + lane];
+        return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+    }
+    __device__ __forceinline__ float2 qb(int lane) const
+    {
+        const uint4 v = sm[(KK / 2 + 1) * 64 + 32 + lane];
+        return make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    }
 };
+
+// Logits (log2 units) of tokens g, g + 8 and heads 2t, 2t + 1 from the
+// codebook sums (hi + lo chains) and the QJL integer sums (high, low byte
+// chains): L = |k| (c + rho (acc u 2/sigma - u T)).
+template <int QJ, typename QF>
+__device__ __forceinline__ void finish_logits(const uint2 kn, const float (&ah)[4], const float (&al)[4],
+                                              const int (&ih)[4], const int (&il)[4], const QF& qf, int lane,
+                                              float (&L)[4])
+{
+    if constexpr (QJ) {
+        const float2 kg = __half22float2(*reinterpret_cast<const __half2*>(&kn.x));   // |k_g|, rho_g
+        const float2 kh = __half22float2(*reinterpret_cast<const __half2*>(&kn.y));
+        const float4 ca = qf.qa(lane);
+        const float2 cb = qf.qb(lane);
+        const float y0 = fmaf((float)(ih[0] * 256 + il[0]), ca.x, cb.x);
+        const float y1 = fmaf((float)(ih[1] * 256 + il[1]), ca.y, cb.y);
+        const float y2 = fmaf((float)(ih[2] * 256 + il[2]), ca.z, cb.x);
+        const float y3 = fmaf((float)(ih[3] * 256 + il[3]), ca.w, cb.y);
+        const float ng = kg.x * (1.0f / 128.0f), nh = kh.x * (1.0f / 128.0f);   // the B operands carry 2^7
+        L[0] = ng * fmaf(kg.y, y0, ah[0] + al[0]);
+        L[1] = ng * fmaf(kg.y, y1, ah[1] + al[1]);
+        L[2] = nh * fmaf(kh.y, y2, ah[2] + al[2]);
+        L[3] = nh * fmaf(kh.y, y3, ah[3] + al[3]);
+    } else {
+        const float2 kk2 = __half22float2(*reinterpret_cast<const __half2*>(&kn.x));
+        const float ng = kk2.x * (1.0f / 128.0f), nh = kk2.y * (1.0f / 128.0f);
+        L[0] = ng * (ah[0] + al[0]);
+        L[1] = ng * (ah[1] + al[1]);
+        L[2] = nh * (ah[2] + al[2]);
+        L[3] = nh * (ah[3] + al[3]);
+    }
+}
 
 template <int D>
 struct SplitState {
@@ -810,22 +946,20 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
                                             const uint32_t* lutk, uint32_t lane4, float (&L)[4])
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    // -rho of tokens g and g+8 in both fp16 halves (A rows g and g+8)
-    const uint32_t nr_g = QJ ? (__byte_perm(td.kn.x, 0u, 0x3232) | 0x80008000u) : 0u;
-    const uint32_t nr_h = QJ ? (__byte_perm(td.kn.y, 0u, 0x3232) | 0x80008000u) : 0u;
-    // two accumulation chains: hi and lo parts of the B operands; each takes
-    // the codebook product and (QJ) the rho-weighted QJL product of every k-step
+    constexpr int SL = SignLayout<KB, QJ>::SL;
+    // codebook term: two fp16 chains, the hi and lo parts of the B operands;
+    // QJL term: two int8 chains, the high and low bytes of its B operands
     float ah[4], al[4];
+    int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
         const uint4 bc = qf.fc(kk, lane);
-        uint32_t ak[4], as[4], akl[4];   // akl: lo parts of per-code key levels
+        uint32_t ak[4], akl[4];   // akl: lo parts of per-code key levels
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int p = 4 * kk + r;
             if constexpr (Tr::PK) {
                 ak[r] = lut_load<Tr::ALIGNED>(lutk, row_off(td.s[kk], r, lane4));
-                if constexpr (QJ) as[r] = sign_pair_byte(td.s[kk], r, (r & 1) ? nr_h : nr_g);
             } else if constexpr (Tr::CK) {
                 // one table row per code, {hi, lo} of its level: the pair's hi
                 // parts form the A fragment, its lo parts a second one
@@ -834,12 +968,8 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
                 const uint32_t e1 = lut_load<Tr::ALIGNED>(lutk, lut_off<8>(td.s, Lay::kbit(p, 1), KB, lane4));
                 ak[r] = __byte_perm(e0, e1, 0x5410u);
                 akl[r] = __byte_perm(e0, e1, 0x7632u);
-                if constexpr (QJ)
-                    as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
             } else {
                 ak[r] = lut_load<Tr::ALIGNED>(lutk, lut_off<Tr::LSH>(td.s, Tr::KF * p, Tr::KF, lane4));
-                if constexpr (QJ)
-                    as[r] = sign_pair(td.s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h : nr_g);
             }
         }
         if (kk == 0) {
@@ -851,25 +981,17 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
         }
         if constexpr (Tr::CK) mma_16816(al, akl[0], akl[1], akl[2], akl[3], bc.x, bc.y);
         if constexpr (QJ) {
-            const uint4 bs = qf.fs(kk, lane);
-            mma_16816(ah, as[0], as[1], as[2], as[3], bs.x, bs.y);
-            mma_16816(al, as[0], as[1], as[2], as[3], bs.z, bs.w);
+            if (kk & 1) {   // one int8 k-step (32 coordinates) every second fp16 k-step
+                const int J = kk >> 1;
+                const uint4 bs = qf.fs(J, lane);
+                uint32_t as[4];
+                qjl_a<SL, Tr::SBW>(td.s, J, as);
+                imma_16832<true>(ih, as[0], as[1], as[2], as[3], bs.x, bs.y);
+                imma_16832<false>(il, as[0], as[1], as[2], as[3], bs.z, bs.w);
+            }
         }
     }
-    // |k| of tokens g and g+8 (fp16); the B operands carry 2^7
-    float kn_g, kn_h;
-    if constexpr (QJ) {
-        kn_g = __low2float(*reinterpret_cast<const __half2*>(&td.kn.x)) * (1.0f / 128.0f);
-        kn_h = __low2float(*reinterpret_cast<const __half2*>(&td.kn.y)) * (1.0f / 128.0f);
-    } else {
-        const float2 kk2 = __half22float2(*reinterpret_cast<const __half2*>(&td.kn.x));
-        kn_g = kk2.x * (1.0f / 128.0f);
-        kn_h = kk2.y * (1.0f / 128.0f);
-    }
-    L[0] = kn_g * (ah[0] + al[0]);
-    L[1] = kn_g * (ah[1] + al[1]);
-    L[2] = kn_h * (ah[2] + al[2]);
-    L[3] = kn_h * (ah[3] + al[3]);
+    finish_logits<QJ>(td.kn, ah, al, ih, il, qf, lane, L);
 }
 
 // Online-softmax update and P V for one tile.
@@ -1301,32 +1423,22 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
                                             const uint32_t* lutk, uint32_t lane4, float (&L)[2][4])
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    uint32_t nr_g[2], nr_h[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        nr_g[u] = QJ ? (__byte_perm(td[u].kn.x, 0u, 0x3232) | 0x80008000u) : 0u;
-        nr_h[u] = QJ ? (__byte_perm(td[u].kn.y, 0u, 0x3232) | 0x80008000u) : 0u;
-    }
+    constexpr int SL = SignLayout<KB, QJ>::SL;
     float ah[2][4], al[2][4];
+    int ih[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, il[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
         const uint4 bc = qf.fc(kk, lane);
-        uint4 bs;
-        if constexpr (QJ) bs = qf.fs(kk, lane);
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            uint32_t ak[4], as[4];
+            uint32_t ak[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const int p = 4 * kk + r;
-                if constexpr (Tr::PK) {
+                if constexpr (Tr::PK)
                     ak[r] = lut_load<true>(lutk, row_off(td[u].s[kk], r, lane4));
-                    if constexpr (QJ) as[r] = sign_pair_byte(td[u].s[kk], r, (r & 1) ? nr_h[u] : nr_g[u]);
-                } else {
+                else
                     ak[r] = lut_load<true>(lutk, lut_off<Tr::LSH>(td[u].s, Tr::KF * p, Tr::KF, lane4));
-                    if constexpr (QJ)
-                        as[r] = sign_pair(td[u].s[Tr::SBW + (p >> 4)], p & 15, (r & 1) ? nr_h[u] : nr_g[u]);
-                }
             }
             if (kk == 0) {
                 mma_16816_first(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
@@ -1335,28 +1447,23 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
                 mma_16816(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
                 mma_16816(al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
             }
-            if constexpr (QJ) {
-                mma_16816(ah[u], as[0], as[1], as[2], as[3], bs.x, bs.y);
-                mma_16816(al[u], as[0], as[1], as[2], as[3], bs.z, bs.w);
+        }
+        if constexpr (QJ) {
+            if (kk & 1) {   // one int8 k-step (32 coordinates) every second fp16 k-step
+                const int J = kk >> 1;
+                const uint4 bs = qf.fs(J, lane);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    uint32_t as[4];
+                    qjl_a<SL, Tr::SBW>(td[u].s, J, as);
+                    imma_16832<true>(ih[u], as[0], as[1], as[2], as[3], bs.x, bs.y);
+                    imma_16832<false>(il[u], as[0], as[1], as[2], as[3], bs.z, bs.w);
+                }
             }
         }
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        float kn_g, kn_h;
-        if constexpr (QJ) {
-            kn_g = __low2float(*reinterpret_cast<const __half2*>(&td[u].kn.x)) * (1.0f / 128.0f);
-            kn_h = __low2float(*reinterpret_cast<const __half2*>(&td[u].kn.y)) * (1.0f / 128.0f);
-        } else {
-            const float2 kk2 = __half22float2(*reinterpret_cast<const __half2*>(&td[u].kn.x));
-            kn_g = kk2.x * (1.0f / 128.0f);
-            kn_h = kk2.y * (1.0f / 128.0f);
-        }
-        L[u][0] = kn_g * (ah[u][0] + al[u][0]);
-        L[u][1] = kn_g * (ah[u][1] + al[u][1]);
-        L[u][2] = kn_h * (ah[u][2] + al[u][2]);
-        L[u][3] = kn_h * (ah[u][3] + al[u][3]);
-    }
+    for (int u = 0; u < 2; ++u) finish_logits<QJ>(td[u].kn, ah[u], al[u], ih[u], il[u], qf, lane, L[u]);
 }
 
 // Online-softmax update and P V for two tiles (one running-maximum check for both).
@@ -1658,7 +1765,7 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
         if ((e = allow_smem(kern, smem, done_append)) != cudaSuccess) return e;
         e = launch_pdl(kern, dim3(units + a.Hkv, a.B), dim3(2 * D), smem, st, tb, a);
     } else {
-        e = launch_pdl(attend_prologue<D>, dim3(units, a.B), dim3(2 * D), 0, st, tb, a);
+        e = launch_pdl(attend_prologue<D, SignLayout<KB, QJ>::SL>, dim3(units, a.B), dim3(2 * D), 0, st, tb, a);
     }
     if (e != cudaSuccess) return e;
     if (scores) {

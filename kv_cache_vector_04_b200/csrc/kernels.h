@@ -39,7 +39,7 @@ struct AttendArgs {
     const uint8_t* cache;
     int B, Hq, Hkv, capacity, max_len;
     long long tile_bytes;
-    uint32_t* qfrag;          // workspace: [B][Hkv*groups][d/16][32][4] fp16x2 B fragments
+    uint32_t* qfrag;          // workspace: [B][Hkv*groups][d/16][64] uint4 query fragments (codebook fp16, QJL int8)
     long long* prefix;        // workspace: [B + 1] first flattened tile of each sequence's units
     float* partial;           // workspace: [ctas + B*Hkv*groups][8][d + 2], slot = CTA + unit
     float* out;               // [B][Hq][d] (attend) or scores [B][Hq][max_len]
