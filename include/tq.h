@@ -255,8 +255,7 @@ int tq_scores(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_c
  * more (tq_attend_workspace) return TQ_ERR_WORKSPACE without launching
  * anything. The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current and keeps it for the life
- * of the process: make that first call before any stream capture, and do not
- * use the library across a cudaDeviceReset (which also invalidates every
+ * of the process; do not use the library across a cudaDeviceReset (which also invalidates every
  * context's device tables). All calls share the one array: calls that
  * overlap on a GPU race and must be serialized by the caller. No memory is
  * allocated or freed. Other arguments, results and launches are those of

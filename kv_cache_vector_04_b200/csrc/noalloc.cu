@@ -17,8 +17,7 @@
 //  - The host cannot pass the array's name to a kernel (in host code it is
 //    only a stand-in): its device address is looked up with
 //    cudaGetSymbolAddress once per device, on the first call made with that
-//    device current, and kept for the life of the process. Make that first
-//    call before any stream capture. A cudaDeviceReset (which also
+//    device current, and kept for the life of the process. A cudaDeviceReset (which also
 //    invalidates every context's tables) can move the array: do not use the
 //    library across one.
 #include <cuda_runtime.h>
