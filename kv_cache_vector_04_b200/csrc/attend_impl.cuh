@@ -903,18 +903,17 @@ struct QueryFrags {
 };
 
 // Logits (log2 units) of tokens g, g + 8 and heads 2t, 2t + 1 from the
-// codebook sums (hi + lo chains) and the QJL integer sums (high, low byte
-// chains): L = |k| (c + rho (acc u 2/sigma - u T)).
-template <int QJ, typename QF>
-__device__ __forceinline__ void finish_logits(const uint2 kn, const float (&ah)[4], const float (&al)[4],
-                                              const int (&ih)[4], const int (&il)[4], const QF& qf, int lane,
+// codebook sums (two fp32 chains: the hi and lo parts of the B operands) and the
+// QJL integer sums (high, low byte chains): L = |k| (c + rho (acc u 2/sigma - u T)).
+// ca, cb: the lane's QJL constants (QueryFrags::qa, qb).
+template <int QJ>
+__device__ __forceinline__ void finish_logits(const uint2 kn, const float (&ah)[4], const float (&al)[4], const int (&ih)[4],
+                                              const int (&il)[4], const float4 ca, const float2 cb,
                                               float (&L)[4])
 {
     if constexpr (QJ) {
         const float2 kg = __half22float2(*reinterpret_cast<const __half2*>(&kn.x));   // |k_g|, rho_g
         const float2 kh = __half22float2(*reinterpret_cast<const __half2*>(&kn.y));
-        const float4 ca = qf.qa(lane);
-        const float2 cb = qf.qb(lane);
         const float y0 = fmaf((float)(ih[0] * 256 + il[0]), ca.x, cb.x);
         const float y1 = fmaf((float)(ih[1] * 256 + il[1]), ca.y, cb.y);
         const float y2 = fmaf((float)(ih[2] * 256 + il[2]), ca.z, cb.x);
@@ -947,7 +946,7 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
     constexpr int SL = SignLayout<KB, QJ>::SL;
-    // codebook term: two fp16 chains, the hi and lo parts of the B operands;
+    // codebook term: two fp32 chains, the hi and lo parts of the B operands;
     // QJL term: two int8 chains, the high and low bytes of its B operands
     float ah[4], al[4];
     int ih[4] = {0, 0, 0, 0}, il[4] = {0, 0, 0, 0};
@@ -991,7 +990,13 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
             }
         }
     }
-    finish_logits<QJ>(td.kn, ah, al, ih, il, qf, lane, L);
+    float4 ca = make_float4(0.f, 0.f, 0.f, 0.f);
+    float2 cb = make_float2(0.f, 0.f);
+    if constexpr (QJ) {
+        ca = qf.qa(lane);
+        cb = qf.qb(lane);
+    }
+    finish_logits<QJ>(td.kn, ah, al, ih, il, ca, cb, L);
 }
 
 // Online-softmax update and P V for one tile.
@@ -1424,7 +1429,7 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
     constexpr int SL = SignLayout<KB, QJ>::SL;
-    float ah[2][4], al[2][4];
+    float ah[2][4], al[2][4];   // codebook term: the hi and lo B parts
     int ih[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, il[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
@@ -1462,14 +1467,20 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
             }
         }
     }
+    float4 ca = make_float4(0.f, 0.f, 0.f, 0.f);
+    float2 cb = make_float2(0.f, 0.f);
+    if constexpr (QJ) {
+        ca = qf.qa(lane);
+        cb = qf.qb(lane);
+    }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) finish_logits<QJ>(td[u].kn, ah[u], al[u], ih[u], il[u], qf, lane, L[u]);
+    for (int u = 0; u < 2; ++u) finish_logits<QJ>(td[u].kn, ah[u], al[u], ih[u], il[u], ca, cb, L[u]);
 }
 
 // Online-softmax update and P V for two tiles (one running-maximum check for both).
 template <int D, int KB, int VB, int QJ>
 __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&td)[2], float (&L)[2][4],
-                                                const bool (&v)[2][2], uint32_t lane4v, SplitState<D>& st)
+                                                uint32_t lane4v, SplitState<D>& st)
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
     const bool above = (L[0][0] > st.m0) || (L[0][2] > st.m0) || (L[0][1] > st.m1) || (L[0][3] > st.m1) ||
@@ -1503,12 +1514,10 @@ __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&
         const float p2 = fast_exp2(L[u][2] - st.m0), p3 = fast_exp2(L[u][3] - st.m1);
         st.l0 += p0 + p2;
         st.l1 += p1 + p3;
-        // slots past seq_len may hold anything (even NaN norms): select, never multiply
+        // masked tokens carry |v| = +0 (set by the caller)
         const float2 vnf = __half22float2(*reinterpret_cast<const __half2*>(&td[u].vn));
-        const float vn_g = v[u][0] ? vnf.x : 0.f;
-        const float vn_h = v[u][1] ? vnf.y : 0.f;
-        b0[u] = movmatrix_trans(pack_half2(p0 * vn_g, p1 * vn_g));
-        b1[u] = movmatrix_trans(pack_half2(p2 * vn_h, p3 * vn_h));
+        b0[u] = movmatrix_trans(pack_half2(p0 * vnf.x, p1 * vnf.x));
+        b1[u] = movmatrix_trans(pack_half2(p2 * vnf.y, p3 * vnf.y));
     }
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
@@ -1652,18 +1661,28 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
             }
             float L[2][4];
             pair_logits<D, KB, VB, QJ>(td, qf, lane, lutk, lane4, L);
-            bool v[2][2];
-            v[0][0] = tl0 * 16 + g < seq;
-            v[0][1] = tl0 * 16 + g + 8 < seq;
-            v[1][0] = two && (tl0 + 1) * 16 + g < seq;
-            v[1][1] = two && (tl0 + 1) * 16 + g + 8 < seq;
+            // Tokens at or past seq_len (only in a unit's last pair, or a missing
+            // second tile): logit -inf and value norm +0. Their slots may hold
+            // anything, NaN norms included: select, never multiply.
+            if (!(two && (tl0 + 2) * 16 <= seq)) {   // warp-uniform
 #pragma unroll
-            for (int uu = 0; uu < 2; ++uu) {
-                if (!v[uu][0]) L[uu][0] = L[uu][1] = -CUDART_INF_F;
-                if (!v[uu][1]) L[uu][2] = L[uu][3] = -CUDART_INF_F;
-                stage_words<CB, P2::VW0, P2::VWN, Tr::NWORDS>(sp + uu * TB, lane, td[uu].s);
+                for (int uu = 0; uu < 2; ++uu) {
+                    const int base = (tl0 + uu) * 16 + g;
+                    const bool ok = uu == 0 || two;
+                    if (!(ok && base < seq)) {
+                        L[uu][0] = L[uu][1] = -CUDART_INF_F;
+                        td[uu].vn &= 0xFFFF0000u;
+                    }
+                    if (!(ok && base + 8 < seq)) {
+                        L[uu][2] = L[uu][3] = -CUDART_INF_F;
+                        td[uu].vn &= 0x0000FFFFu;
+                    }
+                }
             }
-            pair_accumulate<D, KB, VB, QJ>(td, L, v, lane4v, st);
+#pragma unroll
+            for (int uu = 0; uu < 2; ++uu)
+                stage_words<CB, P2::VW0, P2::VWN, Tr::NWORDS>(sp + uu * TB, lane, td[uu].s);
+            pair_accumulate<D, KB, VB, QJ>(td, L, lane4v, st);
         }
 
         float l0 = st.l0, l1 = st.l1;
