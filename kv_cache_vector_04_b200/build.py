@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtq.so")
 SOURCES = ["api.cu", "quantize.cu", "attend.cu", "attend_d64.cu", "attend_d128.cu",
            "attend_d256.cu", "noalloc.cu", "tables.cpp"]
-HEADERS = ["device_common.cuh", "kernels.h", "tables.h", "attend_impl.cuh"]
+HEADERS = ["device_common.cuh", "kernels.h", "tables.h", "attend_impl.cuh", "quantize_fast.cuh"]
 
 
 def nvcc_path() -> str:

@@ -70,7 +70,7 @@ struct QuantSmem {
 };
 
 template <int D, int KB, int VB, int QJ>
-__global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArgs a)
+__global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArgs a, int skip_full)
 {
     using Tr = QuantTraits<D, KB, VB, QJ>;
     constexpr int BK = Tr::BK, BV = Tr::BV, M = Tr::M, VPL = Tr::VPL;
@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
     const int lo_slot = max(start - first, 0);
     const int hi_slot = min(start + a.T - first, 16);
     const bool full = (lo_slot == 0 && hi_slot == 16);
+    if (skip_full && full) return;   // quantize_fast owns the full tiles
 
     if (tid < (1 << BK)) ck_s[tid] = tb.centroids_kd[tid];
     if (tid < (1 << BK) - 1) tk_s[tid] = tb.bounds_k[tid];
@@ -420,6 +421,14 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
     if (sat) atomicOr(tb.status, TQ_STATUS_NORM_SAT);
 }
 
+}  // namespace
+}  // namespace tq
+
+#include "quantize_fast.cuh"
+
+namespace tq {
+namespace {
+
 template <int D, int KB, int VB, int QJ>
 cudaError_t launch_quantize_t(const DevTables& tb, const QuantizeArgs& a, cudaStream_t st)
 {
@@ -437,7 +446,21 @@ cudaError_t launch_quantize_t(const DevTables& tb, const QuantizeArgs& a, cudaSt
         if (e != cudaSuccess) return e;
         __atomic_fetch_or(&done, bit, __ATOMIC_ACQ_REL);
     }
-    kern<<<grid, 128, smem, st>>>(tb, a);
+    int skip_full = 0;
+    if constexpr (FastQ<D, KB, VB, QJ>::OK) {
+        auto fk = quantize_fast<D, KB, VB, QJ>;
+        static unsigned long long done_fast = 0;
+        const size_t fsmem = sizeof(QFastSmem<D>);
+        if (!(__atomic_load_n(&done_fast, __ATOMIC_ACQUIRE) & bit)) {
+            e = cudaFuncSetAttribute(fk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
+            if (e != cudaSuccess) return e;
+            __atomic_fetch_or(&done_fast, bit, __ATOMIC_ACQ_REL);
+        }
+        fk<<<dim3((tiles + 3) / 4, a.Hkv, a.B), 128, fsmem, st>>>(tb, a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        skip_full = 1;
+    }
+    kern<<<grid, 128, smem, st>>>(tb, a, skip_full);
     return cudaGetLastError();
 }
 
