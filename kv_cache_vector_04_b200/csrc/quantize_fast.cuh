@@ -233,6 +233,7 @@ struct QWarp {
 template <int D>
 struct QFastSmem {
     QWarp<D> w[4];
+    uint32_t sgt[256];              // sign scatter: the 8 sign bits of n-tiles 2 kk, 2 kk + 1 -> word bits
     uint32_t dmask[D / 2];          // fp16x2 sign-flip masks of coordinate pairs
     double tk[16], tv[16], ck[16];  // boundaries and key centroids (fp64 copies of the fp32 tables)
 };
@@ -253,6 +254,21 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
     if (tid < (1 << KB) - 1) sm.tk[tid] = tb.bounds_k[tid];
     if (tid < (1 << VB) - 1) sm.tv[tid] = tb.bounds_v[tid];
     if (tid < (1 << KB)) sm.ck[tid] = tb.centroids_kd[tid];
+    if constexpr (QJ) {
+        // source bit 4 hs + 2 rw + e (n-tile 2 kk + hs, element 2 rw + e) is the sign
+        // of pair 4 kk + 2 hs + rw, element e: byte fields put it at bit
+        // 6 + rw + 8 hs + 16 e of word kk, sign words at 16 e + 2 hs + rw (+ 4 (kk & 3))
+        for (int x = tid; x < 256; x += 128) {
+            uint32_t v = 0u;
+#pragma unroll
+            for (int bsrc = 0; bsrc < 8; ++bsrc) {
+                if (!((x >> bsrc) & 1)) continue;
+                const int hs = bsrc >> 2, rw = (bsrc >> 1) & 1, e = bsrc & 1;
+                v |= 1u << (TileLayout<D, KB, VB, QJ>::KS_BYTES ? 6 + rw + 8 * hs + 16 * e : 16 * e + 2 * hs + rw);
+            }
+            sm.sgt[x] = v;
+        }
+    }
     __syncthreads();
 
     const int start = a.start_pos[b];
@@ -400,14 +416,25 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
                 }
             }
             const float thr = TAU_Z * 4096.f;
+            // S^T fragments of n-tile nt + 1 load while nt multiplies
+            uint2 bfn[NB];
+#pragma unroll
+            for (int kk = 0; kk < NB; ++kk) bfn[kk] = __ldg(tb.s_frag + (size_t)kk * (D / 8) * 32 + lane);
 #pragma unroll 1
             for (int nt = 0; nt < D / 8; ++nt) {
+                uint2 bf[NB];
+#pragma unroll
+                for (int kk = 0; kk < NB; ++kk) bf[kk] = bfn[kk];
+                if (nt + 1 < D / 8) {
+#pragma unroll
+                    for (int kk = 0; kk < NB; ++kk)
+                        bfn[kk] = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt + 1) * 32 + lane);
+                }
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int kk = 0; kk < NB; ++kk) {
-                    const uint2 bf = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
-                    mma_16816(acc, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], bf.x, bf.y);
-                    mma_16816(acc, al[kk][0], al[kk][1], al[kk][2], al[kk][3], bf.x, bf.y);
+                    mma_16816(acc, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], bf[kk].x, bf[kk].y);
+                    mma_16816(acc, al[kk][0], al[kk][1], al[kk][2], al[kk][3], bf[kk].x, bf[kk].y);
                 }
                 uint32_t bits = 0u, close = 0u;
 #pragma unroll
@@ -534,33 +561,66 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
     // ---------------- the lane string
     // Key pair 4 kk + r: token g + 8 (r & 1) at coordinates 16 kk + 8 (r >> 1) + 2t + e,
     // element c = 2 (r & 1) + e of [kk][hs = r >> 1]; its signs: n-tile 2 kk + hs.
+    // Fields never overlap and s starts at 0, so every field is OR-ed in.
+    using LayT = TileLayout<D, KB, VB, QJ>;
+    constexpr bool KBYTE = LayT::KS_BYTES || KB == 4;       // key pair p = byte p
     uint32_t s[NW];
 #pragma unroll
     for (int i = 0; i < NW; ++i) s[i] = 0u;
+    auto put_or = [&](int pos, uint32_t v, int nb) {
+        const int wi = pos >> 5, o = pos & 31;
+        s[wi] |= v << o;
+        if (o + nb > 32) s[wi + 1] |= v >> (32 - o);
+    };
     constexpr uint32_t VM = (1u << VB) - 1u;
 #pragma unroll
     for (int kk = 0; kk < NB; ++kk) {
+        const uint32_t kw0 = qw.code[0][2 * kk][lane], kw1 = qw.code[0][2 * kk + 1][lane];
+        const uint32_t vw0 = qw.code[1][2 * kk][lane], vw1 = qw.code[1][2 * kk + 1][lane];
+        // byte r = 2 hs + rw of lo / hi: the pair's element 0 / 1
+        const uint32_t lo = __byte_perm(kw0, kw1, 0x6420u), hi = __byte_perm(kw0, kw1, 0x7531u);
+        const uint32_t pairs = lo | (hi << KB);                 // byte r: the pair's KB-bit fields
+        if constexpr (KBYTE) {
+            s[kk] |= pairs;                                     // word kk = pairs 4 kk .. 4 kk + 3
+        } else if constexpr (KB == 2) {
+            const uint32_t t4 = pairs | (pairs >> 4);           // nibble fields
+            put_or(16 * kk, __byte_perm(t4, 0u, 0x4420u) & 0xFFFFu, 16);
+        } else if constexpr (KB == 1) {
+            const uint32_t t2 = pairs | (pairs >> 6);
+            const uint32_t u = __byte_perm(t2, 0u, 0x4420u) & 0xFFFFu;
+            put_or(8 * kk, (u | (u >> 4)) & 0xFFu, 8);
+        } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) put_or(LayT::kbit(4 * kk + r, 0), (pairs >> (8 * r)) & 0xFFu, 2 * KB);
+        }
+        if constexpr (QJ) {
+            const uint32_t sb = (uint32_t)(sgn >> (8 * kk)) & 0xFFu;
+            const uint32_t m = sm.sgt[sb];
+            if constexpr (LayT::KS_BYTES)
+                s[kk] |= m;
+            else
+                s[LayT::SB0 / 32 + (kk >> 2)] |= m << (4 * (kk & 3));
+        }
+        // values: transpose the 8 x 8 blocks (tokens x coordinates); before, lane
+        // (g, t) holds token g + 8 half at coordinates 2t, 2t + 1; after, tokens
+        // 2t, 2t + 1 (+ 8 half) at coordinate g: value pair j = 2 half + hs
 #pragma unroll
         for (int hs = 0; hs < 2; ++hs) {
-            const uint32_t kw = qw.code[0][2 * kk + hs][lane];
-            const uint32_t vw = qw.code[1][2 * kk + hs][lane];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const int pr = 4 * kk + 2 * hs + (c >> 1);
-                put_bits<NW>(s, Lay::kbit(pr, c & 1), (kw >> (8 * c)) & 0xFFu, KB);
-                if constexpr (QJ)
-                    put_bits<NW>(s, Lay::sbit(pr, c & 1), (uint32_t)(sgn >> (4 * (2 * kk + hs) + c)) & 1u, 1);
-            }
-            // values: transpose the 8 x 8 blocks (tokens x coordinates); before, lane
-            // (g, t) holds token g + 8 half at coordinates 2t, 2t + 1; after, tokens
-            // 2t, 2t + 1 (+ 8 half) at coordinate g: value pair j = 2 half + hs
+            const uint32_t vw = hs ? vw1 : vw0;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const uint32_t x = ((vw >> (16 * half)) & 0xFFu) | (((vw >> (16 * half + 8)) & 0xFFu) << 16);
-                const uint32_t tr = movmatrix_trans(x);
                 const int p = 4 * kk + 2 * half + hs;
-                put_bits<NW>(s, Lay::vbit(p, 0), tr & VM, VB);
-                put_bits<NW>(s, Lay::vbit(p, 1), (tr >> 16) & VM, VB);
+                if constexpr (VB == 4) {
+                    // odd tokens shifted by 4 before the transposition: the pair's byte
+                    // is then the OR of the two halves
+                    const uint32_t tr = movmatrix_trans(x << (4 * (g & 1)));
+                    put_or(LayT::vbit(p, 0), (tr | (tr >> 16)) & 0xFFu, 8);
+                } else {
+                    const uint32_t tr = movmatrix_trans(x);
+                    put_or(LayT::vbit(p, 0), tr & VM, VB);
+                    put_or(LayT::vbit(p, 1), (tr >> 16) & VM, VB);
+                }
             }
         }
     }
