@@ -59,31 +59,31 @@ struct SymCells {
         for (int k = 0; k < H; ++k) cm[k] = cents ? (float)cents[H + k] : 0.f;
     }
     // idx = #{j : y > t_j} (ties are within the guard band and go to fp64);
-    // dmin = the smallest distance from y to a boundary the search compared;
-    // cen = c[idx] when CEN.
+    // dacc = min(dacc, distances from y to every boundary the search compared,
+    // 0 included); cen = c[idx] when CEN.
     template <bool CEN>
-    __device__ __forceinline__ uint32_t encode(float y, float& dmin, float& cen) const
+    __device__ __forceinline__ uint32_t encode(float y, float& dacc, float& cen) const
     {
         const float a = fabsf(y);
-        uint32_t m;
+        uint32_t ip;   // H + m: the index of |y| among the non-negative cells
         float c = 0.f;
-        dmin = a;
         if constexpr (B == 1) {
-            m = 0u;
+            ip = 1u;
             c = cm[0];
+            dacc = fminf(dacc, a);
         } else if constexpr (B == 2) {
             const float d1 = a - mb[0];
             const bool c1 = d1 > 0.f;
-            dmin = fminf(dmin, fabsf(d1));
-            m = c1 ? 1u : 0u;
+            dacc = fminf(dacc, fminf(a, fabsf(d1)));
+            ip = c1 ? 3u : 2u;
             if constexpr (CEN) c = c1 ? cm[1] : cm[0];
         } else if constexpr (B == 3) {
             const float d1 = a - mb[1];
             const bool c1 = d1 > 0.f;
             const float d2 = a - (c1 ? mb[2] : mb[0]);
             const bool c2 = d2 > 0.f;
-            dmin = fminf(dmin, fminf(fabsf(d1), fabsf(d2)));
-            m = (c1 ? 2u : 0u) | (c2 ? 1u : 0u);
+            dacc = fminf(fminf(dacc, a), fminf(fabsf(d1), fabsf(d2)));
+            ip = 4u + (c1 ? 2u : 0u) + (c2 ? 1u : 0u);
             if constexpr (CEN) c = c1 ? (c2 ? cm[3] : cm[2]) : (c2 ? cm[1] : cm[0]);
         } else {
             const float d1 = a - mb[3];
@@ -92,16 +92,16 @@ struct SymCells {
             const bool c2 = d2 > 0.f;
             const float d3 = a - (c1 ? (c2 ? mb[6] : mb[4]) : (c2 ? mb[2] : mb[0]));
             const bool c3 = d3 > 0.f;
-            dmin = fminf(dmin, fminf(fabsf(d1), fminf(fabsf(d2), fabsf(d3))));
-            m = (c1 ? 4u : 0u) | (c2 ? 2u : 0u) | (c3 ? 1u : 0u);
+            dacc = fminf(fminf(dacc, a), fminf(fabsf(d1), fminf(fabsf(d2), fabsf(d3))));
+            ip = 8u + (c1 ? 4u : 0u) + (c2 ? 2u : 0u) + (c3 ? 1u : 0u);
             if constexpr (CEN)
                 c = c1 ? (c2 ? (c3 ? cm[7] : cm[6]) : (c3 ? cm[5] : cm[4]))
                        : (c2 ? (c3 ? cm[3] : cm[2]) : (c3 ? cm[1] : cm[0]));
         }
         // y < 0: idx = H - 1 - m = (H + m) ^ (2H - 1)
-        const uint32_t neg = __float_as_uint(y) >> 31;
+        const uint32_t negm = (uint32_t)(__float_as_int(y) >> 31);
         if constexpr (CEN) cen = copysignf(c, y);
-        return ((uint32_t)H + m) ^ ((0u - neg) & (uint32_t)(2 * H - 1));
+        return ip ^ (negm & (uint32_t)(2 * H - 1));
     }
 };
 
@@ -369,26 +369,26 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
     {
         // ---------------- keys: cells (and residuals in place of y)
         rotate(a.k, kn);
-        float rr[2] = {0.f, 0.f};
+        float rr[2] = {0.f, 0.f}, dk[2] = {1.f, 1.f};
 #pragma unroll 1
         for (int i = 0; i < NI; ++i) {
             float4 v = qw.y[i][lane];
             float yy[4] = {v.x, v.y, v.z, v.w};
-            uint32_t word = 0u;
+            uint32_t idx[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float dmin, cen;
-                const uint32_t idx = kcells.template encode<QJ != 0>(yy[c], dmin, cen);
-                fixk[c >> 1] |= dmin < TAU_Y;
-                word |= idx << (8 * c);
+                float cen;
+                idx[c] = kcells.template encode<QJ != 0>(yy[c], dk[c >> 1], cen);
                 if constexpr (QJ) {
                     yy[c] -= cen;
                     rr[c >> 1] = fmaf(yy[c], yy[c], rr[c >> 1]);
                 }
             }
-            qw.code[0][i][lane] = word;
+            qw.code[0][i][lane] = __byte_perm(__byte_perm(idx[0], idx[1], 0x0040u), __byte_perm(idx[2], idx[3], 0x0040u), 0x5410u);
             if constexpr (QJ) qw.y[i][lane] = make_float4(yy[0], yy[1], yy[2], yy[3]);
         }
+        fixk[0] = dk[0] < TAU_Y;
+        fixk[1] = dk[1] < TAU_Y;
         if constexpr (QJ) {
 #pragma unroll
             for (int o = 1; o <= 2; o <<= 1) {
@@ -436,14 +436,18 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
                     mma_16816(acc, ah[kk][0], ah[kk][1], ah[kk][2], ah[kk][3], bf[kk].x, bf[kk].y);
                     mma_16816(acc, al[kk][0], al[kk][1], al[kk][2], al[kk][3], bf[kk].x, bf[kk].y);
                 }
-                uint32_t bits = 0u, close = 0u;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    bits |= (acc[c] >= 0.f ? 1u : 0u) << c;
-                    close |= (fabsf(acc[c]) < thr ? 1u : 0u) << c;
-                }
+                // sign bits: the complemented float sign bits (z >= 0 -> 1; -0 counts as 0,
+                // and |z| = 0 is a close call anyway)
+                const uint32_t bits =
+                    (~((__float_as_uint(acc[0]) >> 31) | ((__float_as_uint(acc[1]) >> 30) & 2u) |
+                       ((__float_as_uint(acc[2]) >> 29) & 4u) | ((__float_as_uint(acc[3]) >> 28) & 8u))) & 15u;
                 sgn |= (unsigned long long)bits << (4 * nt);
-                zcl |= (unsigned long long)close << (4 * nt);
+                if (fminf(fminf(fabsf(acc[0]), fabsf(acc[1])), fminf(fabsf(acc[2]), fabsf(acc[3]))) < thr) {
+                    uint32_t close = 0u;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) close |= (fabsf(acc[c]) < thr ? 1u : 0u) << c;
+                    zcl |= (unsigned long long)close << (4 * nt);
+                }
             }
             // rows with a close call (elements 0, 1: token g; 2, 3: token g + 8)
             fixk[0] |= (zcl & 0x3333333333333333ull) != 0ull;
@@ -453,20 +457,21 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
     {
         // ---------------- values: cells
         rotate(a.v, vn);
+        float dv[2] = {1.f, 1.f};
 #pragma unroll 1
         for (int i = 0; i < NI; ++i) {
             const float4 v = qw.y[i][lane];
             const float yy[4] = {v.x, v.y, v.z, v.w};
-            uint32_t word = 0u;
+            uint32_t idx[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float dmin, cen;
-                const uint32_t idx = vcells.template encode<false>(yy[c], dmin, cen);
-                fixv[c >> 1] |= dmin < TAU_Y;
-                word |= idx << (8 * c);
+                float cen;
+                idx[c] = vcells.template encode<false>(yy[c], dv[c >> 1], cen);
             }
-            qw.code[1][i][lane] = word;
+            qw.code[1][i][lane] = __byte_perm(__byte_perm(idx[0], idx[1], 0x0040u), __byte_perm(idx[2], idx[3], 0x0040u), 0x5410u);
         }
+        fixv[0] = dv[0] < TAU_Y;
+        fixv[1] = dv[1] < TAU_Y;
     }
     __syncwarp();
 
