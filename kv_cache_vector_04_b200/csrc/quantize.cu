@@ -96,7 +96,11 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
         if (tid == 0 && blockIdx.x == 0 && h == 0) atomicOr(tb.status, TQ_STATUS_CAPACITY);
         return;
     }
-    const int tile = start / 16 + blockIdx.x;
+    // With skip_full only the first and the last tile the tokens touch can be
+    // partial: the grid then has two CTAs per (batch, head), x = 0 and 1.
+    const int span = (start + a.T - 1) / 16 - start / 16;   // touched tiles - 1
+    if (skip_full && blockIdx.x == 1 && span == 0) return;
+    const int tile = start / 16 + (skip_full ? (blockIdx.x == 0 ? 0 : span) : (int)blockIdx.x);
     const int first = tile * 16;
     if (first >= start + a.T) return;
     const int lo_slot = max(start - first, 0);
@@ -459,6 +463,7 @@ cudaError_t launch_quantize_t(const DevTables& tb, const QuantizeArgs& a, cudaSt
         fk<<<dim3((tiles + 3) / 4, a.Hkv, a.B), 128, fsmem, st>>>(tb, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         skip_full = 1;
+        grid.x = 2;
     }
     kern<<<grid, 128, smem, st>>>(tb, a, skip_full);
     return cudaGetLastError();
