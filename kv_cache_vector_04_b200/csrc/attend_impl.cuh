@@ -158,6 +158,20 @@ __device__ __forceinline__ uint32_t row_off(uint32_t w, int r, uint32_t lane4)
     return __byte_perm(w, lane4, 0x7604u | ((uint32_t)r << 4));
 }
 
+// Two and four consecutive 32-bit entries at shared address x.
+__device__ __forceinline__ uint2 lds64(uint32_t x)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(x));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t x)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(x));
+    return v;
+}
+
 // A table entry: at `table` + x, or (ABS) at shared address x.
 template <bool ABS = false>
 __device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t x)
@@ -1390,6 +1404,17 @@ struct PairTraits {
     // table; else its own table at LUT_ADDR + 32 KB (aligned above its size, so
     // an OR with a field offset still yields a full address)
     static constexpr uint32_t V_OFF = Tr::ROWS ? 128u : 0x8000u;
+    // Wide rows for 1- and 2-bit key cells: one byte of the key words holds
+    // NRK = 4 or 2 key pairs, i.e. that many consecutive A registers of a
+    // k-step, so row b of a 256-row table holds all of them (entries of
+    // 4 NRK bytes, replicated over 32 / NRK lanes: an LDS.64 or LDS.128 of a
+    // warp is then conflict-free) in the first 128 bytes of a 256-byte row.
+    // The second 128 bytes hold the value entry: the same wide entry for
+    // 2-bit values (two pairs a byte), else the 32-lane entry of field b.
+    // One byte permute gives a row's full shared address.
+    static constexpr bool WK = !Tr::ROWS && !Tr::CK && (KB == 1 || KB == 2);
+    static constexpr int NRK = KB == 1 ? 4 : 2;
+    static constexpr bool WV = WK && VB == 2;
     static_assert(Tr::ROWS || ((size_t)Tr::NLK * 128 <= 0x8000 && (size_t)Tr::NLV * 128 <= 0x8000),
                   "small tables fit their 32 KB halves");
     // lane-string words holding the key operands (codes and, byte-field keys, signs) and the values
@@ -1437,13 +1462,24 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             uint32_t ak[4];
+            if constexpr (PairTraits<D, KB, VB, QJ>::WK && KB == 2) {
+                // key pairs 4 kk + r: bytes 2 (kk & 1) (r = 0, 1) and + 1 (r = 2, 3) of word kk / 2
+                const uint2 x0 = lds64(row_off(td[u].s[kk >> 1], 2 * (kk & 1), lane4));
+                const uint2 x1 = lds64(row_off(td[u].s[kk >> 1], 2 * (kk & 1) + 1, lane4));
+                ak[0] = x0.x; ak[1] = x0.y; ak[2] = x1.x; ak[3] = x1.y;
+            } else if constexpr (PairTraits<D, KB, VB, QJ>::WK) {
+                // key pairs 4 kk .. 4 kk + 3: byte kk & 3 of word kk / 4
+                const uint4 x = lds128(row_off(td[u].s[kk >> 2], kk & 3, lane4));
+                ak[0] = x.x; ak[1] = x.y; ak[2] = x.z; ak[3] = x.w;
+            } else {
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int p = 4 * kk + r;
-                if constexpr (Tr::PK)
-                    ak[r] = lut_load<true>(lutk, row_off(td[u].s[kk], r, lane4));
-                else
-                    ak[r] = lut_load<true>(lutk, lut_off<Tr::LSH>(td[u].s, Tr::KF * p, Tr::KF, lane4));
+                for (int r = 0; r < 4; ++r) {
+                    const int p = 4 * kk + r;
+                    if constexpr (Tr::PK)
+                        ak[r] = lut_load<true>(lutk, row_off(td[u].s[kk], r, lane4));
+                    else
+                        ak[r] = lut_load<true>(lutk, lut_off<Tr::LSH>(td[u].s, Tr::KF * p, Tr::KF, lane4));
+                }
             }
             if (kk == 0) {
                 mma_16816_first(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
@@ -1524,11 +1560,20 @@ __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             uint32_t av[4];
+            if constexpr (PairTraits<D, KB, VB, QJ>::WV) {
+                // value pairs 4 kk + j: bytes 2 (kk & 1) (j = 0, 1) and + 1 of value word kk / 2
+                const uint32_t w = td[u].s[Tr::VW0 + (kk >> 1)];
+                const uint2 x0 = lds64(row_off(w, 2 * (kk & 1), lane4v));
+                const uint2 x1 = lds64(row_off(w, 2 * (kk & 1) + 1, lane4v));
+                av[0] = x0.x; av[1] = x0.y; av[2] = x1.x; av[3] = x1.y;
+            } else {
+                constexpr int VSH = PairTraits<D, KB, VB, QJ>::WK ? 8 : Tr::LSH;   // row stride
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                av[r] = Tr::PV ? lut_load<true>(nullptr, row_off(td[u].s[Tr::VW0 + kk], r, lane4v))
-                               : lut_load<true>(nullptr, lut_off<Tr::LSH>(td[u].s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
+                for (int r = 0; r < 4; ++r)
+                    av[r] = Tr::PV ? lut_load<true>(nullptr, row_off(td[u].s[Tr::VW0 + kk], r, lane4v))
+                                   : lut_load<true>(nullptr, lut_off<VSH>(td[u].s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
                                                                           Tr::VF, lane4v));
+            }
             mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0[u], b1[u]);
         }
     }
@@ -1556,9 +1601,32 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
     const int c = blockIdx.x;
     const long long G = gridDim.x;
     const int groups = a.plan.groups, upb = a.Hkv * groups;
-    fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
+    if constexpr (P2::WK) {
+        // 256 rows of 64 words: key entry of byte x (NRK words, 32 / NRK replicas), then the
+        // value entry (2-bit values: two words, 16 replicas; else field x, 32 replicas)
+        constexpr int FK = 2 * KB;
+        for (int e = tid; e < 256 * 64; e += NT) {
+            const int x = e >> 6, col = e & 63;
+            uint32_t v;
+            if (col < 32) {
+                const int i = col % P2::NRK;
+                v = __ldg(tb.lut_k + ((x >> (FK * i)) & ((1 << FK) - 1)));
+            } else if constexpr (P2::WV) {
+                v = __ldg(tb.lut_v + ((x >> (4 * (col & 1))) & 15));
+            } else {
+                v = x < Tr::NLV ? __ldg(tb.lut_v + x) : 0u;
+            }
+            lutk[e] = v;
+        }
+    } else {
+        fill_luts<D, KB, VB, QJ, NT>(tb, lutk, lutv, tid);
+    }
     // full shared addresses of this lane's table entries
-    const uint32_t lane4 = P2::LUT_ADDR + 4u * lane, lane4v = lane4 + P2::V_OFF;
+    const uint32_t lane4 = P2::WK ? P2::LUT_ADDR + (uint32_t)(lane % (32 / P2::NRK)) * (4u * P2::NRK)
+                                  : P2::LUT_ADDR + 4u * lane;
+    const uint32_t lane4v = P2::WK ? (P2::WV ? P2::LUT_ADDR + 128u + (uint32_t)(lane & 15) * 8u
+                                             : P2::LUT_ADDR + 128u + 4u * lane)
+                                   : lane4 + P2::V_OFF;
     uint8_t* ring = w < P2::WA ? dyn + P2::QF + (size_t)w * P2::RPW : above + (size_t)(w - P2::WA) * P2::RPW;
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
     const uint32_t bar_s = (uint32_t)__cvta_generic_to_shared(bars + w * 2);
