@@ -74,3 +74,17 @@ def test_l2_note():
 def test_whole_job_gbs():
     # 2 ranks x 562 MB in a 0.2 ms slowest step: 5620 GB/s
     assert abs(bench.whole_job_gbs(2 * 562e6, 0.2) - 5620.0) < 1e-9
+
+
+def test_reference_arm_inputs_do_not_map_the_cuda_library():
+    # The reference arm takes its workload and seeded inputs from inputs.py
+    # without importing the package, whose __init__ loads libtq.so.
+    import subprocess
+    code = ("import sys; sys.path.insert(0, %r); import bench; "
+            "w = bench.workload_by_name(bench.DEFAULT_WORKLOAD); "
+            "q = bench.load_inputs().queries(w, B=1, Hq=8); "
+            "assert q.shape == (1, 8, w.d), q.shape; "
+            "assert 'kv_cache_vector_04_b200' not in sys.modules; "
+            "assert 'libtq' not in open('/proc/self/maps').read(); print('ok')" % ROOT)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr[-2000:]
