@@ -51,7 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the other long-context workloads reported beside the bench line")
-    ap.add_argument("--report", choices=["all", "single", "qwen3b", "qwen32b", "sweep", "formats"],
+    ap.add_argument("--report", choices=["all", "single", "qwen3b", "qwen32b", "sweep", "formats",
+                                         "cudacore"],
                     default=None,
                     help="measure the other workloads instead of the bench line: one JSON line each")
     return ap.parse_args(argv)
@@ -655,6 +656,48 @@ def report_single_head():
             "note": "1.6 MB of packed cache, resident in L2: launch-latency bound"}
 
 
+def report_cudacore():
+    """The tensor-core split kernel against the CUDA-core comparison kernel
+    (lookup tables; QJL term by sign-nibble tables, then by bit-plane
+    popcounts) on one Llama-3.3-70B-shaped layer: tq_attend calls over the
+    same 562 MB cache (larger than L2), CUDA events around each arm's calls."""
+    import torch
+    import kv_cache_vector_04_b200 as tq
+    inputs = load_inputs()
+    w = inputs.WORKLOADS[DEFAULT_WORKLOAD]
+    dev = torch.device("cuda", 0)
+    ctx = tq.tq_init(w.d, w.bits, 1)
+    N = w.N
+    cache = tq.new_cache(ctx, w.B, w.Hkv, N + 16, device=dev)
+    k, v = inputs.kv_pair(w, N, layer=0, device=dev)
+    tq.tq_quantize(ctx, k, v, torch.zeros(w.B, dtype=torch.int32, device=dev), cache)
+    del k, v
+    q = inputs.queries(w, layer=0, device=dev)
+    seq = torch.full((w.B,), N, dtype=torch.int32, device=dev)
+    ws = tq.new_workspace(ctx, w.B, w.Hq, w.Hkv, N)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    per_tok = tq.tq_cache_layout(ctx)["tile_bytes"] // 16
+    nbytes = w.B * w.Hkv * N * per_tok
+    peak, peak_kind = measured_peaks()
+    arms = [("tensor_core", lambda: tq.tq_attend(ctx, q, cache, seq, N, out=out, workspace=ws), 20),
+            ("cuda_core_nibble_qjl", lambda: tq.tq_attend_cudacore(ctx, q, cache, seq, N, 1, out=out,
+                                                                   workspace=ws), 5),
+            ("cuda_core_popcount_qjl", lambda: tq.tq_attend_cudacore(ctx, q, cache, seq, N, 2, out=out,
+                                                                     workspace=ws), 2)]
+    res = {"report": "cudacore_llama70b_32k", "workload": w.name, "bytes_per_call": nbytes,
+           "peak_gbs": peak, "peak_kind": peak_kind}
+    for name, fn, reps in arms:
+        clocks = ClockSampler(0)
+        clocks.start()
+        ms = _time_ms(fn, reps, warm=2)
+        clk = clocks.stop()
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[name] = {"ms_per_call": round(ms, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                     "calls": reps, "sm_mhz": clk.get("sm_mhz"), "reasons": clk.get("reasons")}
+    assert tq.tq_status(ctx) == 0
+    return res
+
+
 def _brief(line: dict) -> dict:
     keep = {"value": line["value"], "unit": line["unit"], "ms_per_step": line["ms_per_step"],
             "ms_per_step_eager": line.get("ms_per_step_eager"),
@@ -690,6 +733,8 @@ def run_report(args, dist: Dist):
         for w in inputs.sweep_workloads():
             print(json.dumps(dict(report=w.name, **run(workload=w.name, layers=1, steps=10,
                                                          warmup=3))), flush=True)
+    if which in ("all", "cudacore"):
+        print(json.dumps(report_cudacore()), flush=True)
     if which in ("all", "formats"):
         from kv_cache_vector_04_b200 import inputs
         for w in inputs.format_workloads():

@@ -246,6 +246,30 @@ int tq_scores(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_c
               const int32_t* seq_len, int max_len, float* scores, void* workspace,
               size_t workspace_bytes, void* stream);
 
+/* tq_attend computed on CUDA cores instead of tensor cores, kept as a measured
+ * comparison for the tensor-core split kernel (it is several times slower).
+ * The operation, the arguments, the workspace and the prologue and reduce
+ * launches are those of tq_attend; only the split kernel differs. It reads the
+ * tiles with the same bulk copies and the same stream-K split, and writes the
+ * same partials. Per unit of 8 query heads it builds shared-memory lookup tables:
+ *  - the logits' codebook term sum_i q~_i c[idx_i] from a table of
+ *    q~_i x c[code] per (coordinate, code, head);
+ *  - the QJL term sum_j (2 s_j - 1) x_j (x = S q~ in the fixed point of the
+ *    tensor-core path) from one of two tables:
+ *    qjl_mode TQ_CC_QJL_NIBBLE: per group of 4 signs, the 16 signed sums;
+ *    qjl_mode TQ_CC_QJL_POPCOUNT: the 16 bit planes of the fixed-point x,
+ *    sum_b w_b popc(signs & plane_b).
+ * P V runs as fp32 FMAs. Built for d = 128 with TurboQuant at 4 bits only
+ * (tq_init(128, 4, ...)); any other context returns TQ_ERR_UNSUPPORTED, and
+ * any other qjl_mode returns TQ_ERR_INVALID_ARG. The estimator is the one
+ * tq_attend implements (the logit estimate at the top of this file, from
+ * §"TurboQuant 是什麼：30 秒懶人包" of the ai-muninn page). */
+#define TQ_CC_QJL_NIBBLE 1
+#define TQ_CC_QJL_POPCOUNT 2
+int tq_attend_cudacore(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,
+                       const int32_t* seq_len, int max_len, float* out, void* workspace,
+                       size_t workspace_bytes, int qjl_mode, void* stream);
+
 /* tq_attend without a workspace argument, for callers that cannot allocate
  * device memory: runtimes whose device memory belongs to an allocator they do
  * not control, and serving loops that forbid allocation after start-up. (The

@@ -27,6 +27,8 @@ TQ_STATUS_CAPACITY = 0x1
 TQ_STATUS_SEQ_LEN = 0x2
 TQ_STATUS_NORM_SAT = 0x4
 TQ_STATUS_WAIT_TIMEOUT = 0x8
+TQ_CC_QJL_NIBBLE = 1
+TQ_CC_QJL_POPCOUNT = 2
 TQ_TILE = 16
 TQ_CODEBOOK_GAUSS = 0
 TQ_CODEBOOK_BETA = 1
@@ -36,7 +38,8 @@ TQ_DTYPE_BF16 = 1
 # every symbol include/tq.h declares
 EXPORTS = ("tq_init", "tq_init_ex", "tq_build_codebook", "tq_destroy", "tq_cache_layout", "tq_cache_bytes", "tq_get_tables",
            "tq_build_tables", "tq_quantize", "tq_attend_workspace", "tq_attend", "tq_scores",
-           "tq_attend_noalloc", "tq_append_attend", "tq_status", "tq_copy", "tq_strerror")
+           "tq_attend_noalloc", "tq_append_attend", "tq_attend_cudacore", "tq_status", "tq_copy",
+           "tq_strerror")
 TQ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -79,6 +82,7 @@ def _load(path: str = LIB_PATH):
         "tq_attend": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, P]),
         "tq_scores": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, P]),
         "tq_attend_noalloc": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P]),
+        "tq_attend_cudacore": (I, [P, P, I, I, I, ctypes.POINTER(_Cache), P, I, P, P, SZ, I, P]),
         "tq_append_attend": (I, [P, P, I, P, P, I, I, I, P, ctypes.POINTER(_Cache), P, I, P, P,
                                  SZ, P]),
         "tq_status": (I, [P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -310,6 +314,28 @@ def tq_attend(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor
         out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     return _attend_like(_lib.tq_attend, "tq_attend", ctx, q, cache, seq_len, max_len, out,
                         workspace, stream)
+
+
+def tq_attend_cudacore(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor,
+                       max_len: int, qjl_mode: int = 1, out: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, stream=None):
+    """tq_attend with the split kernel on CUDA cores (lookup tables; QJL term by
+    sign-nibble tables, qjl_mode 1, or bit-plane popcounts, qjl_mode 2): the
+    measured comparison for the tensor-core kernel. d = 128, 4-bit TurboQuant only."""
+    if q.dim() != 3 or q.shape[2] != ctx.d:
+        raise ValueError("q must be [B, Hq, d] with d = %d" % ctx.d)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    B, Hq, _ = q.shape
+    if workspace is None:
+        workspace = new_workspace(ctx, B, Hq, cache.Hkv, max_len)
+    c = cache.struct()
+    _check(_lib.tq_attend_cudacore(ctx.handle, _dev(q, "q"), _q_dtype(q), B, Hq, ctypes.byref(c),
+                                   _dev(seq_len, "seq_len", torch.int32), int(max_len),
+                                   _dev(out, "out", torch.float32), _dev(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), int(qjl_mode),
+                                   ctypes.c_void_p(_stream_ptr(stream))), "tq_attend_cudacore")
+    return out
 
 
 def tq_scores(ctx: Context, q: torch.Tensor, cache: Cache, seq_len: torch.Tensor, max_len: int,

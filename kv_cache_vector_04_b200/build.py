@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtq.so")
 SOURCES = ["api.cu", "quantize.cu", "attend.cu", "attend_d64.cu", "attend_d128.cu",
            "attend_d256.cu", "noalloc.cu", "tables.cpp"]
-HEADERS = ["device_common.cuh", "kernels.h", "tables.h", "attend_impl.cuh", "quantize_fast.cuh"]
+HEADERS = ["device_common.cuh", "kernels.h", "tables.h", "attend_impl.cuh", "attend_cc.cuh",
+           "quantize_fast.cuh"]
 
 
 def nvcc_path() -> str:

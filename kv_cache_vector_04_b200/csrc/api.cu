@@ -195,7 +195,7 @@ int quantize_common(tq_ctx* ctx, const void* k, const void* v, int B, int Hkv, i
 int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,
                   const int32_t* seq_len, int max_len, float* out, void* ws, size_t ws_bytes,
                   void* stream, bool scores, const void* k = nullptr, const void* v = nullptr,
-                  int T = 0, const int32_t* start_pos = nullptr)
+                  int T = 0, const int32_t* start_pos = nullptr, int cc_mode = 0)
 {
     if (!ctx || !q || !seq_len || !out) return TQ_ERR_INVALID_ARG;
     if (q_dtype != TQ_DTYPE_F16 && q_dtype != TQ_DTYPE_BF16) return TQ_ERR_INVALID_ARG;
@@ -244,6 +244,7 @@ int attend_common(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const 
                                          align256(plan.prefix_bytes));
     a.out = out;
     a.plan = plan;
+    a.cc_mode = cc_mode;
     const cudaError_t e = tq::launch_attend(ctx_format(ctx), ctx->tables, a, scores,
                                             static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
@@ -422,6 +423,17 @@ int tq_attend(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_c
 {
     return attend_common(ctx, q, q_dtype, B, Hq, cache, seq_len, max_len, out, workspace,
                          workspace_bytes, stream, false);
+}
+
+int tq_attend_cudacore(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,
+                       const int32_t* seq_len, int max_len, float* out, void* workspace,
+                       size_t workspace_bytes, int qjl_mode, void* stream)
+{
+    if (!ctx) return TQ_ERR_INVALID_ARG;
+    if (ctx->d != 128 || ctx->kbits != 3 || ctx->vbits != 4 || ctx->qjl != 1) return TQ_ERR_UNSUPPORTED;
+    if (qjl_mode != TQ_CC_QJL_NIBBLE && qjl_mode != TQ_CC_QJL_POPCOUNT) return TQ_ERR_INVALID_ARG;
+    return attend_common(ctx, q, q_dtype, B, Hq, cache, seq_len, max_len, out, workspace,
+                         workspace_bytes, stream, false, nullptr, nullptr, 0, nullptr, qjl_mode);
 }
 
 int tq_scores(tq_ctx* ctx, const void* q, int q_dtype, int B, int Hq, const tq_cache* cache,

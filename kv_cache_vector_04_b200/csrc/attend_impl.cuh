@@ -919,11 +919,13 @@ struct QueryFrags {
 // Logits (log2 units) of tokens g, g + 8 and heads 2t, 2t + 1 from the
 // codebook sums (two fp32 chains: the hi and lo parts of the B operands) and the
 // QJL integer sums (high, low byte chains): L = |k| (c + rho (acc u 2/sigma - u T)).
-// ca, cb: the lane's QJL constants (QueryFrags::qa, qb).
-template <int QJ>
+// ca, cb: the lane's QJL constants (QueryFrags::qa, qb). With OFF, the
+// logits come out offset by the softmax references of heads 2t, 2t+1:
+// L - m, one rounding (nm = {-m0, -m1}).
+template <int QJ, bool ONE = false, bool OFF = false>
 __device__ __forceinline__ void finish_logits(const uint2 kn, const float (&ah)[4], const float (&al)[4], const int (&ih)[4],
                                               const int (&il)[4], const float4 ca, const float2 cb,
-                                              float (&L)[4])
+                                              float (&L)[4], float2 nm = make_float2(0.f, 0.f))
 {
     if constexpr (QJ) {
         const float2 kg = __half22float2(*reinterpret_cast<const __half2*>(&kn.x));   // |k_g|, rho_g
@@ -933,19 +935,48 @@ __device__ __forceinline__ void finish_logits(const uint2 kn, const float (&ah)[
         const float y2 = fmaf((float)(ih[2] * 256 + il[2]), ca.z, cb.x);
         const float y3 = fmaf((float)(ih[3] * 256 + il[3]), ca.w, cb.y);
         const float ng = kg.x * (1.0f / 128.0f), nh = kh.x * (1.0f / 128.0f);   // the B operands carry 2^7
-        L[0] = ng * fmaf(kg.y, y0, ah[0] + al[0]);
-        L[1] = ng * fmaf(kg.y, y1, ah[1] + al[1]);
-        L[2] = nh * fmaf(kh.y, y2, ah[2] + al[2]);
-        L[3] = nh * fmaf(kh.y, y3, ah[3] + al[3]);
+        const float x0 = fmaf(kg.y, y0, ONE ? ah[0] : ah[0] + al[0]);
+        const float x1 = fmaf(kg.y, y1, ONE ? ah[1] : ah[1] + al[1]);
+        const float x2 = fmaf(kh.y, y2, ONE ? ah[2] : ah[2] + al[2]);
+        const float x3 = fmaf(kh.y, y3, ONE ? ah[3] : ah[3] + al[3]);
+        if constexpr (OFF) {
+            L[0] = fmaf(ng, x0, nm.x);
+            L[1] = fmaf(ng, x1, nm.y);
+            L[2] = fmaf(nh, x2, nm.x);
+            L[3] = fmaf(nh, x3, nm.y);
+        } else {
+            L[0] = ng * x0;
+            L[1] = ng * x1;
+            L[2] = nh * x2;
+            L[3] = nh * x3;
+        }
     } else {
         const float2 kk2 = __half22float2(*reinterpret_cast<const __half2*>(&kn.x));
         const float ng = kk2.x * (1.0f / 128.0f), nh = kk2.y * (1.0f / 128.0f);
-        L[0] = ng * (ah[0] + al[0]);
-        L[1] = ng * (ah[1] + al[1]);
-        L[2] = nh * (ah[2] + al[2]);
-        L[3] = nh * (ah[3] + al[3]);
+        const float x0 = ONE ? ah[0] : ah[0] + al[0], x1 = ONE ? ah[1] : ah[1] + al[1];
+        const float x2 = ONE ? ah[2] : ah[2] + al[2], x3 = ONE ? ah[3] : ah[3] + al[3];
+        if constexpr (OFF) {
+            L[0] = fmaf(ng, x0, nm.x);
+            L[1] = fmaf(ng, x1, nm.y);
+            L[2] = fmaf(nh, x2, nm.x);
+            L[3] = fmaf(nh, x3, nm.y);
+        } else {
+            L[0] = ng * x0;
+            L[1] = ng * x1;
+            L[2] = nh * x2;
+            L[3] = nh * x3;
+        }
     }
 }
+
+// Lazy rescale of the online softmax. The reference m of each head (the
+// exponent offset of l and acc) only has to bound every logit seen so far, so
+// that each p = exp2(L - m) <= 1; it need not be the running maximum. When a
+// logit exceeds it, m moves to the new maximum plus this slack (log2 units),
+// which makes later moves rare: for logits of unit spread, about one warp
+// iteration in 16 moves it instead of one in 3. Every merge weights a partial
+// by exp2(m - M), so any such bound gives the same result up to rounding.
+constexpr float kRescaleSlack = 2.0f;
 
 template <int D>
 struct SplitState {
@@ -1020,9 +1051,10 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, KB, VB, QJ>& t
                                                 SplitState<D>& st)
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    // The running max only moves when some logit exceeds it (rarely, after the
-    // first tiles): only then reduce across the 8 token lanes and rescale.
-    // Otherwise every p = exp2(L - m) <= 1, which also keeps p*|v| in fp16 range.
+    // The reference of each head only moves when some logit exceeds it (rarely,
+    // after the first tiles; see kRescaleSlack): only then reduce across the 8
+    // token lanes and rescale. Every p = exp2(L - m) <= 1, which also keeps
+    // p*|v| in fp16 range.
     const bool above = (L[0] > st.m0) || (L[2] > st.m0) || (L[1] > st.m1) || (L[3] > st.m1);
     if (__any_sync(kFull, above)) {
         float mx0 = fmaxf(L[0], L[2]), mx1 = fmaxf(L[1], L[3]);
@@ -1031,7 +1063,7 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, KB, VB, QJ>& t
             mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
             mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
         }
-        const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+        const float mn0 = fmaxf(st.m0, mx0 + kRescaleSlack), mn1 = fmaxf(st.m1, mx1 + kRescaleSlack);
         const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
         st.l0 *= al0;
         st.l1 *= al1;
@@ -1450,11 +1482,17 @@ __device__ __forceinline__ void stage_words(const uint8_t* slot, int lane, uint3
 // query fragments of each k-step serve both tiles.
 template <int D, int KB, int VB, int QJ, typename QF>
 __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[2], const QF& qf, int lane,
-                                            const uint32_t* lutk, uint32_t lane4, float (&L)[2][4])
+                                            const uint32_t* lutk, uint32_t lane4, float2 nm, float (&L)[2][4])
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
     constexpr int SL = SignLayout<KB, QJ>::SL;
-    float ah[2][4], al[2][4];   // codebook term: the hi and lo B parts
+    // Codebook term: the hi and lo B parts in two accumulator chains, or, for
+    // byte-field keys, in one. (Measured at (3, 4, 1), d = 128: one chain alone
+    // gained nothing, the lazy rescale with offset logits alone nothing, both
+    // together -2.5 % per layer; at (2, 3, 1) and (1, 2, 1) one chain cost
+    // 3 % and 7 %.)
+    constexpr bool ONE = Tr::PK;
+    float ah[2][4], al[2][4];
     int ih[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, il[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
     for (int kk = 0; kk < Tr::KK; ++kk) {
@@ -1483,10 +1521,11 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
             }
             if (kk == 0) {
                 mma_16816_first(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
-                mma_16816_first(al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+                if constexpr (ONE) mma_16816(ah[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+                else mma_16816_first(al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
             } else {
                 mma_16816(ah[u], ak[0], ak[1], ak[2], ak[3], bc.x, bc.y);
-                mma_16816(al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
+                mma_16816(ONE ? ah[u] : al[u], ak[0], ak[1], ak[2], ak[3], bc.z, bc.w);
             }
         }
         if constexpr (QJ) {
@@ -1510,18 +1549,21 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
         cb = qf.qb(lane);
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) finish_logits<QJ>(td[u].kn, ah[u], al[u], ih[u], il[u], ca, cb, L[u]);
+    for (int u = 0; u < 2; ++u) finish_logits<QJ, ONE, true>(td[u].kn, ah[u], al[u], ih[u], il[u], ca, cb, L[u], nm);
 }
 
-// Online-softmax update and P V for two tiles (one running-maximum check for both).
+// Online-softmax update and P V for two tiles (one reference check for both).
+// L holds the logits already offset by the references (L - m, see
+// finish_logits). The first pair of a segment sets the references from
+// scratch (m = 0 until then, with l and acc empty).
 template <int D, int KB, int VB, int QJ>
 __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&td)[2], float (&L)[2][4],
-                                                uint32_t lane4v, SplitState<D>& st)
+                                                uint32_t lane4v, SplitState<D>& st, bool first)
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    const bool above = (L[0][0] > st.m0) || (L[0][2] > st.m0) || (L[0][1] > st.m1) || (L[0][3] > st.m1) ||
-                       (L[1][0] > st.m0) || (L[1][2] > st.m0) || (L[1][1] > st.m1) || (L[1][3] > st.m1);
-    if (__any_sync(kFull, above)) {
+    const bool above = (L[0][0] > 0.f) || (L[0][2] > 0.f) || (L[0][1] > 0.f) || (L[0][3] > 0.f) ||
+                       (L[1][0] > 0.f) || (L[1][2] > 0.f) || (L[1][1] > 0.f) || (L[1][3] > 0.f);
+    if (__any_sync(kFull, above) || first) {
         float mx0 = fmaxf(fmaxf(L[0][0], L[0][2]), fmaxf(L[1][0], L[1][2]));
         float mx1 = fmaxf(fmaxf(L[0][1], L[0][3]), fmaxf(L[1][1], L[1][3]));
 #pragma unroll
@@ -1529,8 +1571,10 @@ __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&
             mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, sh));
             mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, sh));
         }
-        const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
-        const float al0 = fast_exp2(st.m0 - mn0), al1 = fast_exp2(st.m1 - mn1);
+        // the references move up by d (every pair holds a valid token, so mx is finite)
+        const float d0 = first ? mx0 + kRescaleSlack : fmaxf(mx0 + kRescaleSlack, 0.f);
+        const float d1 = first ? mx1 + kRescaleSlack : fmaxf(mx1 + kRescaleSlack, 0.f);
+        const float al0 = first ? 0.f : fast_exp2(-d0), al1 = first ? 0.f : fast_exp2(-d1);
         st.l0 *= al0;
         st.l1 *= al1;
 #pragma unroll
@@ -1540,14 +1584,21 @@ __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&
             st.acc[kk][2] *= al0;
             st.acc[kk][3] *= al1;
         }
-        st.m0 = mn0;
-        st.m1 = mn1;
+        st.m0 += d0;
+        st.m1 += d1;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            L[u][0] -= d0;
+            L[u][2] -= d0;
+            L[u][1] -= d1;
+            L[u][3] -= d1;
+        }
     }
     uint32_t b0[2], b1[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-        const float p0 = fast_exp2(L[u][0] - st.m0), p1 = fast_exp2(L[u][1] - st.m1);
-        const float p2 = fast_exp2(L[u][2] - st.m0), p3 = fast_exp2(L[u][3] - st.m1);
+        const float p0 = fast_exp2(L[u][0]), p1 = fast_exp2(L[u][1]);
+        const float p2 = fast_exp2(L[u][2]), p3 = fast_exp2(L[u][3]);
         st.l0 += p0 + p2;
         st.l1 += p1 + p3;
         // masked tokens carry |v| = +0 (set by the caller)
@@ -1674,7 +1725,7 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
         const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
                                              (size_t)a.tile_bytes;
         SplitState<D> st;
-        st.m0 = st.m1 = -CUDART_INF_F;
+        st.m0 = st.m1 = 0.f;   // set by the warp's first pair (see pair_accumulate)
         st.l0 = st.l1 = 0.f;
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
@@ -1728,7 +1779,7 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
                 td[uu].vn = *reinterpret_cast<const uint32_t*>(tp + Tr::CODE_BYTES + Tr::KNB + 4 * g);
             }
             float L[2][4];
-            pair_logits<D, KB, VB, QJ>(td, qf, lane, lutk, lane4, L);
+            pair_logits<D, KB, VB, QJ>(td, qf, lane, lutk, lane4, make_float2(-st.m0, -st.m1), L);
             // Tokens at or past seq_len (only in a unit's last pair, or a missing
             // second tile): logit -inf and value norm +0. Their slots may hold
             // anything, NaN norms included: select, never multiply.
@@ -1750,7 +1801,7 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
 #pragma unroll
             for (int uu = 0; uu < 2; ++uu)
                 stage_words<CB, P2::VW0, P2::VWN, Tr::NWORDS>(sp + uu * TB, lane, td[uu].s);
-            pair_accumulate<D, KB, VB, QJ>(td, L, lane4v, st);
+            pair_accumulate<D, KB, VB, QJ>(td, L, lane4v, st, p == w);
         }
 
         float l0 = st.l0, l1 = st.l1;
@@ -1763,9 +1814,10 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
         __syncthreads();   // every warp is done with its ring: reuse the upper rings for the merge
         float* mw = mrg + (size_t)w * 8 * RS;
         if (g == 0) {
-            mw[(2 * t) * RS] = st.m0;
+            const bool idle = w >= npair;   // no pair: no reference, the merge skips it
+            mw[(2 * t) * RS] = idle ? -CUDART_INF_F : st.m0;
             mw[(2 * t) * RS + 1] = l0;
-            mw[(2 * t + 1) * RS] = st.m1;
+            mw[(2 * t + 1) * RS] = idle ? -CUDART_INF_F : st.m1;
             mw[(2 * t + 1) * RS + 1] = l1;
         }
 #pragma unroll
@@ -1803,6 +1855,8 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
         ++consumed;
     }
 }
+
+#include "attend_cc.cuh"
 
 // cudaFuncSetAttribute once per (kernel, device).
 template <typename K>
@@ -1861,6 +1915,21 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
         if (a.plan.tiles > 0)
             e = launch_pdl(kern, dim3(a.plan.nsplit, units, a.B), dim3(Tr::NT), Tr::DYN_SMEM, st, tb, a);
         return e;
+    }
+    if (a.cc_mode != 0) {
+        if constexpr (D == CcTraits::D && KB == CcTraits::KB && VB == CcTraits::VB && QJ == CcTraits::QJ) {
+            static unsigned long long done_cc1 = 0, done_cc2 = 0;
+            auto kern = a.cc_mode == 2 ? attend_cc<2> : attend_cc<1>;
+            if ((e = allow_smem(kern, CcTraits::SMEM, a.cc_mode == 2 ? done_cc2 : done_cc1)) != cudaSuccess)
+                return e;
+            if (a.plan.tiles > 0 &&
+                (e = launch_pdl(kern, dim3(a.plan.ctas), dim3(CcTraits::NT), CcTraits::SMEM, st, tb, a)) !=
+                    cudaSuccess)
+                return e;
+            return launch_pdl(attend_reduce<D>, dim3(a.Hq, a.B), dim3(D), 0, st, tb, a);
+        } else {
+            return cudaErrorNotSupported;
+        }
     }
     if constexpr (PairTraits<D, KB, VB, QJ>::SUPPORTED) {
         using P2 = PairTraits<D, KB, VB, QJ>;

@@ -50,6 +50,9 @@ struct AttendArgs {
     const int32_t* start_pos; // [B]
     int T;
     uint8_t* cache_w;         // the cache, writable
+    // tq_attend_cudacore: 1 or 2 runs the CUDA-core split kernel (QJL term by
+    // sign-nibble tables or by bit-plane popcounts) in place of the tensor-core one
+    int cc_mode;
 };
 
 cudaError_t launch_quantize(const Format& f, const DevTables& tb, const QuantizeArgs& a,
