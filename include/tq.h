@@ -113,7 +113,11 @@ typedef struct {
  *    Format (3, 4, 1) (TurboQuant at 4 bits) instead keeps each key pair and
  *    two sign bits in one byte: the K code at 8p + 3e (bits 0..5 of byte p),
  *    the sign at 32*(p/4) + 16e + a, a = 6, 7, 14, 15 for p%4 = 0, 1, 2, 3
- *    (bits 6 and 7 of the bytes of word p/4); its V codes as above. With
+ *    (bits 6 and 7 of the bytes of word p/4); its V codes as above.
+ *    Format (2, 3, 1) (TurboQuant at 3 bits) keeps each value pair and two
+ *    sign bits in one byte instead: the K codes as above (the first B_K*d/2
+ *    bits), then the V code at B_K*d/2 + 8p + 3e (bits 0..5 of byte p of that
+ *    region) and the sign at B_K*d/2 + 32*(p/4) + 16e + a, a as above. With
  *    4-bit value cells every V pair is one byte, and with (4, 4, 0) every K
  *    pair too: the decoder turns such a byte into its table row with one
  *    byte permute.

@@ -62,8 +62,10 @@ struct AttTraits {
     static constexpr int CB = SBYTES % 16 == 0 ? 16 : SBYTES % 8 == 0 ? 8 : 4;
     static constexpr int NCH = SBYTES / CB;                  // chunks of a lane string
     static constexpr int NWORDS = SBYTES / 4;
-    static constexpr int SBW = BK * D / 64;                  // first sign word
-    static constexpr int VBIT0 = (BK + QJ) * D / 2;          // first value bit
+    static constexpr int SBW = BK * D / 64;                  // first sign word (generic layout)
+    static constexpr int VBIT0 = TileLayout<D, KB, VB, QJ>::VB0;   // first value bit
+    // value pairs with two sign bits a byte ((2, 3, 1)): the QJL operands come from the value words
+    static constexpr bool VSB = TileLayout<D, KB, VB, QJ>::VS_BYTES;
     static constexpr int KK = D / 16;                        // k-steps / coordinate blocks
     static constexpr int NLK = 1 << KF, NLV = 1 << VF;       // LUT entries
     static constexpr int CODE_BYTES = 2 * W * D;             // code region of a tile
@@ -84,6 +86,9 @@ struct AttTraits {
     static constexpr bool ROWS = PV;
     static constexpr int LSH = ROWS ? 8 : 7;                 // log2 of a table entry's stride
     static constexpr int VW0 = VBIT0 / 32;                   // first value word (byte fields)
+    // first lane-string word of the QJL sign operands: the key words (3-bit keys),
+    // the value words ((2, 3, 1)), else the sign words
+    static constexpr int QW0 = TileLayout<D, KB, VB, QJ>::KS_BYTES ? 0 : VSB ? VW0 : SBW;
     static_assert(!PK || ROWS, "byte-field keys come with byte-field values");
     static_assert(!CK || (ROWS && KB <= 7), "per-code keys use the row table (up to 128 codes)");
     static_assert(!PV || VBIT0 % 32 == 0, "byte-field values start on a word");
@@ -196,10 +201,12 @@ __device__ __forceinline__ uint32_t lut_load(const uint32_t* table, uint32_t x)
 //     sum_i (2 s_i - 1) x_i = u (2 acc / sigma - T) + (rounding of x, <= u/2 a term).
 // Sign layouts (SL): 0 none (no QJL), 1 sign words (two bits a key pair at bits
 // q and q + 16 of the pair's sign word), 2 byte fields (the two top bits of each
-// key byte: token g at bit 6, token g + 8 at bit 7).
-template <int KB, int QJ>
+// key byte, or of each value byte for (2, 3, 1): token g at bit 6, token g + 8
+// at bit 7).
+template <int KB, int VB, int QJ>
 struct SignLayout {
-    static constexpr int SL = QJ == 0 ? 0 : (TileLayout<64, KB, 1, QJ>::KS_BYTES ? 2 : 1);
+    static constexpr int SL =
+        QJ == 0 ? 0 : (TileLayout<64, KB, VB, QJ>::KS_BYTES || TileLayout<64, KB, VB, QJ>::VS_BYTES ? 2 : 1);
 };
 
 // The coordinate held by byte i (0..3) of the B register `half` (0: b0, 1: b1)
@@ -223,17 +230,18 @@ struct QjlSigma {
 };
 
 // A registers of int8 k-step J: a0, a2 token g, a1, a3 token g + 8 (bytes 0 / sigma).
-template <int SL, int SBW>
+// QW0: the first lane-string word holding the signs.
+template <int SL, int QW0>
 __device__ __forceinline__ void qjl_a(const uint32_t* s, int J, uint32_t (&a)[4])
 {
     if constexpr (SL == 2) {
-        const uint32_t w0 = s[2 * J], w1 = s[2 * J + 1];
+        const uint32_t w0 = s[QW0 + 2 * J], w1 = s[QW0 + 2 * J + 1];
         a[0] = w0 & 0x40404040u;
         a[1] = w0 & 0x80808080u;
         a[2] = w1 & 0x40404040u;
         a[3] = w1 & 0x80808080u;
     } else {
-        const uint32_t w = s[SBW + (J >> 1)] >> (4 * (J & 1));
+        const uint32_t w = s[QW0 + (J >> 1)] >> (4 * (J & 1));
         a[0] = w & 0x01010101u;
         a[1] = (w >> 1) & 0x01010101u;
         a[2] = (w >> 2) & 0x01010101u;
@@ -684,7 +692,7 @@ __global__ void __launch_bounds__(2 * D) append_prologue(DevTables tb, AttendArg
     if ((int)blockIdx.x >= units)
         append_tokens<D, KB, VB, QJ>(tb, a, blockIdx.y, blockIdx.x - units, reinterpret_cast<uint8_t*>(app_smem));
     else
-        prologue_body<D, SignLayout<KB, QJ>::SL>(tb, a);
+        prologue_body<D, SignLayout<KB, VB, QJ>::SL>(tb, a);
 }
 
 
@@ -990,7 +998,7 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
                                             const uint32_t* lutk, uint32_t lane4, float (&L)[4])
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    constexpr int SL = SignLayout<KB, QJ>::SL;
+    constexpr int SL = SignLayout<KB, VB, QJ>::SL;
     // codebook term: two fp32 chains, the hi and lo parts of the B operands;
     // QJL term: two int8 chains, the high and low bytes of its B operands
     float ah[4], al[4];
@@ -1029,7 +1037,7 @@ __device__ __forceinline__ void tile_logits(const TileData<D, KB, VB, QJ>& td, c
                 const int J = kk >> 1;
                 const uint4 bs = qf.fs(J, lane);
                 uint32_t as[4];
-                qjl_a<SL, Tr::SBW>(td.s, J, as);
+                qjl_a<SL, Tr::QW0>(td.s, J, as);
                 imma_16832<true>(ih, as[0], as[1], as[2], as[3], bs.x, bs.y);
                 imma_16832<false>(il, as[0], as[1], as[2], as[3], bs.z, bs.w);
             }
@@ -1093,7 +1101,7 @@ __device__ __forceinline__ void tile_accumulate(const TileData<D, KB, VB, QJ>& t
 #pragma unroll
         for (int r = 0; r < 4; ++r)
             av[r] = Tr::PV ? lut_load<Tr::ALIGNED>(lutv, row_off(td.s[Tr::VW0 + kk], r, lane4))
-                           : lut_load<Tr::ALIGNED>(lutv, lut_off<Tr::LSH>(td.s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
+                           : lut_load<Tr::ALIGNED>(lutv, lut_off<Tr::LSH>(td.s, TileLayout<D, KB, VB, QJ>::vbit(4 * kk + r, 0),
                                                                           Tr::VF, lane4));
         mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0, b1);
     }
@@ -1450,7 +1458,9 @@ struct PairTraits {
     static_assert(Tr::ROWS || ((size_t)Tr::NLK * 128 <= 0x8000 && (size_t)Tr::NLV * 128 <= 0x8000),
                   "small tables fit their 32 KB halves");
     // lane-string words holding the key operands (codes and, byte-field keys, signs) and the values
-    static constexpr int KW0 = 0, KWN = Tr::PK ? Tr::KK : Tr::VW0;
+    // (2, 3, 1): the logits' QJL operands sit in the value words, so every word is
+    // staged before the logits
+    static constexpr int KW0 = 0, KWN = Tr::PK ? Tr::KK : Tr::VSB ? Tr::NWORDS : Tr::VW0;
     static constexpr int VW0 = Tr::VW0, VWN = Tr::NWORDS - Tr::VW0;
 };
 
@@ -1485,7 +1495,7 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
                                             const uint32_t* lutk, uint32_t lane4, float2 nm, float (&L)[2][4])
 {
     using Tr = AttTraits<D, KB, VB, QJ>;
-    constexpr int SL = SignLayout<KB, QJ>::SL;
+    constexpr int SL = SignLayout<KB, VB, QJ>::SL;
     // Codebook term: the hi and lo B parts in two accumulator chains, or, for
     // byte-field keys, in one. (Measured at (3, 4, 1), d = 128: one chain alone
     // gained nothing, the lazy rescale with offset logits alone nothing, both
@@ -1535,7 +1545,7 @@ __device__ __forceinline__ void pair_logits(const TileData<D, KB, VB, QJ> (&td)[
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     uint32_t as[4];
-                    qjl_a<SL, Tr::SBW>(td[u].s, J, as);
+                    qjl_a<SL, Tr::QW0>(td[u].s, J, as);
                     imma_16832<true>(ih[u], as[0], as[1], as[2], as[3], bs.x, bs.y);
                     imma_16832<false>(il[u], as[0], as[1], as[2], as[3], bs.z, bs.w);
                 }
@@ -1621,8 +1631,9 @@ __device__ __forceinline__ void pair_accumulate(const TileData<D, KB, VB, QJ> (&
                 constexpr int VSH = PairTraits<D, KB, VB, QJ>::WK ? 8 : Tr::LSH;   // row stride
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
-                    av[r] = Tr::PV ? lut_load<true>(nullptr, row_off(td[u].s[Tr::VW0 + kk], r, lane4v))
-                                   : lut_load<true>(nullptr, lut_off<VSH>(td[u].s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
+                    av[r] = (Tr::PV || Tr::VSB)
+                                ? lut_load<true>(nullptr, row_off(td[u].s[Tr::VW0 + kk], r, lane4v))
+                                : lut_load<true>(nullptr, lut_off<VSH>(td[u].s, Tr::VBIT0 + Tr::VF * (4 * kk + r),
                                                                           Tr::VF, lane4v));
             }
             mma_16816(st.acc[kk], av[0], av[1], av[2], av[3], b0[u], b1[u]);
@@ -1664,6 +1675,8 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
                 v = __ldg(tb.lut_k + ((x >> (FK * i)) & ((1 << FK) - 1)));
             } else if constexpr (P2::WV) {
                 v = __ldg(tb.lut_v + ((x >> (4 * (col & 1))) & 15));
+            } else if constexpr (Tr::VSB) {
+                v = __ldg(tb.lut_v + (x & (Tr::NLV - 1)));   // value pair in bits 0..5, signs above
             } else {
                 v = x < Tr::NLV ? __ldg(tb.lut_v + x) : 0u;
             }
@@ -1798,9 +1811,11 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
                     }
                 }
             }
+            if constexpr (!Tr::VSB) {
 #pragma unroll
-            for (int uu = 0; uu < 2; ++uu)
-                stage_words<CB, P2::VW0, P2::VWN, Tr::NWORDS>(sp + uu * TB, lane, td[uu].s);
+                for (int uu = 0; uu < 2; ++uu)
+                    stage_words<CB, P2::VW0, P2::VWN, Tr::NWORDS>(sp + uu * TB, lane, td[uu].s);
+            }
             pair_accumulate<D, KB, VB, QJ>(td, L, lane4v, st, p == w);
         }
 
@@ -1906,7 +1921,7 @@ cudaError_t launch_attend_t(const DevTables& tb, const AttendArgs& a, bool score
         if ((e = allow_smem(kern, smem, done_append)) != cudaSuccess) return e;
         e = launch_pdl(kern, dim3(units + a.Hkv, a.B), dim3(2 * D), smem, st, tb, a);
     } else {
-        e = launch_pdl(attend_prologue<D, SignLayout<KB, QJ>::SL>, dim3(units, a.B), dim3(2 * D), 0, st, tb, a);
+        e = launch_pdl(attend_prologue<D, SignLayout<KB, VB, QJ>::SL>, dim3(units, a.B), dim3(2 * D), 0, st, tb, a);
     }
     if (e != cudaSuccess) return e;
     if (scores) {

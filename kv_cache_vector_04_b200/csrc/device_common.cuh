@@ -21,23 +21,30 @@ constexpr unsigned kFull = 0xffffffffu;
 // one byte each: key pair p in the low 6 bits of byte p, the sign pairs of
 // word w at bits a and a + 16 for a = 6, 7, 14, 15 (pairs 4w .. 4w + 3), so
 // the decoder finds a key pair's table row with one byte permute and a sign
-// pair with one shift. With 4-bit cells the generic layout is byte-aligned
+// pair with one shift. With 2-bit keys, 3-bit values and QJL ((2, 3, 1)) a
+// value pair and two signs fill one byte each the same way, in the region
+// after the key codes. With 4-bit cells the generic layout is byte-aligned
 // already.
 template <int D, int KB, int VB, int QJ>
 struct TileLayout {
     static constexpr bool KS_BYTES = QJ == 1 && KB == 3;
+    static constexpr bool VS_BYTES = QJ == 1 && KB == 2 && VB == 3;
     static constexpr int SB0 = KB * D / 2;                   // first sign bit (generic)
-    static constexpr int VB0 = (KB + QJ) * D / 2;            // first value bit
+    static constexpr int VB0 = VS_BYTES ? KB * D / 2 : (KB + QJ) * D / 2;   // first value bit
     __host__ __device__ static constexpr int kbit(int p, int e)
     {
         return (KS_BYTES ? 8 : 2 * KB) * p + e * KB;
     }
     __host__ __device__ static constexpr int sbit(int p, int e)
     {
-        return KS_BYTES ? 32 * (p >> 2) + 16 * e + 6 + (p & 1) + 8 * ((p >> 1) & 1)
-                        : SB0 + 32 * (p >> 4) + 16 * e + (p & 15);
+        return KS_BYTES   ? 32 * (p >> 2) + 16 * e + 6 + (p & 1) + 8 * ((p >> 1) & 1)
+               : VS_BYTES ? VB0 + 32 * (p >> 2) + 16 * e + 6 + (p & 1) + 8 * ((p >> 1) & 1)
+                          : SB0 + 32 * (p >> 4) + 16 * e + (p & 15);
     }
-    __host__ __device__ static constexpr int vbit(int p, int e) { return VB0 + 2 * VB * p + e * VB; }
+    __host__ __device__ static constexpr int vbit(int p, int e)
+    {
+        return VS_BYTES ? VB0 + 8 * p + 3 * e : VB0 + 2 * VB * p + e * VB;
+    }
 };
 
 // Device copies of one context's tables (all pointers into one allocation).

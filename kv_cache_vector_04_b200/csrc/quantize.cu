@@ -41,7 +41,10 @@ struct QuantTraits {
     static constexpr int CW = CB / 4;                  // words per chunk
     static constexpr int KF = 2 * BK, VF = 2 * BV;     // field widths (two codes each)
     static constexpr int SBW = BK * D / 64;            // first sign word of a lane string
-    static constexpr int VBW = (BK + QJ) * D / 64;     // first value word
+    // (2, 3, 1) keeps each value pair and two signs in one byte: no sign words,
+    // the value words start after the key codes
+    static constexpr bool VSB = TileLayout<D, KB, VB, QJ>::VS_BYTES;
+    static constexpr int VBW = VSB ? SBW : (BK + QJ) * D / 64;   // first value word
     static constexpr int CODE_BYTES = 2 * W * D;       // code region of a tile
     static constexpr int KNB = 32 + 32 * QJ;           // K norm bytes of a tile
     static constexpr int NT = M / 8;                   // n-tiles of z = S r
@@ -340,6 +343,26 @@ __global__ void __launch_bounds__(128) quantize_kernel(DevTables tb, QuantizeArg
                         const uint32_t bits = (sg[tok][row >> 5] >> (row & 31)) & 3u;
                         val |= ((bits & 1u) << q2) | ((bits >> 1) << (16 + q2));
                         if (is_new(tok)) msk |= (1u << q2) | (1u << (16 + q2));
+                    }
+                } else if (Tr::VSB) {                     // value pairs 4 kk + j with the signs of the same pairs
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        using Lay = TileLayout<D, BK, BV, QJ>;
+                        const int kk = wi - Tr::VBW, p = 4 * kk + j;
+                        const int tok0 = 2 * tL + 8 * (j >> 1);
+                        const int coord = 16 * kk + gL + 8 * (j & 1);
+                        const uint32_t f = ((uint32_t)vc[tok0][coord] & 7u) | (((uint32_t)vc[tok0 + 1][coord] & 7u) << 3);
+                        const uint32_t fm = (is_new(tok0) ? 0x07u : 0u) | (is_new(tok0 + 1) ? 0x38u : 0u);
+                        const int o = Lay::vbit(p, 0) - 32 * wi;
+                        val |= f << o;
+                        msk |= fm << o;
+                        // the signs of pair p: key token gL + 8 (j & 1), rows 16 kk + 8 (j >> 1) + 2 tL + {0, 1}
+                        const int tok = gL + 8 * (j & 1);
+                        const int row = 16 * kk + 8 * (j >> 1) + 2 * tL;
+                        const uint32_t bits = (sg[tok][row >> 5] >> (row & 31)) & 3u;
+                        const int a0 = Lay::sbit(p, 0) - 32 * wi, a1 = Lay::sbit(p, 1) - 32 * wi;
+                        val |= ((bits & 1u) << a0) | ((bits >> 1) << a1);
+                        if (is_new(tok)) msk |= (1u << a0) | (1u << a1);
                     }
                 } else if (Tr::VF == 8) {                 // 4-bit value pairs, one byte each
 #pragma unroll

@@ -257,14 +257,16 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
     if constexpr (QJ) {
         // source bit 4 hs + 2 rw + e (n-tile 2 kk + hs, element 2 rw + e) is the sign
         // of pair 4 kk + 2 hs + rw, element e: byte fields put it at bit
-        // 6 + rw + 8 hs + 16 e of word kk, sign words at 16 e + 2 hs + rw (+ 4 (kk & 3))
+        // 6 + rw + 8 hs + 16 e of word kk (of the key words for (3, 4, 1), of the
+        // value words for (2, 3, 1)), sign words at 16 e + 2 hs + rw (+ 4 (kk & 3))
         for (int x = tid; x < 256; x += 128) {
             uint32_t v = 0u;
 #pragma unroll
             for (int bsrc = 0; bsrc < 8; ++bsrc) {
                 if (!((x >> bsrc) & 1)) continue;
                 const int hs = bsrc >> 2, rw = (bsrc >> 1) & 1, e = bsrc & 1;
-                v |= 1u << (TileLayout<D, KB, VB, QJ>::KS_BYTES ? 6 + rw + 8 * hs + 16 * e : 16 * e + 2 * hs + rw);
+                using L = TileLayout<D, KB, VB, QJ>;
+                v |= 1u << (L::KS_BYTES || L::VS_BYTES ? 6 + rw + 8 * hs + 16 * e : 16 * e + 2 * hs + rw);
             }
             sm.sgt[x] = v;
         }
@@ -603,6 +605,8 @@ __global__ void __launch_bounds__(128) quantize_fast(DevTables tb, QuantizeArgs 
             const uint32_t m = sm.sgt[sb];
             if constexpr (LayT::KS_BYTES)
                 s[kk] |= m;
+            else if constexpr (LayT::VS_BYTES)
+                s[LayT::VB0 / 32 + kk] |= m;
             else
                 s[LayT::SB0 / 32 + (kk >> 2)] |= m << (4 * (kk & 3));
         }

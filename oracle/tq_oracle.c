@@ -515,6 +515,10 @@ void oracle_quantize_values(int d, int N, const uint16_t* x, const int8_t* D,
 /* code at bit 8p + 3e (the low 6 bits of byte p), the sign at bit            */
 /* 32*(p/4) + 16e + a with a = 6, 7, 14, 15 for p%4 = 0, 1, 2, 3 (the top     */
 /* two bits of the bytes of word p/4); the V codes as above.                  */
+/* And except for (2, 3, 1), whose value pair and two signs share a byte: the */
+/* K codes as above (the first B_K*d/2 bits), then the V code at bit          */
+/* B_K*d/2 + 8p + 3e (the low 6 bits of byte p of that region) and the sign   */
+/* at bit B_K*d/2 + 32*(p/4) + 16e + a, a as above.                           */
 /* The TurboQuant format at b bits is (b-1, b, 1): tiles of 16*(b*d/4 + 6).   */
 /* ------------------------------------------------------------------------- */
 
@@ -556,8 +560,9 @@ static unsigned get_bits(const uint8_t* tile, int C, int lane, int64_t bit, int 
 }
 
 /* Whether format (kb, vb, qjl) keeps each key pair and two sign bits in one
- * byte. */
+ * byte; whether it keeps each value pair and two sign bits in one byte. */
 static int key_sign_bytes(int kb, int qjl) { return qjl == 1 && kb == 3; }
+static int value_sign_bytes(int kb, int vb, int qjl) { return qjl == 1 && kb == 2 && vb == 3; }
 
 /* Lane-string bit of key code (p, e). */
 static int64_t key_bit(int kb, int qjl, int p, int e)
@@ -569,11 +574,21 @@ static int64_t key_bit(int kb, int qjl, int p, int e)
 /* Lane-string bit of sign (p, e). Generic layout: sign pair p of a lane has
  * element 0 at bit p%16, element 1 at bit 16 + p%16 of the lane's sign word
  * p/16, after the key codes (sign words start at bit kb*d/2). */
-static int64_t sign_bit(int d, int kb, int qjl, int p, int e)
+static int64_t sign_bit(int d, int kb, int vb, int qjl, int p, int e)
 {
     static const int top[4] = {6, 7, 14, 15};
     if (key_sign_bytes(kb, qjl)) return 32LL * (p / 4) + 16 * e + top[p % 4];
+    if (value_sign_bytes(kb, vb, qjl)) return (int64_t)kb * d / 2 + 32LL * (p / 4) + 16 * e + top[p % 4];
     return (int64_t)kb * d / 2 + 32LL * (p / 16) + 16 * e + (p % 16);
+}
+
+/* Lane-string bit of value code (p, e): after the key codes and sign words,
+ * two vb-bit fields a pair; for (2, 3, 1) byte p of the region after the key
+ * codes, element e at bit 3e. */
+static int64_t value_bit(int d, int kb, int vb, int qjl, int p, int e)
+{
+    if (value_sign_bytes(kb, vb, qjl)) return (int64_t)kb * d / 2 + 8LL * p + 3 * e;
+    return (int64_t)(kb + qjl) * d / 2 + 2LL * vb * p + (int64_t)e * vb;
 }
 
 static void put_half(uint8_t* p, uint16_t h) { p[0] = (uint8_t)(h & 0xff); p[1] = (uint8_t)(h >> 8); }
@@ -605,7 +620,6 @@ void oracle_pack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* ki
     int64_t TB = oracle_tile_bytes(d, kb, vb, qjl);
     int ntiles = (N + TQO_TILE - 1) / TQO_TILE;
     memset(out, 0, (size_t)(TB * ntiles));
-    int64_t vbase = (int64_t)(kb + qjl) * d / 2;
     for (int tl = 0; tl < ntiles; ++tl) {
         uint8_t* tile = out + TB * tl;
         for (int lane = 0; lane < 32; ++lane) {
@@ -620,11 +634,11 @@ void oracle_pack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* ki
                     if (nk < N) {
                         put_bits(tile, C, lane, key_bit(kb, qjl, p, e), kb, kidx[(size_t)nk * d + ik]);
                         if (qjl)
-                            put_bits(tile, C, lane, sign_bit(d, kb, qjl, p, e), 1,
+                            put_bits(tile, C, lane, sign_bit(d, kb, vb, qjl, p, e), 1,
                                      ksign[(size_t)nk * m + ik]);
                     }
                     if (nv < N)
-                        put_bits(tile, C, lane, vbase + 2LL * vb * p + e * vb, vb,
+                        put_bits(tile, C, lane, value_bit(d, kb, vb, qjl, p, e), vb,
                                  vidx[(size_t)nv * d + iv]);
                 }
             }
@@ -650,7 +664,6 @@ void oracle_unpack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* 
     int m = d, C = chunk_bytes(d, kb, vb, qjl);
     int64_t TB = oracle_tile_bytes(d, kb, vb, qjl);
     int ntiles = (N + TQO_TILE - 1) / TQO_TILE;
-    int64_t vbase = (int64_t)(kb + qjl) * d / 2;
     for (int tl = 0; tl < ntiles; ++tl) {
         const uint8_t* tile = in + TB * tl;
         for (int lane = 0; lane < 32; ++lane) {
@@ -666,11 +679,11 @@ void oracle_unpack_stream(int d, int kb, int vb, int qjl, int N, const uint8_t* 
                         kidx[(size_t)nk * d + ik] =
                             (uint8_t)get_bits(tile, C, lane, key_bit(kb, qjl, p, e), kb);
                         ksign[(size_t)nk * m + ik] =
-                            (uint8_t)(qjl ? get_bits(tile, C, lane, sign_bit(d, kb, qjl, p, e), 1) : 0);
+                            (uint8_t)(qjl ? get_bits(tile, C, lane, sign_bit(d, kb, vb, qjl, p, e), 1) : 0);
                     }
                     if (nv < N)
                         vidx[(size_t)nv * d + iv] =
-                            (uint8_t)get_bits(tile, C, lane, vbase + 2LL * vb * p + e * vb, vb);
+                            (uint8_t)get_bits(tile, C, lane, value_bit(d, kb, vb, qjl, p, e), vb);
                 }
             }
         }

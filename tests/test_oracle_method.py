@@ -369,3 +369,45 @@ def test_attend_batch_matches_per_head():
             o, l1 = O.attend_head(tab, qbits[b, h], True, s, int(seq[b]))
             assert np.array_equal(out[b, h], o)
             assert np.array_equal(lg[b, h, :seq[b]], l1)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_pack_value_sign_bytes_of_3bit_values(d):
+    # Format (2, 3, 1) (TurboQuant at 3 bits) keeps each value pair with two
+    # sign bits in one byte of the region after the key codes: every value code
+    # lies in bits 0..5 of a byte there, every sign in bit 6 or 7 of a byte
+    # there, the two signs of a sign pair sit 16 bits apart in one 32-bit word,
+    # and the key codes keep the first 2*d/2 bits of each lane string.
+    fmt, N = (2, 3, 1), 16
+    zero = dict(kidx=np.zeros((N, d), np.uint8), ksign=np.zeros((N, d), np.uint8),
+                knorm=np.zeros(N, np.uint16), rnorm=np.zeros(N, np.uint16),
+                vidx=np.zeros((N, d), np.uint8), vnorm=np.zeros(N, np.uint16))
+    C = 16 if (6 * d // 16) % 16 == 0 else 8   # chunk bytes of a lane string of 6d/16 bytes
+    key_bytes = 2 * d // 2 // 8                # key codes: the first kb*d/2 bits of a lane string
+
+    def lane_pos(bit_in_tile):
+        byte = bit_in_tile // 8
+        chunk, lane, off = byte // (32 * C), (byte // C) % 32, byte % C
+        return lane, (chunk * C + off) * 8 + bit_in_tile % 8
+
+    for n in (0, 5, 8, 15):
+        for i in range(0, d, 3):
+            c = {k: v.copy() for k, v in zero.items()}
+            c["vidx"][n, i] = 7
+            bits = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+            assert bits.size == 3 and len({b // 8 for b in bits}) == 1
+            lane, pos = lane_pos(bits[0])
+            assert all(lane_pos(b)[1] % 8 <= 5 for b in bits) and pos // 8 >= key_bytes
+            c = {k: v.copy() for k, v in zero.items()}
+            c["kidx"][n, i] = 3
+            kbits = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+            assert kbits.size == 2 and all(lane_pos(b)[1] // 8 < key_bytes for b in kbits)
+            c = {k: v.copy() for k, v in zero.items()}
+            c["ksign"][n, i] = 1
+            sb = np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))
+            li, bi = lane_pos(sb[0])
+            assert sb.size == 1 and bi % 8 in (6, 7) and bi // 8 >= key_bytes
+            c["ksign"][n, i] = 0
+            c["ksign"][n, i ^ 1] = 1
+            lj, bj = lane_pos(np.flatnonzero(np.unpackbits(O.pack_stream(d, fmt, c), bitorder="little"))[0])
+            assert li == lj and abs(bi - bj) == 16 and bi // 32 == bj // 32
