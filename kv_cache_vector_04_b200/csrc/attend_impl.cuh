@@ -33,6 +33,7 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <type_traits>
 #include <utility>
 
 #include "device_common.cuh"
@@ -924,6 +925,34 @@ struct QueryFrags {
     }
 };
 
+// The same fragments held in registers for a whole segment (loaded from the
+// workspace, where the prologue wrote them): no shared-memory reads per tile,
+// for 4 (KK + KK/2 + 2) registers a thread.
+template <int KK, int QJ>
+struct QueryFragsReg {
+    uint4 c[KK];
+    uint4 s[QJ ? KK / 2 : 1];
+    float4 a;
+    float2 bq;
+    __device__ __forceinline__ void load(const uint4* src, int lane)
+    {
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) c[kk] = __ldg(src + kk * 64 + lane);
+        if constexpr (QJ) {
+#pragma unroll
+            for (int J = 0; J < KK / 2; ++J) s[J] = __ldg(src + J * 64 + 32 + lane);
+            const uint4 va = __ldg(src + (KK / 2) * 64 + 32 + lane);
+            const uint4 vb = __ldg(src + (KK / 2 + 1) * 64 + 32 + lane);
+            a = make_float4(__uint_as_float(va.x), __uint_as_float(va.y), __uint_as_float(va.z), __uint_as_float(va.w));
+            bq = make_float2(__uint_as_float(vb.x), __uint_as_float(vb.y));
+        }
+    }
+    __device__ __forceinline__ uint4 fc(int kk, int) const { return c[kk]; }
+    __device__ __forceinline__ uint4 fs(int J, int) const { return s[J]; }
+    __device__ __forceinline__ float4 qa(int) const { return a; }
+    __device__ __forceinline__ float2 qb(int) const { return bq; }
+};
+
 // Logits (log2 units) of tokens g, g + 8 and heads 2t, 2t + 1 from the
 // codebook sums (two fp32 chains: the hi and lo parts of the B operands) and the
 // QJL integer sums (high, low byte chains): L = |k| (c + rho (acc u 2/sigma - u T)).
@@ -1430,10 +1459,19 @@ template <int D, int KB, int VB, int QJ>
 struct PairTraits {
     using Tr = AttTraits<D, KB, VB, QJ>;
     static constexpr uint32_t LUT_ADDR = 0x10000u;
-    static constexpr int WARPS = 16, NT = 32 * WARPS;
+    // Query fragments in registers (12 warps of up to 168 registers) or read from
+    // shared memory for every pair (16 warps of 128 registers). Measured (per
+    // layer, 65K context, batch 8): registers win at d = 128 for (1, 2, 1)
+    // (139 against 147 us) and (2, 3, 1) (equal; the Qwen2.5-32B-shaped 128K layer
+    // 55.7 against 56.8 us), lose for (3, 4, 1) (151.4 against 148.5 us at the 70B
+    // shape, 107 against 101 us at d = 64): with a quarter fewer shared-memory
+    // wavefronts the kernel then waits on latency with three warps a scheduler.
+    static constexpr bool FREG = D == 128 && QJ == 1 && KB <= 2;
+    static constexpr int WARPS = FREG ? 12 : 16, NT = 32 * WARPS;
+    using QFrag = typename std::conditional<FREG, QueryFragsReg<D / 16, QJ>, QueryFrags<D / 16, NT>>::type;
     static constexpr int PSLOT = 2 * Tr::TILE_BYTES;      // one pair of tiles
     static constexpr int RPW = 2 * PSLOT;                 // ring of one warp: two pair slots
-    static constexpr size_t QF = Tr::QF_SMEM;
+    static constexpr size_t QF = FREG ? 0 : Tr::QF_SMEM;
     static constexpr int WA_FIT = (int)((LUT_ADDR - 4096 - QF) / RPW);
     static constexpr int WA = WA_FIT > WARPS ? WARPS : WA_FIT;   // rings below the table
     static constexpr size_t MERGE = (size_t)WARPS * 8 * (D + 2) * 4;
@@ -1710,7 +1748,7 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
     // slot n % 2 and completes phase (n / 2) & 1 of that slot's barrier.
     uint32_t issued = 0, consumed = 0;
     bool stalled = false;
-    QueryFrags<KK, NT> qf;
+    typename P2::QFrag qf;
 
     long long x = x0;
 #pragma unroll 1
@@ -1732,7 +1770,10 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
         const int seq = min(max(a.seq_len[b], 0), lim);
         const int hkv = j / groups;
         const size_t u = (size_t)b * upb + j;
-        qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
+        if constexpr (P2::FREG)
+            qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, lane);
+        else
+            qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
         __syncthreads();   // tables (first segment) and query fragments visible
 
         const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
