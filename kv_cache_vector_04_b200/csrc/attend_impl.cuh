@@ -311,6 +311,21 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
     const int groups = a.plan.groups, ratio = a.Hq / a.Hkv;
     const int hkv = unit / groups, grp = unit % groups;
     const size_t units = (size_t)a.Hkv * groups;
+    // The S^T fragments of this warp's two n-tiles (w, w + NT/32), requested
+    // before the rotation so that their latency overlaps it (d <= 128: at
+    // d = 256 they would take 64 registers, and are loaded where they are used).
+    constexpr int NTW = (D / 8) / (NT / 32);   // n-tiles per warp: 2
+    static_assert(NTW * (NT / 32) == D / 8, "every warp takes the same number of n-tiles");
+    constexpr bool PRE = SL != 0 && D <= 128;
+    uint2 bfs[PRE ? NTW : 1][D / 16];
+    if constexpr (PRE) {
+        const int w = tid >> 5, lane = tid & 31;
+#pragma unroll
+        for (int q = 0; q < NTW; ++q)
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                bfs[q][kk] = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + w + q * (NT / 32)) * 32 + lane);
+    }
     if (unit == 0 && b == 0 && tid < 32) tile_prefix(tb, a, tid);
 
     // One warp per head: lane l holds coordinates i = 32k + l (k < D/32), so the
@@ -375,13 +390,16 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
     {
         const int w = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
         const float sc = es[g];
-        for (int nt = w; nt < D / 8; nt += NT / 32) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            // all of this n-tile's S fragments first: one L2 round trip, not D/16
-            uint2 bfs[D / 16];
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-                bfs[kk] = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
+        for (int q = 0; q < NTW; ++q) {
+            const int nt = w + q * (NT / 32);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (!PRE) {
+                // all of this n-tile's S fragments first: one L2 round trip, not D/16
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    bfs[0][kk] = __ldg(tb.s_frag + ((size_t)kk * (D / 8) + nt) * 32 + lane);
+            }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const int c0 = 16 * kk + 2 * t;
@@ -389,7 +407,7 @@ __device__ __forceinline__ void prologue_body(const DevTables& tb, const AttendA
                 const float x2 = qt[c0 + 8][g] * sc, x3 = qt[c0 + 9][g] * sc;
                 const float h0 = __half2float(__float2half_rn(x0)), h1 = __half2float(__float2half_rn(x1));
                 const float h2 = __half2float(__float2half_rn(x2)), h3 = __half2float(__float2half_rn(x3));
-                const uint2 bf = bfs[kk];
+                const uint2 bf = bfs[PRE ? q : 0][kk];
                 mma_16816(acc, pack_half2(h0, h1), 0u, pack_half2(h2, h3), 0u, bf.x, bf.y);
                 mma_16816(acc, pack_half2(x0 - h0, x1 - h1), 0u, pack_half2(x2 - h2, x3 - h3), 0u,
                           bf.x, bf.y);
@@ -543,6 +561,18 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
     double* zp = rk + 16 * D;                                                // [16][M] half-sums of z
     const int t0 = start / 16, ntile = (start + T - 1) / 16 - t0 + 1;
     uint8_t* stream = a.cache_w + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity / 16) * TB;
+    // The decode step (T = 1): this thread's first batch of S^T entries for the
+    // QJL signs, requested now so that their latency overlaps the rotation.
+    constexpr int SB = 32;   // S entries per batch
+    constexpr bool PRE = QJ && D <= 128;   // at d = 256 the registers are short
+    float sv0[PRE ? SB : 1];
+    if constexpr (PRE) {
+        if (T == 1) {
+            const int j = tid % M, c0 = (tid / M) * (D / 2);
+#pragma unroll
+            for (int u = 0; u < SB; ++u) sv0[u] = __ldg(tb.s_t + (size_t)(c0 + u) * M + j);
+        }
+    }
     for (int e = tid; e < ntile * TB / 16; e += NT)
         reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(stream + (size_t)t0 * TB)[e];
     if (tid < (1 << BK)) tabs[tid] = tb.centroids_kd[tid];
@@ -630,14 +660,20 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
 #pragma unroll
         for (int i = 0; i < 16; ++i) z[i] = 0.0;
         if (T == 1) {   // the decode step: one key, four independent partial sums
-            // the loads of S in batches of 32, all in flight at once
-            constexpr int NB = 32;
+            // the loads of S in batches of SB, all in flight at once (the first
+            // batch was requested before the rotation)
+            constexpr int NB = SB;
             double z1 = 0.0, z2 = 0.0, z3 = 0.0;
 #pragma unroll 1
             for (int c0 = hf * (D / 2); c0 < (hf + 1) * (D / 2); c0 += NB) {
                 float sv[NB];
+                if (PRE && c0 == hf * (D / 2)) {
 #pragma unroll
-                for (int u = 0; u < NB; ++u) sv[u] = __ldg(tb.s_t + (size_t)(c0 + u) * M + j);
+                    for (int u = 0; u < NB; ++u) sv[u] = sv0[PRE ? u : 0];
+                } else {
+#pragma unroll
+                    for (int u = 0; u < NB; ++u) sv[u] = __ldg(tb.s_t + (size_t)(c0 + u) * M + j);
+                }
 #pragma unroll
                 for (int u = 0; u < NB; u += 4) {
                     z[0] = fma((double)sv[u], rk[c0 + u], z[0]);
