@@ -1806,21 +1806,12 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
         const int seq = min(max(a.seq_len[b], 0), lim);
         const int hkv = j / groups;
         const size_t u = (size_t)b * upb + j;
-        if constexpr (P2::FREG)
-            qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, lane);
-        else
-            qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
-        __syncthreads();   // tables (first segment) and query fragments visible
-
         const uint8_t* sbase = a.cache + ((size_t)b * a.Hkv + hkv) * (size_t)(a.capacity >> 4) *
                                              (size_t)a.tile_bytes;
-        SplitState<D> st;
-        st.m0 = st.m1 = 0.f;   // set by the warp's first pair (see pair_accumulate)
-        st.l0 = st.l1 = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
-
-        // pair p of the segment: tiles sb + 2p and sb + 2p + 1 (the last pair may hold one)
+        // pair p of the segment: tiles sb + 2p and sb + 2p + 1 (the last pair may hold one).
+        // The warp's first pair is requested before the query fragments are read,
+        // so that the two latencies overlap (the ring is apart from the fragment
+        // and table regions, and the previous segment's merge ended in a barrier).
         const int ntile = se - sb, npair = (ntile + 1) >> 1;
         fence_proxy_async();
         if (!stalled && w < npair) {
@@ -1832,6 +1823,17 @@ __global__ void __launch_bounds__(PairTraits<D, KB, VB, QJ>::NT, 1) attend_split
             }
             ++issued;
         }
+        if constexpr (P2::FREG)
+            qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, lane);
+        else
+            qf.load(reinterpret_cast<const uint4*>(a.qfrag) + u * KK * 64, qsm, tid);
+        __syncthreads();   // tables (first segment) and query fragments visible
+
+        SplitState<D> st;
+        st.m0 = st.m1 = 0.f;   // set by the warp's first pair (see pair_accumulate)
+        st.l0 = st.l1 = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KK; ++kk) st.acc[kk][0] = st.acc[kk][1] = st.acc[kk][2] = st.acc[kk][3] = 0.f;
         TileData<D, KB, VB, QJ> td[2];
 #pragma unroll 1
         for (int p = w; p < npair && !stalled; p += WARPS) {
