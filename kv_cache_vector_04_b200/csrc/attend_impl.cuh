@@ -573,6 +573,16 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
             for (int u = 0; u < SB; ++u) sv0[u] = __ldg(tb.s_t + (size_t)(c0 + u) * M + j);
         }
     }
+    // T = 1: warp 0 quantizes the new key, warp 1 the new value; their fp16
+    // coordinates are requested together with the tiles (d = 128: at d = 256
+    // the registers are short)
+    constexpr bool XPRE = D == 128;
+    __half2 xin[XPRE ? VPL / 2 : 1];
+    if (XPRE && T == 1 && w < 2) {
+        const __half* src = (w == 0 ? a.k_new : a.v_new) + ((size_t)b * a.Hkv + hkv) * (size_t)D + lane * VPL;
+#pragma unroll
+        for (int k = 0; k < VPL; k += 2) xin[k / 2] = *reinterpret_cast<const __half2*>(src + k);
+    }
     for (int e = tid; e < ntile * TB / 16; e += NT)
         reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(stream + (size_t)t0 * TB)[e];
     if (tid < (1 << BK)) tabs[tid] = tb.centroids_kd[tid];
@@ -593,7 +603,7 @@ __device__ __forceinline__ void append_tokens(const DevTables& tb, const AttendA
         double x[VPL];
 #pragma unroll
         for (int k = 0; k < VPL; k += 2) {
-            const __half2 p = *reinterpret_cast<const __half2*>(src + k);
+            const __half2 p = (XPRE && T == 1) ? xin[XPRE ? k / 2 : 0] : *reinterpret_cast<const __half2*>(src + k);
             x[k] = (double)__low2float(p);
             x[k + 1] = (double)__high2float(p);
         }
